@@ -1,0 +1,161 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) Multi-head Latent Attention hot path.
+ *
+ * What is computed (DeepSeek-V2, "DeepSeek-V2 summary" (7shi.hateblo.jp),
+ * App. C "Full Formulas of MLA" and §2.1.2-§2.1.3):
+ *
+ *   c^Q_t  = W_DQ h_t          q^C_t = W_UQ c^Q_t        q^R_t = RoPE(W_QR c^Q_t)
+ *   c^KV_t = W_DKV h_t         k^R_t = RoPE(W_KR h_t)   (shared by all heads)
+ *   o_{t,i} = sum_{j<=t} softmax_j([q^C;q^R]_{t,i} . [W_UK_i c^KV_j ; k^R_j] / sqrt(d_h+d_R)) W_UV_i c^KV_j
+ *   u_t    = W_O [o_{t,1}; ...; o_{t,n_h}]
+ *
+ * Only [c^KV_t | k^R_t] (d_c + d_R elements per token) is cached (App. C,
+ * the boxed vectors; §2.1.4).  Decode uses the absorbed form from the last
+ * paragraph of App. C: W_UK is folded into the query and W_UV is applied to
+ * the latent output, so per-head keys and values are never formed.  Prefill
+ * forms them once per token (the un-absorbed form) because there every key
+ * serves many queries.
+ *
+ * Conventions shared by every entry point
+ *  - Weights use the pages' shapes W in R^{out x in} (y = W x), row-major,
+ *    dtype `mla_dims.dtype`.  Head i owns rows [i d_h, (i+1) d_h) of W_UQ,
+ *    W_UK, W_UV, rows [i d_R, (i+1) d_R) of W_QR and columns
+ *    [i d_h, (i+1) d_h) of W_O.  Shapes: W_DQ [d_cq x d], W_UQ [n_h d_h x q_in],
+ *    W_QR [n_h d_R x q_in] with q_in = d_cq (or d when d_cq == 0), W_DKV
+ *    [d_c x d], W_KR [d_R x d], W_UK and W_UV [n_h d_h x d_c], W_O [d x n_h d_h].
+ *  - RoPE rotates interleaved pairs (2m, 2m+1) by pos * rope_base^(-2m/d_R);
+ *    pos is the token's 0-based index in its sequence.
+ *  - Cache row of a token: [c^KV (d_c) | RoPE'd k^R (d_R)], dtype
+ *    `mla_dims.dtype`, row stride (d_c + d_R) elements, contiguous per sequence:
+ *    token p of sequence s lives in row seq_start[s] + p.
+ *  - All pointers except the structs themselves are device pointers owned by
+ *    the caller.  The library allocates nothing and keeps no state between
+ *    calls (apart from the diagnostic timing hook at the end of this file).
+ *    Work is enqueued on `stream` and the calls return without synchronising.
+ *  - Every device pointer must be 16-byte aligned (TMA requirement).
+ *  - Errors in arguments, shapes, alignment or workspace size are found on the
+ *    host and returned before anything is enqueued.  Faults found on the
+ *    device (a position at or beyond `capacity`, a pipeline wait that timed
+ *    out) set a status word in the workspace; `mla_get_device_status` reads it.
+ */
+#ifndef MLA_B200_H
+#define MLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* mla_stream_t;   /* same type as cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = -1,   /* NULL pointer, non-positive size, inconsistent dims */
+    MLA_ERR_UNSUPPORTED = -2,   /* dims/dtype outside what the kernels implement */
+    MLA_ERR_MISALIGNED = -3,    /* a device pointer is not 16-byte aligned */
+    MLA_ERR_WORKSPACE = -4,     /* workspace NULL or smaller than mla_workspace_bytes() */
+    MLA_ERR_CUDA = -5,          /* a CUDA runtime/driver call failed (launch, tensor map) */
+    MLA_ERR_DEVICE_FAULT = -6   /* a kernel reported a fault through the status word */
+} mla_status;
+
+typedef enum { MLA_BF16 = 0, MLA_FP32 = 1 } mla_dtype;
+
+typedef struct {
+    int d_model;       /* d: hidden size */
+    int n_h;           /* attention heads */
+    int d_h;           /* per-head dimension of q^C, k^C, v */
+    int d_R;           /* per-head rotary dimension (d_e on some pages), even */
+    int d_c;           /* KV compression dimension (latent width) */
+    int d_cq;          /* query compression dimension d_c'; 0 = no query compression (V2-Lite) */
+    double rope_base;  /* RoPE base, e.g. 10000 */
+    int dtype;         /* mla_dtype: storage type of h, weights and cache */
+} mla_dims;
+
+typedef struct {
+    const void* W_DQ;  /* [d_cq x d]; ignored when d_cq == 0 */
+    const void* W_UQ;
+    const void* W_QR;
+    const void* W_DKV;
+    const void* W_UK;
+    const void* W_UV;
+    const void* W_KR;
+    const void* W_O;
+} mla_weights;
+
+typedef struct {
+    void* base;                 /* device: rows of (d_c + d_R) elements */
+    const int64_t* seq_start;   /* device [n_seq]: row of token 0 of each sequence */
+    const int32_t* capacity;    /* device [n_seq] or NULL: rows reserved per sequence; a write at
+                                   pos >= capacity[s] is skipped and raises MLA_ERR_DEVICE_FAULT */
+} mla_cache;
+
+/* Bytes of workspace needed by mla_decode for batches up to `max_batch` and by
+ * mla_cache_append / mla_prefill for up to `max_tokens` tokens per call.  The
+ * workspace is caller-owned device memory (256-byte aligned); one workspace
+ * must not be used by two calls that run at the same time. */
+size_t mla_workspace_bytes(const mla_dims* dims, int max_batch, int max_tokens);
+
+/* Cache append (the cache-write half of App. C): for t in [0, T),
+ *   row = seq_start[seq_idx[t]] + pos[t]
+ *   cache[row] = [ c^KV = W_DKV h_t | k^R = RoPE_{pos[t]}(W_KR h_t) ]  rounded to the cache dtype.
+ * h: device [T x d_model]; seq_idx, pos: device int32 [T]. */
+mla_status mla_cache_append(const mla_dims* dims, const mla_weights* w,
+                            const void* h, int T,
+                            const int32_t* seq_idx, const int32_t* pos,
+                            const mla_cache* cache,
+                            void* workspace, size_t workspace_bytes,
+                            mla_stream_t stream);
+
+/* Decode step (App. C with absorption): one new token per sequence b in [0, B).
+ * seqlen[b] (device int32) = L_b tokens already cached for sequence b.  The new
+ * token's cache row is written at position L_b (row seq_start[b] + L_b) and the
+ * token attends over positions 0..L_b.  seqlen is not modified.
+ * h: device [B x d_model]; u: device fp32 [B x d_model] (output, overwritten). */
+mla_status mla_decode(const mla_dims* dims, const mla_weights* w,
+                      const void* h, int B,
+                      const mla_cache* cache, const int32_t* seqlen,
+                      float* u,
+                      void* workspace, size_t workspace_bytes,
+                      mla_stream_t stream);
+
+/* Causal prefill of T tokens of sequence `seq` at positions start_pos .. start_pos+T-1
+ * (App. C with j <= t).  Writes their cache rows, then each token attends over
+ * the cached prefix (positions < start_pos, already in the cache) and over the
+ * new tokens up to itself.  h: device [T x d_model]; u: device fp32 [T x d_model]. */
+mla_status mla_prefill(const mla_dims* dims, const mla_weights* w,
+                       const void* h, int T, int start_pos,
+                       const mla_cache* cache, int seq,
+                       float* u,
+                       void* workspace, size_t workspace_bytes,
+                       mla_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the device status word kept in the
+ * workspace.  Returns MLA_OK, MLA_ERR_DEVICE_FAULT (a kernel flagged a fault;
+ * *detail, if non-NULL, receives the fault bits) or MLA_ERR_CUDA. */
+mla_status mla_get_device_status(void* workspace, mla_stream_t stream, int* detail);
+
+/* Static description of a status code. */
+const char* mla_status_string(mla_status s);
+
+/* Byte offset inside the workspace of an intermediate left by the last
+ * mla_decode call with batch `max_batch` (`max_tokens` is ignored), for
+ * inspection in tests.  All are in the storage dtype: 0 = c^Q [B x d_cq],
+ * 1 = q^C [B x n_h d_h], 2 = Q_lat [B x n_h x (d_c+d_R)] = [W_UK_i^T q^C_i ; q^R_i]
+ * pre-multiplied by log2(e)/sqrt(d_h+d_R), 3 = O_lat [B x n_h x d_c]
+ * (normalised latent output), 4 = o [B x n_h d_h].  Returns (size_t)-1 for an
+ * unknown id or invalid dims. */
+size_t mla_workspace_offset(const mla_dims* dims, int max_batch, int max_tokens, int which);
+
+/* Diagnostic timing hook.  While set, every mla_decode / mla_prefill call
+ * records CUDA event `begin` (a cudaEvent_t) on its stream just before the
+ * launch of its attention kernel and `end` just after it, so a caller can time
+ * that kernel alone.  NULL, NULL clears it.  Process-wide setting; callers on
+ * several threads must not use it concurrently. */
+void mla_set_attention_events(void* begin, void* end);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_B200_H */

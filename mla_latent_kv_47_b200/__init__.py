@@ -1,0 +1,174 @@
+"""Python binding of the B200 MLA latent-KV library (libmla_b200.so).
+
+Argument marshalling only: every step of the MLA path runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  The
+library must be built (``python -m mla_latent_kv_47_b200.build``); importing
+this module without it raises, there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmla_b200.so")
+
+MLA_BF16, MLA_FP32 = 0, 1
+STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3: "MLA_ERR_MISALIGNED",
+          -4: "MLA_ERR_WORKSPACE", -5: "MLA_ERR_CUDA", -6: "MLA_ERR_DEVICE_FAULT"}
+FAULT_CAPACITY, FAULT_WAIT_TIMEOUT, FAULT_PLAN = 1, 2, 4
+WS_CQ, WS_QC, WS_QLAT, WS_OLAT, WS_O = range(5)
+
+EXPORTS = ("mla_workspace_bytes", "mla_cache_append", "mla_decode", "mla_prefill",
+           "mla_get_device_status", "mla_status_string", "mla_workspace_offset", "mla_set_attention_events")
+
+
+class MLAError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({status_string(code)})")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int), ("n_h", ctypes.c_int), ("d_h", ctypes.c_int), ("d_R", ctypes.c_int),
+                ("d_c", ctypes.c_int), ("d_cq", ctypes.c_int), ("rope_base", ctypes.c_double),
+                ("dtype", ctypes.c_int)]
+
+
+class Weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("W_DQ", "W_UQ", "W_QR", "W_DKV", "W_UK", "W_UV", "W_KR", "W_O")]
+
+
+class Cache(ctypes.Structure):
+    _fields_ = [("base", ctypes.c_void_p), ("seq_start", ctypes.c_void_p), ("capacity", ctypes.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m mla_latent_kv_47_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    P = ctypes.POINTER
+    lib.mla_workspace_bytes.argtypes = [P(Dims), i32, i32]
+    lib.mla_workspace_bytes.restype = sz
+    lib.mla_workspace_offset.argtypes = [P(Dims), i32, i32, i32]
+    lib.mla_workspace_offset.restype = sz
+    lib.mla_cache_append.argtypes = [P(Dims), P(Weights), vp, i32, vp, vp, P(Cache), vp, sz, vp]
+    lib.mla_cache_append.restype = i32
+    lib.mla_decode.argtypes = [P(Dims), P(Weights), vp, i32, P(Cache), vp, vp, vp, sz, vp]
+    lib.mla_decode.restype = i32
+    lib.mla_prefill.argtypes = [P(Dims), P(Weights), vp, i32, i32, P(Cache), i32, vp, vp, sz, vp]
+    lib.mla_prefill.restype = i32
+    lib.mla_get_device_status.argtypes = [vp, vp, P(i32)]
+    lib.mla_get_device_status.restype = i32
+    lib.mla_status_string.argtypes = [i32]
+    lib.mla_status_string.restype = ctypes.c_char_p
+    lib.mla_set_attention_events.argtypes = [vp, vp]
+    lib.mla_set_attention_events.restype = None
+    return lib
+
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        _LIB = _load()
+    return _LIB
+
+
+def __getattr__(name):
+    # `lib` is loaded on first use, so the build script can import this package
+    # before the library exists.  A missing library raises ImportError here.
+    if name == "lib":
+        return _lib()
+    raise AttributeError(name)
+
+
+def status_string(code: int) -> str:
+    return _lib().mla_status_string(int(code)).decode()
+
+
+def make_dims(d) -> Dims:
+    """ctypes dims from any object with the fields of synth.Dims."""
+    return Dims(d.d_model, d.n_h, d.d_h, d.d_R, d.d_c, d.d_cq, float(d.rope_base),
+                MLA_FP32 if getattr(d, "dtype", "bf16") == "fp32" else MLA_BF16)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    assert t.is_cuda and t.is_contiguous(), "device tensors must be contiguous CUDA tensors"
+    return t.data_ptr()
+
+
+def make_weights(W: dict) -> Weights:
+    return Weights(*[_ptr(W.get(n)) for n in ("W_DQ", "W_UQ", "W_QR", "W_DKV", "W_UK", "W_UV", "W_KR", "W_O")])
+
+
+def make_cache(base, seq_start, capacity=None) -> Cache:
+    assert seq_start.dtype == torch.int64
+    assert capacity is None or capacity.dtype == torch.int32
+    return Cache(_ptr(base), _ptr(seq_start), _ptr(capacity))
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(code, where):
+    if code != 0:
+        raise MLAError(code, where)
+
+
+def workspace_bytes(dims: Dims, max_batch: int, max_tokens: int) -> int:
+    return int(_lib().mla_workspace_bytes(ctypes.byref(dims), int(max_batch), int(max_tokens)))
+
+
+def workspace_offset(dims: Dims, batch: int, which: int) -> int:
+    return int(_lib().mla_workspace_offset(ctypes.byref(dims), int(batch), 0, int(which)))
+
+
+def alloc_workspace(dims: Dims, max_batch: int, max_tokens: int, device="cuda") -> torch.Tensor:
+    n = workspace_bytes(dims, max_batch, max_tokens)
+    if n == 0:
+        raise MLAError(-2, "mla_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def cache_append(dims, weights, h, seq_idx, pos, cache, workspace, stream=None):
+    assert seq_idx.dtype == torch.int32 and pos.dtype == torch.int32
+    _check(_lib().mla_cache_append(ctypes.byref(dims), ctypes.byref(weights), _ptr(h), int(h.shape[0]),
+                                _ptr(seq_idx), _ptr(pos), ctypes.byref(cache), _ptr(workspace),
+                                workspace.numel(), _stream(stream)), "mla_cache_append")
+
+
+def decode(dims, weights, h, cache, seqlen, u, workspace, stream=None):
+    assert seqlen.dtype == torch.int32 and u.dtype == torch.float32
+    _check(_lib().mla_decode(ctypes.byref(dims), ctypes.byref(weights), _ptr(h), int(h.shape[0]),
+                          ctypes.byref(cache), _ptr(seqlen), _ptr(u), _ptr(workspace), workspace.numel(),
+                          _stream(stream)), "mla_decode")
+
+
+def prefill(dims, weights, h, start_pos, cache, seq, u, workspace, stream=None):
+    assert u.dtype == torch.float32
+    _check(_lib().mla_prefill(ctypes.byref(dims), ctypes.byref(weights), _ptr(h), int(h.shape[0]), int(start_pos),
+                           ctypes.byref(cache), int(seq), _ptr(u), _ptr(workspace), workspace.numel(),
+                           _stream(stream)), "mla_prefill")
+
+
+def device_status(workspace, stream=None):
+    """(status code, fault bits); synchronises the stream and clears the word."""
+    detail = ctypes.c_int(0)
+    code = _lib().mla_get_device_status(_ptr(workspace), _stream(stream), ctypes.byref(detail))
+    return int(code), int(detail.value)
+
+
+def set_attention_events(begin=None, end=None):
+    """Bracket the attention kernel of the next calls with two torch.cuda.Event objects (None clears)."""
+    _lib().mla_set_attention_events(ctypes.c_void_p(begin.cuda_event) if begin is not None else None,
+                                 ctypes.c_void_p(end.cuda_event) if end is not None else None)

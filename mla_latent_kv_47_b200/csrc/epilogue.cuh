@@ -1,0 +1,152 @@
+// epilogue.cuh -- what happens to one GEMM output element y[m, n] (feature m,
+// token n) once its dot product is complete: plain stores, the decoupled RoPE
+// of "DeepSeek-V2 summary" (7shi.hateblo.jp) §2.1.3 applied to q^R and k^R,
+// and the cache-row writes of the boxed vectors of App. C.
+#pragma once
+#include "ptx.cuh"
+
+namespace mla {
+
+enum EpiKind : int {
+  EPI_STORE = 0,       // out[n * ld + col0 + m] = y * scale
+  EPI_QLAT_ROPE = 1,   // m = head * d_R + j:  Qlat[n][head][d_c + j] = RoPE(y)_j * scale
+  EPI_PER_HEAD = 2,    // per-head GEMM:  out[n * ld + head * hs + m] = y * scale
+  EPI_CACHE_CKV = 3,   // m = c:  cache[row(n)][c] = y
+  EPI_CACHE_KR = 4,    // m = j:  cache[row(n)][d_c + j] = RoPE(y)_j
+  EPI_QP_ROPE = 5,     // m = head * d_R + j:  out[n][head][d_h + j] = RoPE(y)_j * scale  (prefill q)
+  EPI_HEADS = 6,       // m = head * d_h + e:  out[n][head][e] = y * scale  (row stride ld, head stride hs)
+};
+
+struct Epi {
+  int kind;
+  int out_f32;      // 1: fp32 output, 0: bf16 (or the storage type on the CUDA-core path)
+  void* out;
+  long long ld;     // elements between consecutive tokens n
+  long long hs;     // elements between heads (EPI_HEADS / EPI_QP_ROPE / EPI_QLAT_*)
+  int col0;         // column offset (EPI_STORE) or head-local offset (EPI_HEADS, EPI_QP_ROPE)
+  int dh;           // rows per head for EPI_HEADS
+  float scale;
+};
+
+// Where token n of a GEMM sits: its sequence, its position, its cache row.
+struct TokenMap {
+  const int32_t* pos;        // position of token n, or NULL: pos_base + n
+  int pos_base;
+  const int32_t* seq;        // sequence of token n, or NULL: seq_const (>= 0) or n (seq_const < 0)
+  int seq_const;
+  const int64_t* seq_start;  // cache row of token 0 of each sequence
+  const int32_t* capacity;   // NULL or rows reserved per sequence
+  void* cache;
+  int row_elems;             // d_c + d_R
+  int d_c, d_R;
+  double log2_base;          // log2(rope_base)
+};
+
+__device__ __forceinline__ int tok_pos(const TokenMap& t, int n) { return t.pos ? t.pos[n] : t.pos_base + n; }
+__device__ __forceinline__ int tok_seq(const TokenMap& t, int n) {
+  return t.seq ? t.seq[n] : (t.seq_const >= 0 ? t.seq_const : n);
+}
+
+// Rotation angle of pair i at position pos, reduced to [-pi, pi].  The
+// product pos * base^(-2i/d_R) is formed and reduced in fp64 (positions reach
+// 1.3e5, where an fp32 angle would already be off by ~4e-3 rad), then sine and
+// cosine are taken in fp32.
+__device__ __forceinline__ double rope_inv_freq(int i, int d_R, double log2_base) {
+  return exp2(-(2.0 * i / d_R) * log2_base);
+}
+__device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float& c, float& s) {
+  const double two_pi_hi = 6.283185307179586;
+  const double two_pi_lo = 2.4492935982947064e-16;
+  double phi = static_cast<double>(pos) * inv_freq;
+  double k = rint(phi * (1.0 / two_pi_hi));
+  double r = fma(-k, two_pi_hi, phi);
+  r = fma(-k, two_pi_lo, r);
+  sincosf(static_cast<float>(r), &s, &c);
+}
+
+// Rotated value of component j (of an interleaved pair) given its own value y
+// and its partner's value yp: (a, b) -> (a cos - b sin, a sin + b cos).
+__device__ __forceinline__ float rope_apply(int j, float y, float yp, float c, float s) {
+  return (j & 1) ? (yp * s + y * c) : (y * c - yp * s);
+}
+
+template <typename T>
+__device__ __forceinline__ void store_elem(void* base, long long idx, float v, int out_f32) {
+  if (out_f32) {
+    reinterpret_cast<float*>(base)[idx] = v;
+  } else {
+    reinterpret_cast<T*>(base)[idx] = static_cast<T>(v);
+  }
+}
+
+// Cache row of token n or -1 when the write must be skipped (capacity).
+__device__ __forceinline__ long long cache_row(const TokenMap& t, int n, int* status) {
+  const int s = tok_seq(t, n);
+  const int p = tok_pos(t, n);
+  if (p < 0 || (t.capacity && p >= t.capacity[s])) {
+    atomicOr(status, FAULT_CAPACITY);
+    return -1;
+  }
+  return t.seq_start[s] + p;
+}
+
+// Applies the epilogue to y = output (m, n).  `yp` is the value of the rotary
+// partner (m ^ 1, n), needed by the RoPE kinds.  `head` is the batch index of
+// per-head GEMMs.  T is the storage type of bf16/fp32 outputs.
+template <typename T>
+__device__ __forceinline__ void epi_apply(const Epi& e, const TokenMap& tk, int m, int n, int head, float y,
+                                          float yp, double inv_freq, int* status) {
+  switch (e.kind) {
+    case EPI_STORE:
+      store_elem<T>(e.out, static_cast<long long>(n) * e.ld + e.col0 + m, y * e.scale, e.out_f32);
+      break;
+    case EPI_QLAT_ROPE: {
+      const int hh = m / tk.d_R, j = m % tk.d_R;
+      float c, s;
+      rope_cos_sin(tok_pos(tk, n), inv_freq, c, s);
+      const float r = rope_apply(j, y, yp, c, s);
+      store_elem<T>(e.out, static_cast<long long>(n) * e.ld + hh * e.hs + tk.d_c + j, r * e.scale, e.out_f32);
+      break;
+    }
+    case EPI_PER_HEAD:
+      store_elem<T>(e.out, static_cast<long long>(n) * e.ld + head * e.hs + m, y * e.scale, e.out_f32);
+      break;
+    case EPI_CACHE_CKV: {
+      const long long row = cache_row(tk, n, status);
+      if (row >= 0) store_elem<T>(tk.cache, row * tk.row_elems + m, y, 0);
+      break;
+    }
+    case EPI_CACHE_KR: {
+      const long long row = cache_row(tk, n, status);
+      float c, s;
+      rope_cos_sin(tok_pos(tk, n), inv_freq, c, s);
+      const float r = rope_apply(m, y, yp, c, s);
+      if (row >= 0) store_elem<T>(tk.cache, row * tk.row_elems + tk.d_c + m, r, 0);
+      break;
+    }
+    case EPI_QP_ROPE: {
+      const int hh = m / tk.d_R, j = m % tk.d_R;
+      float c, s;
+      rope_cos_sin(tok_pos(tk, n), inv_freq, c, s);
+      const float r = rope_apply(j, y, yp, c, s);
+      store_elem<T>(e.out, static_cast<long long>(n) * e.ld + hh * e.hs + e.col0 + j, r * e.scale, e.out_f32);
+      break;
+    }
+    case EPI_HEADS: {
+      const int hh = m / e.dh, j = m % e.dh;
+      store_elem<T>(e.out, static_cast<long long>(n) * e.ld + hh * e.hs + e.col0 + j, y * e.scale, e.out_f32);
+      break;
+    }
+  }
+}
+
+__device__ __forceinline__ bool epi_needs_rope(int kind) {
+  return kind == EPI_QLAT_ROPE || kind == EPI_CACHE_KR || kind == EPI_QP_ROPE;
+}
+__device__ __forceinline__ double epi_inv_freq(const Epi& e, const TokenMap& tk, int m) {
+  if (!epi_needs_rope(e.kind)) return 0.0;
+  const int j = (e.kind == EPI_CACHE_KR) ? m : (m % tk.d_R);
+  return rope_inv_freq(j >> 1, tk.d_R, tk.log2_base);
+}
+
+}  // namespace mla

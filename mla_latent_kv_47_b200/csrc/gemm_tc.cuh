@@ -1,0 +1,238 @@
+// gemm_tc.cuh -- tcgen05 tensor-core GEMM used for every projection of the
+// MLA path (W_DQ/W_DKV/W_KR, W_UQ/W_QR, the absorbed W_UK and W_UV, W_O, and
+// the prefill key/value up-projection).
+//
+//   y[m, n] = sum_k A[m, k] * X[n, k]      A: weight rows (out features), X: tokens
+//
+// "Swap-AB" orientation: the weight is the M=128 operand and the tokens are
+// the N operand (N = 32..256), so decode batches of 32-128 tokens still use
+// full-rate M=128 MMAs and the kernel streams the weights at HBM speed.
+// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
+// issues tcgen05.mma, warps 2-5 run the epilogue (one TMEM lane per thread).
+// Split-K: CTAs of one output tile write fp32 partials; the last one to finish
+// (an atomic ticket, no waiting) sums them in split order and runs the epilogue.
+#pragma once
+#include "epilogue.cuh"
+
+namespace mla {
+
+enum GemmMode : int {
+  GEMM_DENSE = 0,        // A = one of up to 4 weight segments, K-major
+  GEMM_HEAD_KMAJOR = 1,  // per-head A block rows [head*head_rows, +head_rows), K-major (W_UV)
+  GEMM_HEAD_MNMAJOR = 2, // per-head A = W[head*head_rows + k, m]: M contiguous (W_UK^T)
+};
+
+constexpr int kMaxSeg = 4;
+
+struct GemmArgs {
+  CUtensorMap mapA[kMaxSeg];
+  CUtensorMap mapB;
+  int mode;
+  int nseg;
+  int seg_tile0[kMaxSeg + 1];  // first M tile of each segment (cumulative); per-head modes: [0, tiles/head]
+  int seg_rows[kMaxSeg];       // valid rows of each segment (per-head modes: rows of one head's output)
+  int boxA_rows[kMaxSeg];      // TMA box rows of each A segment (K-major: min(128, rows))
+  Epi epi[kMaxSeg];
+  int head_rows;               // per-head modes: A rows per head along the K (MN-major) or M (K-major) axis
+  int b_head_stride;           // per-head modes: column offset of a head's K range inside X
+  int N;                       // tokens
+  int boxB_rows;               // TMA box rows of X (min(BN, N))
+  int kb_total;                // K / 64
+  int kb_per_split;
+  int splits;
+  float* partials;             // [tiles][splits][BN][128] fp32 (splits > 1)
+  int* counters;               // [tiles] tickets, zero before the launch; reset by the last CTA
+  int* status;
+  TokenMap tok;
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
+}
+
+template <int BN, int STAGES>
+struct GemmSmem {
+  static constexpr int kA = 16384;        // 128 rows x 128 B
+  static constexpr int kB = BN * 128;     // BN rows x 128 B
+  static constexpr int kStage = kA + kB;
+  static constexpr int kBytes = 1024 + STAGES * kStage + 256;
+};
+
+template <int BN, bool A_MN, int STAGES>
+__global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ GemmArgs args) {
+  using L = GemmSmem<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * L::kA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * L::kB);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accum = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+
+  // ---- which tile
+  const int mt = blockIdx.x, nt = blockIdx.y, split = blockIdx.z;
+  int seg = 0, head = 0, m0;
+  if (args.mode == GEMM_DENSE) {
+    while (seg + 1 < args.nseg && mt >= args.seg_tile0[seg + 1]) ++seg;
+    m0 = (mt - args.seg_tile0[seg]) * 128;
+  } else {
+    const int tph = args.seg_tile0[1];
+    head = mt / tph;
+    m0 = (mt % tph) * 128;
+  }
+  const int kb0 = split * args.kb_per_split;
+  const int kb1 = min(args.kb_total, kb0 + args.kb_per_split);
+  const int nk = kb1 - kb0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accum, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&args.mapA[seg]);
+    prefetch_tmap(&args.mapB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  WaitCtx wc{args.status, abort_flag};
+
+  if (warp == 0) {
+    if (elect_one()) {
+      const uint64_t polA = policy_evict_first();
+      const uint64_t polB = policy_evict_last();
+      const uint32_t bytesA = A_MN ? 16384u : static_cast<uint32_t>(args.boxA_rows[seg]) * 128u;
+      const uint32_t bytesB = static_cast<uint32_t>(args.boxB_rows) * 128u;
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % STAGES;
+        const uint32_t ph = (i / STAGES) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, wc)) break;
+        mbar_arrive_expect_tx(&full[s], bytesA + bytesB);
+        const int kb = kb0 + i;
+        uint8_t* a = sA + s * L::kA;
+        if (A_MN) {
+          const int y = head * args.head_rows + kb * 64;
+          tma_load_2d(a, &args.mapA[0], &full[s], m0, y, polA);
+          tma_load_2d(a + 8192, &args.mapA[0], &full[s], m0 + 64, y, polA);
+        } else if (args.mode == GEMM_HEAD_KMAJOR) {
+          tma_load_2d(a, &args.mapA[0], &full[s], kb * 64, head * args.head_rows + m0, polA);
+        } else {
+          tma_load_2d(a, &args.mapA[seg], &full[s], kb * 64, m0, polA);
+        }
+        tma_load_2d(sB + s * L::kB, &args.mapB, &full[s], head * args.b_head_stride + kb * 64, nt * BN, polB);
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      constexpr uint32_t idesc = idesc_bf16(128, BN, A_MN, false);
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % STAGES;
+        const uint32_t ph = (i / STAGES) & 1;
+        if (!mbar_wait(&full[s], ph, wc)) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sA + s * L::kA);
+        const uint32_t b_base = smem_u32(sB + s * L::kB);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t ad = A_MN ? sdesc_sw128(a_base + k * 2048, 8192, 1024) : sdesc_sw128(a_base + k * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(b_base + k * 32, 16, 1024);
+          mma_ss(tmem, ad, bd, idesc, (i > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);
+      }
+      mma_commit(accum);
+    }
+  } else {
+    // ---- epilogue: warps 2..5, thread <-> TMEM lane (row of the tile)
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    mbar_wait(accum, 0, wc);
+    tc_fence_after();
+    named_bar_sync(1, 128);            // every epilogue thread sees the same abort decision
+    if (!*abort_flag) {
+      const Epi& e = args.epi[seg];
+      const int m = m0 + row;
+      const int rows_valid = args.seg_rows[seg];
+      const int tile_id = mt + gridDim.x * nt;
+      const double inv_freq = epi_inv_freq(e, args.tok, m);
+      bool do_epi = true;
+      if (args.splits > 1) {
+        float* my = args.partials + (static_cast<long long>(tile_id) * args.splits + split) * (BN * 128);
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          float v[16];
+          tmem_ld16(trow + c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) my[(c + j) * 128 + row] = v[j];
+        }
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 64) {
+          const int old = atomicAdd(&args.counters[tile_id], 1);
+          const int last = (old == args.splits - 1);
+          if (last) args.counters[tile_id] = 0;
+          *last_flag = last;
+        }
+        named_bar_sync(1, 128);
+        do_epi = *last_flag != 0;
+        if (do_epi) __threadfence();
+      }
+      if (do_epi) {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          float v[16];
+          tmem_ld16(trow + c, v);
+          tmem_wait_ld();
+          if (args.splits > 1) {
+            float acc[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+            for (int s = 0; s < args.splits; ++s) {
+              if (s == split) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) acc[j] += v[j];
+              } else {
+                const float* p = args.partials + (static_cast<long long>(tile_id) * args.splits + s) * (BN * 128);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) acc[j] += ld_cg_f32(p + (c + j) * 128 + row);
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = acc[j];
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float yp = __shfl_xor_sync(0xffffffffu, v[j], 1);
+            const int n = nt * BN + c + j;
+            if (n < args.N && m < rows_valid) epi_apply<__nv_bfloat16>(e, args.tok, m, n, head, v[j], yp, inv_freq, args.status);
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace mla

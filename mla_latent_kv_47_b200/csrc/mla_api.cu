@@ -1,0 +1,803 @@
+// mla_api.cu -- the C ABI declared in include/mla.h: argument checks, the
+// workspace layout, TMA tensor maps, and the launch sequence of each entry
+// point.  Every arithmetic step runs in the kernels of this directory.
+#include "mla.h"
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "attn_decode_tc.cuh"
+#include "gemm_tc.cuh"
+#include "simt.cuh"
+
+using namespace mla;
+
+namespace {
+
+constexpr int kMaxWorkers = 296;        // attention workers (partial slots beyond B)
+constexpr int kMaxCounters = 4096;      // split-K tickets
+constexpr int kMaxGemmCtas = 296;       // split-K target: two CTAs per SM on 148 SMs
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace: [status | split-K tickets | split-K partials] followed by ONE of
+// the decode region (sized by the batch) or the prefill region (sized by the
+// number of key tokens); a call uses only its own region.
+struct Layout {
+  size_t status, counters, gpart, base_end;
+  size_t tile_start, seg_start, cq, qc, qlat, olat, o, opart, ml, decode_end;
+  size_t p_cq, p_qp, p_rows, p_kc, p_v, p_out, prefill_end;
+};
+
+int elem_size(const mla_dims& d) { return d.dtype == MLA_FP32 ? 4 : 2; }
+int row_elems(const mla_dims& d) { return d.d_c + d.d_R; }
+
+int pick_bn(int N) { return N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256; }
+
+Layout make_layout(const mla_dims& d, int max_batch, int max_tokens) {
+  Layout L{};
+  const size_t es = elem_size(d);
+  const size_t B = static_cast<size_t>(max_batch < 1 ? 1 : max_batch);
+  const size_t T = static_cast<size_t>(max_tokens < 1 ? 1 : max_tokens);
+  const size_t nh = d.n_h, dh = d.d_h, row = row_elems(d);
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, kAlign); return o; };
+  L.status = take(256);
+  L.counters = take(kMaxCounters * sizeof(int));
+  L.gpart = take(static_cast<size_t>(kMaxGemmCtas) * 256 * 128 * sizeof(float));
+  L.base_end = off;
+  L.tile_start = take((B + 1) * sizeof(int));
+  L.seg_start = take((B + 1) * sizeof(int));
+  L.cq = take(B * (d.d_cq ? d.d_cq : 1) * es);
+  L.qc = take(B * nh * dh * es);
+  L.qlat = take(B * nh * row * es);
+  L.olat = take(B * nh * d.d_c * es);
+  L.o = take(B * nh * dh * es);
+  L.opart = take((B + kMaxWorkers) * nh * d.d_c * sizeof(float));
+  L.ml = take((B + kMaxWorkers) * nh * 2 * sizeof(float));
+  L.decode_end = off;
+  off = L.base_end;
+  L.p_cq = take(T * (d.d_cq ? d.d_cq : 1) * es);
+  L.p_qp = take(T * nh * (dh + d.d_R) * es);
+  L.p_rows = take(T * row * es);
+  L.p_kc = take(T * nh * dh * es);
+  L.p_v = take(T * nh * dh * es);
+  L.p_out = take(T * nh * dh * es);
+  L.prefill_end = off;
+  return L;
+}
+
+// ------------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [rows x cols] with row stride `ld` elements; box {64, box_rows}; 128-byte swizzle.
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t ld, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ GEMM description
+struct GemmSpec {
+  int mode = GEMM_DENSE;
+  int nseg = 0;
+  const void* A[kMaxSeg] = {};
+  int rows[kMaxSeg] = {};       // dense: rows of each weight; per-head: output rows per head
+  long long a_ld = 0;           // dense/K-major: row stride of A (elements) = K;  MN-major: row stride (d_c)
+  long long a_total_rows = 0;   // per-head modes: rows of the whole weight tensor
+  int K = 0;
+  Epi epi[kMaxSeg] = {};
+  const void* X = nullptr;
+  long long x_cols = 0, x_ld = 0;
+  int N = 0;
+  int heads = 1;
+  int head_rows = 0;            // rows of A per head
+  int b_head_stride = 0;        // X column offset per head
+  TokenMap tok{};
+};
+
+struct Ctx {
+  mla_dims d;
+  Layout L;
+  uint8_t* ws;
+  int* status;
+  cudaStream_t st;
+  int num_sms;
+};
+
+template <int BN, bool AMN, int STAGES>
+mla_status launch_tc(const GemmArgs& a, dim3 grid, cudaStream_t st) {
+  constexpr int smem = GemmSmem<BN, STAGES>::kBytes;
+  auto kern = gemm_tc_kernel<BN, AMN, STAGES>;
+  static bool attr_set = false;  // idempotent attribute set; races are harmless
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    attr_set = true;
+  }
+  kern<<<grid, 192, smem, st>>>(a);
+  return cudaPeekAtLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+template <bool AMN>
+mla_status launch_tc_bn(int bn, const GemmArgs& a, dim3 grid, cudaStream_t st) {
+  switch (bn) {
+    case 32: return launch_tc<32, AMN, 5>(a, grid, st);
+    case 64: return launch_tc<64, AMN, 4>(a, grid, st);
+    case 128: return launch_tc<128, AMN, 3>(a, grid, st);
+    default: return launch_tc<256, AMN, 4>(a, grid, st);
+  }
+}
+
+mla_status run_gemm_tc(const Ctx& c, const GemmSpec& g) {
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  const int bn = pick_bn(g.N);
+  const int n_tiles = (g.N + bn - 1) / bn;
+  a.mode = g.mode;
+  a.N = g.N;
+  a.boxB_rows = std::min(bn, g.N);
+  a.kb_total = g.K / 64;
+  a.head_rows = g.head_rows;
+  a.b_head_stride = g.b_head_stride;
+  a.status = c.status;
+  a.tok = g.tok;
+  int m_tiles = 0;
+  if (g.mode == GEMM_DENSE) {
+    a.nseg = g.nseg;
+    for (int s = 0; s < g.nseg; ++s) {
+      a.seg_tile0[s] = m_tiles;
+      m_tiles += (g.rows[s] + 127) / 128;
+      a.seg_rows[s] = g.rows[s];
+      a.boxA_rows[s] = std::min(128, g.rows[s]);
+      a.epi[s] = g.epi[s];
+      if (!make_map_2d(&a.mapA[s], g.A[s], g.K, g.rows[s], g.a_ld, a.boxA_rows[s])) return MLA_ERR_CUDA;
+    }
+    a.seg_tile0[g.nseg] = m_tiles;
+  } else {
+    const int tph = (g.rows[0] + 127) / 128;
+    a.nseg = 1;
+    a.seg_tile0[0] = 0;
+    a.seg_tile0[1] = tph;
+    a.seg_rows[0] = g.rows[0];
+    a.epi[0] = g.epi[0];
+    m_tiles = tph * g.heads;
+    if (g.mode == GEMM_HEAD_MNMAJOR) {
+      a.boxA_rows[0] = 64;
+      if (!make_map_2d(&a.mapA[0], g.A[0], g.a_ld, g.a_total_rows, g.a_ld, 64)) return MLA_ERR_CUDA;
+    } else {
+      a.boxA_rows[0] = 128;
+      if (!make_map_2d(&a.mapA[0], g.A[0], g.K, g.a_total_rows, g.a_ld, 128)) return MLA_ERR_CUDA;
+    }
+  }
+  if (!make_map_2d(&a.mapB, g.X, g.x_cols, g.N, g.x_ld, a.boxB_rows)) return MLA_ERR_CUDA;
+  // split-K so that small tile counts still cover the SMs
+  const int tiles = m_tiles * n_tiles;
+  int splits = 1;
+  if (n_tiles == 1 && tiles < kMaxGemmCtas && tiles <= kMaxCounters) {
+    splits = std::max(1, std::min(a.kb_total / 2, kMaxGemmCtas / tiles));
+  }
+  int kbps = (a.kb_total + splits - 1) / splits;
+  splits = (a.kb_total + kbps - 1) / kbps;
+  a.splits = splits;
+  a.kb_per_split = kbps;
+  a.partials = reinterpret_cast<float*>(c.ws + c.L.gpart);
+  a.counters = reinterpret_cast<int*>(c.ws + c.L.counters);
+  dim3 grid(m_tiles, n_tiles, splits);
+  return g.mode == GEMM_HEAD_MNMAJOR ? launch_tc_bn<true>(bn, a, grid, c.st) : launch_tc_bn<false>(bn, a, grid, c.st);
+}
+
+template <typename T>
+mla_status run_gemm_simt(const Ctx& c, const GemmSpec& g) {
+  SimtGemmArgs a;
+  memset(&a, 0, sizeof(a));
+  int M = 0;
+  if (g.mode == GEMM_DENSE) {
+    a.nseg = g.nseg;
+    for (int s = 0; s < g.nseg; ++s) {
+      a.A[s] = g.A[s];
+      a.seg_row0[s] = M;
+      M += g.rows[s];
+      a.epi[s] = g.epi[s];
+    }
+    a.seg_row0[g.nseg] = M;
+    a.a_sm = g.a_ld;
+    a.a_sk = 1;
+    a.a_hoff = 0;
+  } else {
+    a.nseg = 1;
+    a.A[0] = g.A[0];
+    M = g.rows[0];
+    a.seg_row0[0] = 0;
+    a.seg_row0[1] = M;
+    a.epi[0] = g.epi[0];
+    a.a_hoff = static_cast<long long>(g.head_rows) * g.a_ld;
+    if (g.mode == GEMM_HEAD_MNMAJOR) { a.a_sm = 1; a.a_sk = g.a_ld; }
+    else { a.a_sm = g.a_ld; a.a_sk = 1; }
+  }
+  a.X = g.X;
+  a.x_sn = g.x_ld;
+  a.x_hoff = g.b_head_stride;
+  a.M = M;
+  a.N = g.N;
+  a.K = g.K;
+  a.heads = g.heads;
+  a.tok = g.tok;
+  a.status = c.status;
+  dim3 grid((M + 31) / 32, (g.N + 7) / 8, g.heads);
+  simt_gemm_kernel<T><<<grid, dim3(32, 8), 0, c.st>>>(a);
+  return cudaPeekAtLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+bool tc_gemm_ok(const mla_dims& d) {
+  return d.dtype == MLA_BF16 && d.d_model % 64 == 0 && d.d_cq % 64 == 0 && d.d_c % 128 == 0 && d.d_h == 128 &&
+         (d.n_h * d.d_h) % 64 == 0 && d.d_R % 2 == 0 && d.d_R <= 128;
+}
+
+mla_status run_gemm(const Ctx& c, const GemmSpec& g) {
+  if (tc_gemm_ok(c.d)) return run_gemm_tc(c, g);
+  return c.d.dtype == MLA_FP32 ? run_gemm_simt<float>(c, g) : run_gemm_simt<__nv_bfloat16>(c, g);
+}
+
+// ------------------------------------------------------------------ checks
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+mla_status check_dims(const mla_dims* d) {
+  if (!d) return MLA_ERR_INVALID_ARG;
+  if (d->d_model <= 0 || d->n_h <= 0 || d->d_h <= 0 || d->d_R <= 0 || d->d_c <= 0 || d->d_cq < 0)
+    return MLA_ERR_INVALID_ARG;
+  if (!(d->rope_base > 1.0) || !std::isfinite(d->rope_base)) return MLA_ERR_INVALID_ARG;
+  if (d->dtype != MLA_BF16 && d->dtype != MLA_FP32) return MLA_ERR_UNSUPPORTED;
+  if (d->d_R % 2 != 0) return MLA_ERR_UNSUPPORTED;
+  // CUDA-core kernels hold d_c/32 <= 16 latent columns and d_h/32 <= 8 value columns per lane.
+  if (d->d_c > 512 || d->d_h > 256 || d->d_c % 4 != 0) return MLA_ERR_UNSUPPORTED;
+  // 16-byte rows for every tensor the kernels load
+  const int es = d->dtype == MLA_FP32 ? 4 : 2;
+  if ((row_elems(*d) * es) % 16 || (d->d_model * es) % 16 || (d->d_c * es) % 16) return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
+mla_status check_weights(const mla_dims* d, const mla_weights* w) {
+  if (!w) return MLA_ERR_INVALID_ARG;
+  const void* ps[] = {w->W_UQ, w->W_QR, w->W_DKV, w->W_UK, w->W_UV, w->W_KR, w->W_O};
+  for (const void* p : ps) {
+    if (!p) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(p)) return MLA_ERR_MISALIGNED;
+  }
+  if (d->d_cq) {
+    if (!w->W_DQ) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(w->W_DQ)) return MLA_ERR_MISALIGNED;
+  }
+  return MLA_OK;
+}
+
+mla_status check_cache(const mla_cache* c) {
+  if (!c || !c->base || !c->seq_start) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(c->base)) return MLA_ERR_MISALIGNED;
+  return MLA_OK;
+}
+
+enum Region { REGION_BASE, REGION_DECODE, REGION_PREFILL };
+
+mla_status make_ctx(Ctx& c, const mla_dims* d, int max_batch, int max_tokens, Region region, void* ws,
+                    size_t ws_bytes, mla_stream_t stream) {
+  c.d = *d;
+  c.L = make_layout(*d, max_batch, max_tokens);
+  if (!ws) return MLA_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return MLA_ERR_MISALIGNED;
+  const size_t need = region == REGION_DECODE ? c.L.decode_end
+                      : region == REGION_PREFILL ? c.L.prefill_end : c.L.base_end;
+  if (ws_bytes < need) return MLA_ERR_WORKSPACE;
+  c.ws = static_cast<uint8_t*>(ws);
+  c.status = reinterpret_cast<int*>(c.ws + c.L.status);
+  c.st = reinterpret_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&c.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+TokenMap cache_tokens(const mla_dims& d, const mla_cache* cache) {
+  TokenMap t{};
+  t.seq_start = cache->seq_start;
+  t.capacity = cache->capacity;
+  t.cache = cache->base;
+  t.row_elems = row_elems(d);
+  t.d_c = d.d_c;
+  t.d_R = d.d_R;
+  t.log2_base = std::log2(d.rope_base);
+  t.seq_const = -1;
+  return t;
+}
+
+Epi epi_store(void* out, long long ld, int col0, float scale, int out_f32 = 0) {
+  Epi e{};
+  e.kind = EPI_STORE;
+  e.out = out;
+  e.ld = ld;
+  e.col0 = col0;
+  e.scale = scale;
+  e.out_f32 = out_f32;
+  return e;
+}
+Epi epi_kind(int kind, void* out = nullptr, long long ld = 0, long long hs = 0, int col0 = 0, int dh = 0,
+             float scale = 1.f) {
+  Epi e{};
+  e.kind = kind;
+  e.out = out;
+  e.ld = ld;
+  e.hs = hs;
+  e.col0 = col0;
+  e.dh = dh;
+  e.scale = scale;
+  return e;
+}
+
+float qlat_scale(const mla_dims& d) {
+  return static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d.d_h + d.d_R)));
+}
+
+// Appends the [W_DKV; W_KR] segments (cache-row epilogues) to a dense GEMM.
+void add_cache_segments(GemmSpec& g, const mla_dims& d, const mla_weights* w) {
+  g.A[g.nseg] = w->W_DKV;
+  g.rows[g.nseg] = d.d_c;
+  g.epi[g.nseg] = epi_kind(EPI_CACHE_CKV);
+  ++g.nseg;
+  g.A[g.nseg] = w->W_KR;
+  g.rows[g.nseg] = d.d_R;
+  g.epi[g.nseg] = epi_kind(EPI_CACHE_KR);
+  ++g.nseg;
+}
+
+cudaEvent_t g_attn_begin = nullptr, g_attn_end = nullptr;  // diagnostic hook (mla_set_attention_events)
+
+void attn_event(cudaEvent_t e, cudaStream_t st) {
+  if (e) cudaEventRecord(e, st);
+}
+
+bool attn_tc_ok(const mla_dims& d) {
+  return kAttnTcReady && d.dtype == MLA_BF16 && d.n_h == 128 && d.d_c == 512 && d.d_R == 64;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+void mla_set_attention_events(void* begin, void* end) {
+  g_attn_begin = static_cast<cudaEvent_t>(begin);
+  g_attn_end = static_cast<cudaEvent_t>(end);
+}
+
+size_t mla_workspace_bytes(const mla_dims* dims, int max_batch, int max_tokens) {
+  if (check_dims(dims) != MLA_OK) return 0;
+  const Layout L = make_layout(*dims, max_batch, max_tokens);
+  return std::max(L.decode_end, L.prefill_end);
+}
+
+size_t mla_workspace_offset(const mla_dims* dims, int max_batch, int max_tokens, int which) {
+  if (check_dims(dims) != MLA_OK) return static_cast<size_t>(-1);
+  const Layout L = make_layout(*dims, max_batch, max_tokens);
+  switch (which) {
+    case 0: return L.cq;
+    case 1: return L.qc;
+    case 2: return L.qlat;
+    case 3: return L.olat;
+    case 4: return L.o;
+    default: return static_cast<size_t>(-1);
+  }
+}
+
+const char* mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "ok";
+    case MLA_ERR_INVALID_ARG: return "invalid argument";
+    case MLA_ERR_UNSUPPORTED: return "unsupported dims or dtype";
+    case MLA_ERR_MISALIGNED: return "pointer not 16-byte aligned (workspace: 256-byte)";
+    case MLA_ERR_WORKSPACE: return "workspace missing or too small";
+    case MLA_ERR_CUDA: return "CUDA error";
+    case MLA_ERR_DEVICE_FAULT: return "device fault reported by a kernel";
+  }
+  return "unknown status";
+}
+
+mla_status mla_get_device_status(void* workspace, mla_stream_t stream, int* detail) {
+  if (!workspace) return MLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  // the status word is the first int of every layout
+  if (cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+  if (detail) *detail = v;
+  if (v != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess) return MLA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+    return MLA_ERR_DEVICE_FAULT;
+  }
+  return MLA_OK;
+}
+
+mla_status mla_cache_append(const mla_dims* dims, const mla_weights* w, const void* h, int T, const int32_t* seq_idx,
+                            const int32_t* pos, const mla_cache* cache, void* workspace, size_t workspace_bytes,
+                            mla_stream_t stream) {
+  mla_status s = check_dims(dims);
+  if (s != MLA_OK) return s;
+  if ((s = check_weights(dims, w)) != MLA_OK) return s;
+  if ((s = check_cache(cache)) != MLA_OK) return s;
+  if (T < 0) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (!h || !seq_idx || !pos) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h)) return MLA_ERR_MISALIGNED;
+  Ctx c;
+  if ((s = make_ctx(c, dims, 1, 1, REGION_BASE, workspace, workspace_bytes, stream)) != MLA_OK) return s;
+  const mla_dims& d = *dims;
+  GemmSpec g;
+  g.K = d.d_model;
+  g.a_ld = d.d_model;
+  g.X = h;
+  g.x_cols = d.d_model;
+  g.x_ld = d.d_model;
+  g.N = T;
+  g.tok = cache_tokens(d, cache);
+  g.tok.pos = pos;
+  g.tok.seq = seq_idx;
+  add_cache_segments(g, d, w);
+  if (cudaMemsetAsync(c.ws + c.L.counters, 0, kMaxCounters * sizeof(int), c.st) != cudaSuccess) return MLA_ERR_CUDA;
+  return run_gemm(c, g);
+}
+
+mla_status mla_decode(const mla_dims* dims, const mla_weights* w, const void* h, int B, const mla_cache* cache,
+                      const int32_t* seqlen, float* u, void* workspace, size_t workspace_bytes, mla_stream_t stream) {
+  mla_status s = check_dims(dims);
+  if (s != MLA_OK) return s;
+  if ((s = check_weights(dims, w)) != MLA_OK) return s;
+  if ((s = check_cache(cache)) != MLA_OK) return s;
+  if (B <= 0 || !h || !seqlen || !u) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(u)) return MLA_ERR_MISALIGNED;
+  Ctx c;
+  if ((s = make_ctx(c, dims, B, 1, REGION_DECODE, workspace, workspace_bytes, stream)) != MLA_OK) return s;
+  const mla_dims& d = *dims;
+  const int es = elem_size(d);
+  const int row = row_elems(d);
+  const long long HD = static_cast<long long>(d.n_h) * d.d_h;
+  uint8_t* ws = c.ws;
+  void* cq = ws + c.L.cq;
+  void* qc = ws + c.L.qc;
+  void* qlat = ws + c.L.qlat;
+  void* olat = ws + c.L.olat;
+  void* o = ws + c.L.o;
+  int* tile_start = reinterpret_cast<int*>(ws + c.L.tile_start);
+  int* seg_start = reinterpret_cast<int*>(ws + c.L.seg_start);
+  const float qs = qlat_scale(d);
+  TokenMap tk = cache_tokens(d, cache);
+  tk.pos = seqlen;  // the new token of sequence b sits at position L_b
+  (void)es;
+
+  if (cudaMemsetAsync(ws + c.L.counters, 0, kMaxCounters * sizeof(int), c.st) != cudaSuccess) return MLA_ERR_CUDA;
+
+  // ---- attention plan (device side: reads seqlen, no host sync)
+  const bool tc_attn = attn_tc_ok(d);
+  const int tile_tokens = tc_attn ? kAttnTileTokens : 64;
+  int W = tc_attn ? std::min(kMaxWorkers, c.num_sms / 2) : std::min(kMaxWorkers, c.num_sms * 2);
+  if (W < 1) W = 1;
+  plan_kernel<<<1, 1024, 0, c.st>>>(seqlen, B, tile_tokens, W, tile_start, seg_start, c.status);
+  if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
+
+  // ---- a1 (+a2): down-projections from h, cache append of the new token
+  {
+    GemmSpec g;
+    g.K = d.d_model;
+    g.a_ld = d.d_model;
+    g.X = h;
+    g.x_cols = d.d_model;
+    g.x_ld = d.d_model;
+    g.N = B;
+    g.tok = tk;
+    if (d.d_cq) {
+      g.A[0] = w->W_DQ;
+      g.rows[0] = d.d_cq;
+      g.epi[0] = epi_store(cq, d.d_cq, 0, 1.f);
+      g.nseg = 1;
+    } else {
+      g.A[0] = w->W_UQ;
+      g.rows[0] = static_cast<int>(HD);
+      g.epi[0] = epi_store(qc, HD, 0, 1.f);
+      g.A[1] = w->W_QR;
+      g.rows[1] = d.n_h * d.d_R;
+      g.epi[1] = epi_kind(EPI_QLAT_ROPE, qlat, static_cast<long long>(d.n_h) * row, row, 0, 0, qs);
+      g.nseg = 2;
+    }
+    add_cache_segments(g, d, w);
+    if ((s = run_gemm(c, g)) != MLA_OK) return s;
+  }
+  // ---- a3: query up-projection from c^Q (+ RoPE on q^R)
+  if (d.d_cq) {
+    GemmSpec g;
+    g.K = d.d_cq;
+    g.a_ld = d.d_cq;
+    g.X = cq;
+    g.x_cols = d.d_cq;
+    g.x_ld = d.d_cq;
+    g.N = B;
+    g.tok = tk;
+    g.A[0] = w->W_UQ;
+    g.rows[0] = static_cast<int>(HD);
+    g.epi[0] = epi_store(qc, HD, 0, 1.f);
+    g.A[1] = w->W_QR;
+    g.rows[1] = d.n_h * d.d_R;
+    g.epi[1] = epi_kind(EPI_QLAT_ROPE, qlat, static_cast<long long>(d.n_h) * row, row, 0, 0, qs);
+    g.nseg = 2;
+    if ((s = run_gemm(c, g)) != MLA_OK) return s;
+  }
+  // ---- a4: absorb W_UK into the query: q_abs_i = W_UK_i^T q^C_i
+  {
+    GemmSpec g;
+    g.mode = GEMM_HEAD_MNMAJOR;
+    g.A[0] = w->W_UK;
+    g.rows[0] = d.d_c;
+    g.a_ld = d.d_c;
+    g.a_total_rows = HD;
+    g.K = d.d_h;
+    g.X = qc;
+    g.x_cols = HD;
+    g.x_ld = HD;
+    g.N = B;
+    g.heads = d.n_h;
+    g.head_rows = d.d_h;
+    g.b_head_stride = d.d_h;
+    g.tok = tk;
+    g.epi[0] = epi_kind(EPI_PER_HEAD, qlat, static_cast<long long>(d.n_h) * row, row, 0, 0, qs);
+    g.nseg = 1;
+    if ((s = run_gemm(c, g)) != MLA_OK) return s;
+  }
+  // ---- a5: attention over the latent cache -> per-piece partials;  a6: combine
+  float* opart = reinterpret_cast<float*>(ws + c.L.opart);
+  float* ml = reinterpret_cast<float*>(ws + c.L.ml);
+  attn_event(g_attn_begin, c.st);
+  if (tc_attn) {
+    if ((s = launch_attn_decode_tc(reinterpret_cast<const __nv_bfloat16*>(qlat), cache, seqlen, tile_start, seg_start,
+                                   B, W, opart, ml, c.status, c.st)) != MLA_OK)
+      return s;
+  } else {
+    const size_t shm = (row + 4 * d.d_c + 8) * sizeof(float);
+    dim3 grid(W, d.n_h);
+    if (d.dtype == MLA_FP32)
+      simt_decode_attn_kernel<float><<<grid, 128, shm, c.st>>>(
+          static_cast<const float*>(qlat), static_cast<const float*>(cache->base), cache->seq_start, seqlen,
+          tile_start, seg_start, B, W, d.n_h, d.d_c, d.d_R, tile_tokens, opart, ml);
+    else
+      simt_decode_attn_kernel<__nv_bfloat16><<<grid, 128, shm, c.st>>>(
+          static_cast<const __nv_bfloat16*>(qlat), static_cast<const __nv_bfloat16*>(cache->base), cache->seq_start,
+          seqlen, tile_start, seg_start, B, W, d.n_h, d.d_c, d.d_R, tile_tokens, opart, ml);
+    if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  attn_event(g_attn_end, c.st);
+  {
+    dim3 grid(B, d.n_h);
+    if (d.dtype == MLA_FP32)
+      combine_kernel<float><<<grid, 128, 0, c.st>>>(opart, ml, seg_start, d.n_h, d.d_c, static_cast<float*>(olat));
+    else
+      combine_kernel<__nv_bfloat16><<<grid, 128, 0, c.st>>>(opart, ml, seg_start, d.n_h, d.d_c,
+                                                           static_cast<__nv_bfloat16*>(olat));
+    if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  // ---- a7: absorbed W_UV on the latent output: o_i = W_UV_i o_lat_i
+  {
+    GemmSpec g;
+    g.mode = GEMM_HEAD_KMAJOR;
+    g.A[0] = w->W_UV;
+    g.rows[0] = d.d_h;
+    g.a_ld = d.d_c;
+    g.a_total_rows = HD;
+    g.K = d.d_c;
+    g.X = olat;
+    g.x_cols = static_cast<long long>(d.n_h) * d.d_c;
+    g.x_ld = g.x_cols;
+    g.N = B;
+    g.heads = d.n_h;
+    g.head_rows = d.d_h;
+    g.b_head_stride = d.d_c;
+    g.tok = tk;
+    g.epi[0] = epi_kind(EPI_PER_HEAD, o, HD, d.d_h, 0, 0, 1.f);
+    g.nseg = 1;
+    if ((s = run_gemm(c, g)) != MLA_OK) return s;
+  }
+  // ---- a8: u = W_O o
+  {
+    GemmSpec g;
+    g.A[0] = w->W_O;
+    g.rows[0] = d.d_model;
+    g.a_ld = HD;
+    g.K = static_cast<int>(HD);
+    g.X = o;
+    g.x_cols = HD;
+    g.x_ld = HD;
+    g.N = B;
+    g.tok = tk;
+    g.epi[0] = epi_store(u, d.d_model, 0, 1.f, 1);
+    g.nseg = 1;
+    if ((s = run_gemm(c, g)) != MLA_OK) return s;
+  }
+  return MLA_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+template <typename T>
+__global__ void gather_rows_kernel(const T* __restrict__ cache, const int64_t* __restrict__ seq_start, int seq,
+                                   long long nrows, int row, T* __restrict__ out) {
+  const T* src = cache + seq_start[seq] * row;
+  const long long n = nrows * row;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    out[i] = src[i];
+}
+
+}  // namespace
+
+extern "C" mla_status mla_prefill(const mla_dims* dims, const mla_weights* w, const void* h, int T, int start_pos,
+                                  const mla_cache* cache, int seq, float* u, void* workspace, size_t workspace_bytes,
+                                  mla_stream_t stream) {
+  mla_status s = check_dims(dims);
+  if (s != MLA_OK) return s;
+  if ((s = check_weights(dims, w)) != MLA_OK) return s;
+  if ((s = check_cache(cache)) != MLA_OK) return s;
+  if (T <= 0 || start_pos < 0 || seq < 0 || !h || !u) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(u)) return MLA_ERR_MISALIGNED;
+  const int S = start_pos + T;  // keys of the last token
+  Ctx c;
+  if ((s = make_ctx(c, dims, 1, S, REGION_PREFILL, workspace, workspace_bytes, stream)) != MLA_OK) return s;
+  const mla_dims& d = *dims;
+  const int row = row_elems(d);
+  const int dq = d.d_h + d.d_R;
+  const long long HD = static_cast<long long>(d.n_h) * d.d_h;
+  uint8_t* ws = c.ws;
+  void* cq = ws + c.L.p_cq;
+  void* qp = ws + c.L.p_qp;
+  void* rows = ws + c.L.p_rows;
+  void* kc = ws + c.L.p_kc;
+  void* vv = ws + c.L.p_v;
+  void* att = ws + c.L.p_out;
+  const float qs = qlat_scale(d);
+  TokenMap tk = cache_tokens(d, cache);
+  tk.pos_base = start_pos;
+  tk.seq_const = seq;
+  if (cudaMemsetAsync(ws + c.L.counters, 0, kMaxCounters * sizeof(int), c.st) != cudaSuccess) return MLA_ERR_CUDA;
+  // ---- p1: down-projections and cache rows of the T new tokens
+  {
+    GemmSpec g;
+    g.K = d.d_model;
+    g.a_ld = d.d_model;
+    g.X = h;
+    g.x_cols = d.d_model;
+    g.x_ld = d.d_model;
+    g.N = T;
+    g.tok = tk;
+    if (d.d_cq) {
+      g.A[0] = w->W_DQ;
+      g.rows[0] = d.d_cq;
+      g.epi[0] = epi_store(cq, d.d_cq, 0, 1.f);
+      g.nseg = 1;
+    } else {
+      g.A[0] = w->W_UQ;
+      g.rows[0] = static_cast<int>(HD);
+      g.epi[0] = epi_kind(EPI_HEADS, qp, static_cast<long long>(d.n_h) * dq, dq, 0, d.d_h, qs);
+      g.A[1] = w->W_QR;
+      g.rows[1] = d.n_h * d.d_R;
+      g.epi[1] = epi_kind(EPI_QP_ROPE, qp, static_cast<long long>(d.n_h) * dq, dq, d.d_h, 0, qs);
+      g.nseg = 2;
+    }
+    add_cache_segments(g, d, w);
+    if ((s = run_gemm(c, g)) != MLA_OK) return s;
+  }
+  // ---- p2: queries [q^C ; RoPE(q^R)] per head
+  if (d.d_cq) {
+    GemmSpec g;
+    g.K = d.d_cq;
+    g.a_ld = d.d_cq;
+    g.X = cq;
+    g.x_cols = d.d_cq;
+    g.x_ld = d.d_cq;
+    g.N = T;
+    g.tok = tk;
+    g.A[0] = w->W_UQ;
+    g.rows[0] = static_cast<int>(HD);
+    g.epi[0] = epi_kind(EPI_HEADS, qp, static_cast<long long>(d.n_h) * dq, dq, 0, d.d_h, qs);
+    g.A[1] = w->W_QR;
+    g.rows[1] = d.n_h * d.d_R;
+    g.epi[1] = epi_kind(EPI_QP_ROPE, qp, static_cast<long long>(d.n_h) * dq, dq, d.d_h, 0, qs);
+    g.nseg = 2;
+    if ((s = run_gemm(c, g)) != MLA_OK) return s;
+  }
+  // ---- the sequence's cache rows (prefix + new) as one contiguous block
+  {
+    const int blocks = std::min<long long>(4096, (static_cast<long long>(S) * row + 255) / 256);
+    if (d.dtype == MLA_FP32)
+      gather_rows_kernel<float><<<blocks, 256, 0, c.st>>>(static_cast<const float*>(cache->base), cache->seq_start,
+                                                          seq, S, row, static_cast<float*>(rows));
+    else
+      gather_rows_kernel<__nv_bfloat16><<<blocks, 256, 0, c.st>>>(
+          static_cast<const __nv_bfloat16*>(cache->base), cache->seq_start, seq, S, row,
+          static_cast<__nv_bfloat16*>(rows));
+    if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  // ---- p3: un-absorbed keys and values of every key token: K^C = W_UK c, V = W_UV c
+  {
+    GemmSpec g;
+    g.K = d.d_c;
+    g.a_ld = d.d_c;
+    g.X = rows;
+    g.x_cols = row;
+    g.x_ld = row;
+    g.N = S;
+    g.tok = tk;
+    g.A[0] = w->W_UK;
+    g.rows[0] = static_cast<int>(HD);
+    g.epi[0] = epi_store(kc, HD, 0, 1.f);
+    g.A[1] = w->W_UV;
+    g.rows[1] = static_cast<int>(HD);
+    g.epi[1] = epi_store(vv, HD, 0, 1.f);
+    g.nseg = 2;
+    if ((s = run_gemm(c, g)) != MLA_OK) return s;
+  }
+  // ---- p4: causal attention per head
+  attn_event(g_attn_begin, c.st);
+  {
+    const size_t shm = (dq + 4 * d.d_h + 8) * sizeof(float);
+    dim3 grid(T, d.n_h);
+    if (d.dtype == MLA_FP32)
+      simt_prefill_attn_kernel<float><<<grid, 128, shm, c.st>>>(
+          static_cast<const float*>(qp), static_cast<const float*>(kc), static_cast<const float*>(vv),
+          static_cast<const float*>(rows), T, start_pos, d.n_h, d.d_h, d.d_R, d.d_c, static_cast<float*>(att));
+    else
+      simt_prefill_attn_kernel<__nv_bfloat16><<<grid, 128, shm, c.st>>>(
+          static_cast<const __nv_bfloat16*>(qp), static_cast<const __nv_bfloat16*>(kc),
+          static_cast<const __nv_bfloat16*>(vv), static_cast<const __nv_bfloat16*>(rows), T, start_pos, d.n_h,
+          d.d_h, d.d_R, d.d_c, static_cast<__nv_bfloat16*>(att));
+    if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  attn_event(g_attn_end, c.st);
+  // ---- p5: u = W_O o
+  {
+    GemmSpec g;
+    g.A[0] = w->W_O;
+    g.rows[0] = d.d_model;
+    g.a_ld = HD;
+    g.K = static_cast<int>(HD);
+    g.X = att;
+    g.x_cols = HD;
+    g.x_ld = HD;
+    g.N = T;
+    g.tok = tk;
+    g.epi[0] = epi_store(u, d.d_model, 0, 1.f, 1);
+    g.nseg = 1;
+    if ((s = run_gemm(c, g)) != MLA_OK) return s;
+  }
+  return MLA_OK;
+}

@@ -1,0 +1,318 @@
+// simt.cuh -- CUDA-core kernels of the MLA path.  They serve fp32 storage
+// (the tiny preset, where tensor cores would need tf32 and the work is a few
+// kFLOP) and any dims the tensor-core kernels do not cover.  Also here: the
+// device-side split planner and the split-combine, shared by all attention
+// kernels.
+#pragma once
+#include "epilogue.cuh"
+
+namespace mla {
+
+constexpr int kMaxSegSimt = 4;
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// ---------------------------------------------------------------- GEMM
+// y[m, n] = sum_k A[head*a_hoff + m*a_sm + k*a_sk] * X[head*x_hoff + n*x_sn + k]
+// Block: 32 x 8 threads, threadIdx.x -> m (so the RoPE partner m^1 is a lane
+// shuffle away), threadIdx.y -> n.
+struct SimtGemmArgs {
+  const void* A[kMaxSegSimt];
+  int seg_row0[kMaxSegSimt + 1];   // cumulative rows of the segments (dense mode)
+  long long a_sm, a_sk, a_hoff;    // element strides of A (per-head offset)
+  const void* X;
+  long long x_sn, x_hoff;
+  int M, N, K, nseg, heads;
+  Epi epi[kMaxSegSimt];
+  TokenMap tok;
+  int* status;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) simt_gemm_kernel(const __grid_constant__ SimtGemmArgs a) {
+  const int m_all = blockIdx.x * 32 + threadIdx.x;
+  const int n = blockIdx.y * 8 + threadIdx.y;
+  const int head = blockIdx.z;
+  int seg = 0;
+  while (seg + 1 < a.nseg && m_all >= a.seg_row0[seg + 1]) ++seg;
+  const int m = m_all - a.seg_row0[seg];
+  const bool valid = (m_all < a.M) && (n < a.N);
+  float acc = 0.f;
+  if (valid) {
+    const T* A = reinterpret_cast<const T*>(a.A[seg]) + head * a.a_hoff + m * a.a_sm;
+    const T* X = reinterpret_cast<const T*>(a.X) + head * a.x_hoff + static_cast<long long>(n) * a.x_sn;
+    for (int k = 0; k < a.K; ++k) acc += to_f32(A[k * a.a_sk]) * to_f32(X[k]);
+  }
+  const float partner = __shfl_xor_sync(0xffffffffu, acc, 1);
+  if (valid) {
+    const Epi& e = a.epi[seg];
+    epi_apply<T>(e, a.tok, m, n, head, acc, partner, epi_inv_freq(e, a.tok, m), a.status);
+  }
+}
+
+// ---------------------------------------------------------------- planner
+// Splits the attention work of a decode batch into W contiguous ranges of
+// tiles (`tile_tokens` tokens of one sequence each).  Outputs, for every
+// sequence b: tile_start[b] (cumulative tiles, [B+1]) and seg_start[b]
+// (cumulative number of (worker, sequence) pieces, [B+1]).  The piece of
+// worker w on sequence b is partial slot seg_start[b] + w - worker_of(tile_start[b]).
+__host__ __device__ __forceinline__ int worker_of_tile(long long t, long long T, int W) {
+  return static_cast<int>(((t + 1) * W + T - 1) / T) - 1;
+}
+__host__ __device__ __forceinline__ long long worker_begin(int w, long long T, int W) {
+  return (static_cast<long long>(w) * T) / W;
+}
+
+__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seqlen, int B, int tile_tokens, int W,
+                                                    int* tile_start, int* seg_start, int* status) {
+  __shared__ long long s_scan[1024];
+  __shared__ long long s_base;
+  // pass 1: cumulative tiles
+  if (threadIdx.x == 0) s_base = 0;
+  __syncthreads();
+  for (int b0 = 0; b0 < B; b0 += 1024) {
+    const int b = b0 + threadIdx.x;
+    long long v = 0;
+    if (b < B) {
+      const int L = seqlen[b];
+      if (L < 0) atomicOr(status, FAULT_PLAN);
+      v = (max(L, 0) + 1 + tile_tokens - 1) / tile_tokens;
+    }
+    s_scan[threadIdx.x] = v;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {
+      const long long add = threadIdx.x >= off ? s_scan[threadIdx.x - off] : 0;
+      __syncthreads();
+      s_scan[threadIdx.x] += add;
+      __syncthreads();
+    }
+    if (b < B) tile_start[b + 1] = static_cast<int>(s_base + s_scan[threadIdx.x]);
+    __syncthreads();
+    if (threadIdx.x == 1023) s_base += s_scan[1023];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) tile_start[0] = 0;
+  const long long T = s_base;
+  __syncthreads();
+  // pass 2: pieces per sequence
+  if (threadIdx.x == 0) s_base = 0;
+  __syncthreads();
+  for (int b0 = 0; b0 < B; b0 += 1024) {
+    const int b = b0 + threadIdx.x;
+    long long v = 0;
+    if (b < B) {
+      const long long t0 = (b == 0) ? 0 : tile_start[b];
+      const long long t1 = tile_start[b + 1];
+      v = worker_of_tile(t1 - 1, T, W) - worker_of_tile(t0, T, W) + 1;
+    }
+    s_scan[threadIdx.x] = v;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {
+      const long long add = threadIdx.x >= off ? s_scan[threadIdx.x - off] : 0;
+      __syncthreads();
+      s_scan[threadIdx.x] += add;
+      __syncthreads();
+    }
+    if (b < B) seg_start[b + 1] = static_cast<int>(s_base + s_scan[threadIdx.x]);
+    __syncthreads();
+    if (threadIdx.x == 1023) s_base += s_scan[1023];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) seg_start[0] = 0;
+}
+
+// One piece of a worker's range: sequence b, tiles [t0, t1) of that sequence
+// (sequence-local tile indices), partial slot `slot`.
+struct Piece {
+  int b, t0, t1, slot;
+};
+
+// Pieces of worker w, in order.  Calls f(piece) for each.
+template <typename F>
+__device__ __forceinline__ void for_each_piece(int w, int W, int B, const int* tile_start, const int* seg_start, F&& f) {
+  const long long T = tile_start[B];
+  if (T <= 0) return;
+  const long long r0 = worker_begin(w, T, W), r1 = worker_begin(w + 1, T, W);
+  if (r0 >= r1) return;
+  int lo = 0, hi = B - 1;  // first b with tile_start[b+1] > r0
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (tile_start[mid + 1] > r0) hi = mid; else lo = mid + 1;
+  }
+  for (int b = lo; b < B && tile_start[b] < r1; ++b) {
+    const long long s0 = tile_start[b], s1 = tile_start[b + 1];
+    Piece p;
+    p.b = b;
+    p.t0 = static_cast<int>(max(r0, s0) - s0);
+    p.t1 = static_cast<int>(min(r1, s1) - s0);
+    p.slot = seg_start[b] + (w - worker_of_tile(s0, T, W));
+    f(p);
+  }
+}
+
+// ---------------------------------------------------------------- decode attention (CUDA cores)
+// One CTA per (worker, head); 4 warps split the tokens of each piece.  Scores
+// are in log2 units: Q_lat is pre-multiplied by log2(e)/sqrt(d_h + d_R).
+// Output per piece: unnormalised O = sum_j 2^(s_j - m) c_j, with m and
+// l = sum_j 2^(s_j - m).
+template <typename T>
+__global__ void __launch_bounds__(128) simt_decode_attn_kernel(
+    const T* __restrict__ qlat, const T* __restrict__ cache, const int64_t* __restrict__ seq_start,
+    const int32_t* __restrict__ seqlen, const int* tile_start, const int* seg_start, int B, int W, int n_h,
+    int d_c, int d_R, int tile_tokens, float* __restrict__ o_part, float* __restrict__ ml_part) {
+  extern __shared__ float sm[];
+  const int row = d_c + d_R;
+  float* q = sm;                       // [row]
+  float* wo = sm + row;                // [4][d_c]
+  float* wml = wo + 4 * d_c;           // [4][2]
+  const int w = blockIdx.x, h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for_each_piece(w, W, B, tile_start, seg_start, [&](const Piece& p) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < row; i += 128)
+      q[i] = to_f32(qlat[(static_cast<long long>(p.b) * n_h + h) * row + i]);
+    __syncthreads();
+    const int L1 = seqlen[p.b] + 1;
+    const int j0 = p.t0 * tile_tokens, j1 = min(L1, p.t1 * tile_tokens);
+    const T* base = cache + seq_start[p.b] * row;
+    float m = -INFINITY, l = 0.f;
+    float o[16];
+    const int per = (d_c + 31) / 32;
+    for (int i = 0; i < 16; ++i) o[i] = 0.f;
+    for (int j = j0 + warp; j < j1; j += 4) {
+      const T* r = base + static_cast<long long>(j) * row;
+      float s = 0.f;
+      for (int i = lane; i < row; i += 32) s += q[i] * to_f32(r[i]);
+      for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+      const float mn = fmaxf(m, s);
+      const float alpha = exp2f(m - mn);
+      const float pj = exp2f(s - mn);
+      l = l * alpha + pj;
+      for (int i = 0; i < per && i < 16; ++i) {
+        const int c = lane + 32 * i;
+        o[i] = o[i] * alpha + (c < d_c ? pj * to_f32(r[c]) : 0.f);
+      }
+      m = mn;
+    }
+    for (int i = 0; i < per && i < 16; ++i) {
+      const int c = lane + 32 * i;
+      if (c < d_c) wo[warp * d_c + c] = o[i];
+    }
+    if (lane == 0) {
+      wml[warp * 2] = m;
+      wml[warp * 2 + 1] = l;
+    }
+    __syncthreads();
+    float M = -INFINITY;
+    for (int k = 0; k < 4; ++k) M = fmaxf(M, wml[2 * k]);
+    float sc[4], Lsum = 0.f;
+    for (int k = 0; k < 4; ++k) {
+      sc[k] = (wml[2 * k] == -INFINITY) ? 0.f : exp2f(wml[2 * k] - M);
+      Lsum += sc[k] * wml[2 * k + 1];
+    }
+    float* op = o_part + (static_cast<long long>(p.slot) * n_h + h) * d_c;
+    for (int c = threadIdx.x; c < d_c; c += 128) {
+      float acc = 0.f;
+      for (int k = 0; k < 4; ++k) acc += sc[k] * wo[k * d_c + c];
+      op[c] = acc;
+    }
+    if (threadIdx.x == 0) {
+      ml_part[(static_cast<long long>(p.slot) * n_h + h) * 2] = M;
+      ml_part[(static_cast<long long>(p.slot) * n_h + h) * 2 + 1] = Lsum;
+    }
+  });
+}
+
+// ---------------------------------------------------------------- split combine
+// O_lat[b][h][c] = sum_s 2^(m_s - M) O_s[c] / sum_s 2^(m_s - M) l_s over the
+// pieces s of sequence b (the log-sum-exp merge of softmax partials).
+template <typename T>
+__global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ o_part, const float* __restrict__ ml_part,
+                                                     const int* seg_start, int n_h, int d_c, T* __restrict__ olat) {
+  const int b = blockIdx.x, h = blockIdx.y;
+  const int s0 = seg_start[b], s1 = seg_start[b + 1];
+  float M = -INFINITY;
+  for (int s = s0; s < s1; ++s) M = fmaxf(M, ml_part[(static_cast<long long>(s) * n_h + h) * 2]);
+  float Ls = 0.f;
+  for (int s = s0; s < s1; ++s) {
+    const long long i = (static_cast<long long>(s) * n_h + h) * 2;
+    Ls += exp2f(ml_part[i] - M) * ml_part[i + 1];
+  }
+  const float inv = 1.f / Ls;
+  for (int c = threadIdx.x * 4; c < d_c; c += 128 * 4) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = s0; s < s1; ++s) {
+      const float wgt = exp2f(ml_part[(static_cast<long long>(s) * n_h + h) * 2] - M);
+      const float4 v = *reinterpret_cast<const float4*>(o_part + (static_cast<long long>(s) * n_h + h) * d_c + c);
+      acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
+    }
+    T* dst = olat + (static_cast<long long>(b) * n_h + h) * d_c + c;
+    dst[0] = static_cast<T>(acc.x * inv);
+    dst[1] = static_cast<T>(acc.y * inv);
+    dst[2] = static_cast<T>(acc.z * inv);
+    dst[3] = static_cast<T>(acc.w * inv);
+  }
+}
+
+// ---------------------------------------------------------------- prefill attention (CUDA cores)
+// Un-absorbed causal attention for token t (position start_pos + t) and head h:
+//   s_j = [q^C; q^R] . [K^C_j; k^R_j]  (log2 units, q pre-scaled), j = 0..start_pos+t
+//   o   = sum_j softmax(s)_j V_j
+// qp: [T][n_h][d_h + d_R]; kc, v: [start_pos + T][n_h][d_h]; k^R from the cache rows.
+template <typename T>
+__global__ void __launch_bounds__(128) simt_prefill_attn_kernel(
+    const T* __restrict__ qp, const T* __restrict__ kc, const T* __restrict__ vv, const T* __restrict__ cache_seq,
+    int T_new, int start_pos, int n_h, int d_h, int d_R, int d_c, T* __restrict__ out) {
+  extern __shared__ float sm[];
+  const int dq = d_h + d_R;
+  float* q = sm;              // [dq]
+  float* wo = sm + dq;        // [4][d_h]
+  float* wml = wo + 4 * d_h;  // [4][2]
+  const int t = blockIdx.x, h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < dq; i += 128) q[i] = to_f32(qp[(static_cast<long long>(t) * n_h + h) * dq + i]);
+  __syncthreads();
+  const int nkeys = start_pos + t + 1;
+  const int row = d_c + d_R;
+  float m = -INFINITY, l = 0.f;
+  float o[8];
+  for (int i = 0; i < 8; ++i) o[i] = 0.f;
+  for (int j = warp; j < nkeys; j += 4) {
+    const T* kj = kc + (static_cast<long long>(j) * n_h + h) * d_h;
+    const T* kr = cache_seq + static_cast<long long>(j) * row + d_c;
+    float s = 0.f;
+    for (int i = lane; i < d_h; i += 32) s += q[i] * to_f32(kj[i]);
+    for (int i = lane; i < d_R; i += 32) s += q[d_h + i] * to_f32(kr[i]);
+    for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    const float mn = fmaxf(m, s);
+    const float alpha = exp2f(m - mn), pj = exp2f(s - mn);
+    l = l * alpha + pj;
+    const T* vj = vv + (static_cast<long long>(j) * n_h + h) * d_h;
+    for (int i = 0; i < 8; ++i) {
+      const int c = lane + 32 * i;
+      o[i] = o[i] * alpha + (c < d_h ? pj * to_f32(vj[c]) : 0.f);
+    }
+    m = mn;
+  }
+  for (int i = 0; i < 8; ++i) {
+    const int c = lane + 32 * i;
+    if (c < d_h) wo[warp * d_h + c] = o[i];
+  }
+  if (lane == 0) { wml[2 * warp] = m; wml[2 * warp + 1] = l; }
+  __syncthreads();
+  float M = -INFINITY;
+  for (int k = 0; k < 4; ++k) M = fmaxf(M, wml[2 * k]);
+  float sc[4], Ls = 0.f;
+  for (int k = 0; k < 4; ++k) {
+    sc[k] = (wml[2 * k] == -INFINITY) ? 0.f : exp2f(wml[2 * k] - M);
+    Ls += sc[k] * wml[2 * k + 1];
+  }
+  for (int c = threadIdx.x; c < d_h; c += 128) {
+    float acc = 0.f;
+    for (int k = 0; k < 4; ++k) acc += sc[k] * wo[k * d_h + c];
+    out[(static_cast<long long>(t) * n_h + h) * d_h + c] = static_cast<T>(acc / Ls);
+  }
+}
+
+}  // namespace mla

@@ -181,12 +181,13 @@ def decode_absorbed(W: dict, h_seq, dims, return_parts=False):
     return u
 
 
-def prefill_unabsorbed(W: dict, h, dims, start_pos: int = 0, h_prefix=None):
-    """u for every token of a causal prefill, by the naive App. C formulas.
+def prefill_unabsorbed(W: dict, h, dims, start_pos: int = 0, h_prefix=None, rows=None):
+    """u for the tokens of a causal prefill, by the naive App. C formulas.
 
     h [T, d] are tokens at positions start_pos .. start_pos+T-1; h_prefix
     [start_pos, d] are the hidden states of the tokens already cached.
-    Token t attends over every j <= t.
+    Token t attends over every j <= t.  `rows` (indices into h) limits which
+    outputs are formed; the result then has one row per entry of `rows`.
     """
     h = _f64(h)
     T = h.shape[0]
@@ -195,14 +196,15 @@ def prefill_unabsorbed(W: dict, h, dims, start_pos: int = 0, h_prefix=None):
     pos_all = np.arange(start_pos + T, dtype=np.float64)
     c_kv, k_r = latent_rows(W, h_all, pos_all, dims)
     k, v = keys_values(W, c_kv, k_r, dims)
-    q_c, q_r = queries(W, h, pos_all[start_pos:], dims)
-    q = np.concatenate([q_c, q_r], axis=-1)                            # [T, n_h, dq]
+    rows = list(range(T)) if rows is None else [int(r) for r in rows]
+    q_c, q_r = queries(W, h[rows], pos_all[start_pos:][rows], dims)
+    q = np.concatenate([q_c, q_r], axis=-1)                            # [len(rows), n_h, dq]
     scale = 1.0 / np.sqrt(dims.d_h + dims.d_R)
-    u = np.empty((T, dims.d_model), dtype=np.float64)
-    for t in range(T):
+    u = np.empty((len(rows), dims.d_model), dtype=np.float64)
+    for i, t in enumerate(rows):
         n = start_pos + t + 1
-        o, _ = attend(q[t], k[:n], v[:n], scale)
-        u[t] = _output(W, o, dims)
+        o, _ = attend(q[i], k[:n], v[:n], scale)
+        u[i] = _output(W, o, dims)
     return u
 
 

@@ -1,0 +1,123 @@
+"""CPU checks of the C ABI: the library loads without a GPU, exports every entry
+point declared in include/mla.h, and rejects bad arguments on the host before
+anything is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def m():
+    from mla_latent_kv_47_b200 import build
+    build.build()
+    import mla_latent_kv_47_b200 as mod
+    return mod
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "mla.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(m):
+    names = declared_functions()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(m.lib, n), n
+    assert set(m.EXPORTS) == set(names)
+
+
+def test_status_strings(m):
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert m.status_string(code) and m.status_string(code) != "unknown status"
+    assert m.status_string(-99) == "unknown status"
+
+
+def test_workspace_sizes(m):
+    import synth
+    for name, p in synth.PRESETS.items():
+        dims = m.make_dims(p.dims)
+        n = m.workspace_bytes(dims, p.batch, p.prefill_T or 1)
+        assert n > 0
+        for which in range(5):
+            off = m.workspace_offset(dims, p.batch, which)
+            assert 0 < off < n and off % 256 == 0
+        assert m.workspace_offset(dims, p.batch, 7) == 2 ** 64 - 1
+    bad = m.make_dims(synth.PRESETS["v2"].dims)
+    bad.d_R = 63
+    assert m.workspace_bytes(bad, 4, 4) == 0
+    bad = m.make_dims(synth.PRESETS["v2"].dims)
+    bad.dtype = 7
+    assert m.workspace_bytes(bad, 4, 4) == 0
+
+
+def test_decode_workspace_grows_with_batch(m):
+    import synth
+    dims = m.make_dims(synth.PRESETS["v2"].dims)
+    assert m.workspace_bytes(dims, 128, 1) > m.workspace_bytes(dims, 64, 1)
+    # prefill region is sized by the key tokens
+    assert m.workspace_bytes(dims, 1, 16384) > m.workspace_bytes(dims, 1, 1024)
+
+
+def _call_decode(m, dims, weights, h, B, cache, seqlen, u, ws, nbytes):
+    return m.lib.mla_decode(ctypes.byref(dims) if dims is not None else None,
+                            ctypes.byref(weights) if weights is not None else None, h, B,
+                            ctypes.byref(cache) if cache is not None else None, seqlen, u, ws, nbytes, None)
+
+
+def test_host_argument_checks_without_gpu(m):
+    """Fake (never dereferenced) device addresses: every case fails a host check."""
+    import synth
+    dims = m.make_dims(synth.PRESETS["v2"].dims)
+    A = 1 << 20  # 16-byte aligned fake address
+    W = m.Weights(*[A] * 8)
+    C = m.Cache(A, A, None)
+    assert _call_decode(m, None, W, A, 4, C, A, A, A, 1 << 40) == -1
+    assert _call_decode(m, dims, None, A, 4, C, A, A, A, 1 << 40) == -1
+    assert _call_decode(m, dims, W, A, 0, C, A, A, A, 1 << 40) == -1
+    assert _call_decode(m, dims, W, A + 2, 4, C, A, A, A, 1 << 40) == -3
+    W_bad = m.Weights(*[A] * 8)
+    W_bad.W_UK = A + 8
+    assert _call_decode(m, dims, W_bad, A, 4, C, A, A, A, 1 << 40) == -3
+    assert _call_decode(m, dims, W, A, 4, m.Cache(A + 4, A, None), A, A, A, 1 << 40) == -3
+    assert _call_decode(m, dims, W, A, 4, C, A, A, None, 1 << 40) == -4
+    assert _call_decode(m, dims, W, A, 4, C, A, A, A, 1024) == -4
+    assert _call_decode(m, dims, W, A, 4, C, A, A, A + 16, 1 << 40) == -3   # workspace wants 256-byte alignment
+    odd = m.make_dims(synth.PRESETS["v2"].dims)
+    odd.d_R = 63
+    assert _call_decode(m, odd, W, A, 4, C, A, A, A, 1 << 40) == -2
+    noq = m.make_dims(synth.PRESETS["v2"].dims)
+    W_noq = m.Weights(*[A] * 8)
+    W_noq.W_DQ = None
+    assert _call_decode(m, noq, W_noq, A, 4, C, A, A, A, 1 << 40) == -1   # d_cq > 0 needs W_DQ
+
+
+def test_prefill_and_append_argument_checks(m):
+    import synth
+    dims = m.make_dims(synth.PRESETS["v2"].dims)
+    A = 1 << 20
+    W = m.Weights(*[A] * 8)
+    C = m.Cache(A, A, None)
+    lib = m.lib
+    assert lib.mla_prefill(ctypes.byref(dims), ctypes.byref(W), A, 0, 0, ctypes.byref(C), 0, A, A, 1 << 40, None) == -1
+    assert lib.mla_prefill(ctypes.byref(dims), ctypes.byref(W), A, 8, -1, ctypes.byref(C), 0, A, A, 1 << 40, None) == -1
+    assert lib.mla_prefill(ctypes.byref(dims), ctypes.byref(W), A, 8, 0, ctypes.byref(C), -2, A, A, 1 << 40, None) == -1
+    assert lib.mla_cache_append(ctypes.byref(dims), ctypes.byref(W), A, 0, A, A, ctypes.byref(C), A, 1 << 40, None) == 0
+    assert lib.mla_cache_append(ctypes.byref(dims), ctypes.byref(W), A, -1, A, A, ctypes.byref(C), A, 1 << 40, None) == -1
+    assert lib.mla_cache_append(ctypes.byref(dims), ctypes.byref(W), A, 4, None, A, ctypes.byref(C), A, 1 << 40, None) == -1
+    assert lib.mla_get_device_status(None, None, None) == -4
+
+
+def test_oracle_is_not_reachable_from_the_product():
+    """The product package never imports the oracle (it is test infrastructure)."""
+    pkg = os.path.join(ROOT, "mla_latent_kv_47_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in src and "from oracle" not in src, f

@@ -291,3 +291,12 @@ def test_planted_mistake_is_caught(name, monkeypatch):
     ref = np.array(bf.mla_token_output(W, h.tolist(), 3, dims))
     u = om.decode_unabsorbed(W, h, dims)
     assert np.max(np.abs(u - ref)) > 1e-6, f"mutant {name} went unnoticed"
+
+
+def test_prefill_row_subset_matches_full():
+    dims = SMALL
+    W = rand_weights(dims, 14)
+    h = rand_h(dims, 6, 14)
+    full = om.prefill_unabsorbed(W, h, dims)
+    part = om.prefill_unabsorbed(W, h, dims, rows=[5, 0, 3])
+    assert np.array_equal(part, full[[5, 0, 3]])
