@@ -36,12 +36,16 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["v2", "lite", "ragged"], default="v2")
+    ap.add_argument("--ctx", type=int, default=0, help="override cached tokens per sequence (profiling cases)")
+    ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling cases)")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="decode steps only (no clock sampling, e2e, prefill or CPU baseline): for ncu captures")
     return ap.parse_args()
 
 
@@ -54,10 +58,15 @@ def peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def workload_lengths(name):
+def workload_lengths(name, ctx=0, batch=0):
     import synth
     p = synth.preset(name)
-    return p, list(p.seqlen)
+    L = list(p.seqlen)
+    if batch:
+        L = (L * ((batch + len(L) - 1) // len(L)))[:batch]
+    if ctx:
+        L = [ctx] * len(L)
+    return p, L
 
 
 def decode_flops_bytes(d, L):
@@ -244,7 +253,7 @@ def run_ours(args):
     import mla_latent_kv_47_b200 as m
     from mla_latent_kv_47_b200.cache import LatentCache
 
-    p, L = workload_lengths(args.workload)
+    p, L = workload_lengths(args.workload, args.ctx, args.batch)
     d = p.dims
     dims = m.make_dims(d)
     B = len(L)
@@ -258,7 +267,7 @@ def run_ours(args):
     wts = m.make_weights(Wd)
     cache = LatentCache(dims, [x + 1 for x in L], device=dev)
     chunk = 16384
-    ws = m.alloc_workspace(dims, B, chunk + 1, device=dev)
+    ws = m.alloc_workspace(dims, B, 1, device=dev)
     for b, n in enumerate(L):
         for t0 in range(0, n, chunk):
             k = min(chunk, n - t0)
@@ -293,9 +302,19 @@ def run_ours(args):
     ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for e in ev_b + ev_e:  # torch creates the CUDA event on its first record
+        e.record()
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(dev.index) as clk:
+        # keep the GPU busy while the sampler starts, so its samples see load
+        t0 = time.perf_counter()
+        while not args.profile and time.perf_counter() - t0 < 0.5:
+            for _ in range(20):
+                step()
+            torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
         t_start.record()
         for i in range(K):
             m.set_attention_events(ev_b[i], ev_e[i])
@@ -309,6 +328,9 @@ def run_ours(args):
     code, detail = m.device_status(ws)
     assert code == 0, ("decode fault", code, detail)
 
+    if args.profile:
+        print(json.dumps({"profile_run": True, "ms_per_step": ms, "attn_ms": attn_ms}), flush=True)
+        return 0
     # ---- end to end: host (pinned) inputs in, host output back, every step
     h_host = h_new.cpu().pin_memory()
     sl_host = seqlen.cpu().pin_memory()
@@ -351,6 +373,8 @@ def run_ours(args):
         pb = [torch.cuda.Event(enable_timing=True) for _ in range(KP)]
         pe = [torch.cuda.Event(enable_timing=True) for _ in range(KP)]
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for e in pb + pe:
+            e.record()
         barrier()
         torch.cuda.synchronize()
         s0.record()

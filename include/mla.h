@@ -89,6 +89,8 @@ typedef struct {
     const int64_t* seq_start;   /* device [n_seq]: row of token 0 of each sequence */
     const int32_t* capacity;    /* device [n_seq] or NULL: rows reserved per sequence; a write at
                                    pos >= capacity[s] is skipped and raises MLA_ERR_DEVICE_FAULT */
+    int64_t n_rows;             /* rows allocated at `base` (> 0): bounds of every tile load; a
+                                   write at a row >= n_rows is skipped and raises MLA_ERR_DEVICE_FAULT */
 } mla_cache;
 
 /* Bytes of workspace needed by mla_decode for batches up to `max_batch` and by

@@ -42,7 +42,8 @@ class Weights(ctypes.Structure):
 
 
 class Cache(ctypes.Structure):
-    _fields_ = [("base", ctypes.c_void_p), ("seq_start", ctypes.c_void_p), ("capacity", ctypes.c_void_p)]
+    _fields_ = [("base", ctypes.c_void_p), ("seq_start", ctypes.c_void_p), ("capacity", ctypes.c_void_p),
+                ("n_rows", ctypes.c_int64)]
 
 
 def _load():
@@ -110,9 +111,10 @@ def make_weights(W: dict) -> Weights:
 
 
 def make_cache(base, seq_start, capacity=None) -> Cache:
+    """base: [n_rows, d_c + d_R] device tensor; seq_start int64 [n_seq]; capacity int32 [n_seq] or None."""
     assert seq_start.dtype == torch.int64
     assert capacity is None or capacity.dtype == torch.int32
-    return Cache(_ptr(base), _ptr(seq_start), _ptr(capacity))
+    return Cache(_ptr(base), _ptr(seq_start), _ptr(capacity), int(base.shape[0]))
 
 
 def _stream(stream):

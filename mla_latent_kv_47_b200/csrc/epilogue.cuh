@@ -36,6 +36,7 @@ struct TokenMap {
   int seq_const;
   const int64_t* seq_start;  // cache row of token 0 of each sequence
   const int32_t* capacity;   // NULL or rows reserved per sequence
+  long long n_rows;          // rows allocated in the cache
   void* cache;
   int row_elems;             // d_c + d_R
   int d_c, d_R;
@@ -87,7 +88,12 @@ __device__ __forceinline__ long long cache_row(const TokenMap& t, int n, int* st
     atomicOr(status, FAULT_CAPACITY);
     return -1;
   }
-  return t.seq_start[s] + p;
+  const long long row = t.seq_start[s] + p;
+  if (row < 0 || row >= t.n_rows) {
+    atomicOr(status, FAULT_CAPACITY);
+    return -1;
+  }
+  return row;
 }
 
 // Applies the epilogue to y = output (m, n).  `yp` is the value of the rotary

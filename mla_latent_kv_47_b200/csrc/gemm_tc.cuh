@@ -46,10 +46,6 @@ struct GemmArgs {
   TokenMap tok;
 };
 
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
-}
-
 template <int BN, int STAGES>
 struct GemmSmem {
   static constexpr int kA = 16384;        // 128 rows x 128 B

@@ -296,7 +296,7 @@ mla_status check_weights(const mla_dims* d, const mla_weights* w) {
 }
 
 mla_status check_cache(const mla_cache* c) {
-  if (!c || !c->base || !c->seq_start) return MLA_ERR_INVALID_ARG;
+  if (!c || !c->base || !c->seq_start || c->n_rows <= 0) return MLA_ERR_INVALID_ARG;
   if (!aligned16(c->base)) return MLA_ERR_MISALIGNED;
   return MLA_OK;
 }
@@ -325,6 +325,7 @@ TokenMap cache_tokens(const mla_dims& d, const mla_cache* cache) {
   TokenMap t{};
   t.seq_start = cache->seq_start;
   t.capacity = cache->capacity;
+  t.n_rows = cache->n_rows;
   t.cache = cache->base;
   t.row_elems = row_elems(d);
   t.d_c = d.d_c;
@@ -379,8 +380,37 @@ void attn_event(cudaEvent_t e, cudaStream_t st) {
   if (e) cudaEventRecord(e, st);
 }
 
+mla_status launch_attn_decode_tc(const __nv_bfloat16* qlat, const mla_cache* cache, const int32_t* seqlen,
+                                 const int* tile_start, const int* seg_start, int B, int W, int n_h, float* o_part,
+                                 float* ml, int* status, cudaStream_t st) {
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  if (cache->n_rows > (1ll << 31) - 128) return MLA_ERR_UNSUPPORTED;  // tile rows are int32 TMA coordinates
+  if (!make_map_2d(&a.map_cache, cache->base, attn::kRow, cache->n_rows, attn::kRow, 64)) return MLA_ERR_CUDA;
+  a.qlat = qlat;
+  a.seq_start = cache->seq_start;
+  a.seqlen = seqlen;
+  a.tile_start = tile_start;
+  a.seg_start = seg_start;
+  a.B = B;
+  a.W = W;
+  a.n_h = n_h;
+  a.o_part = o_part;
+  a.ml_part = ml;
+  a.status = status;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, attn::kSmem) !=
+        cudaSuccess)
+      return MLA_ERR_CUDA;
+    attr_set = true;
+  }
+  attn_decode_tc_kernel<<<2 * W, 192, attn::kSmem, st>>>(a);
+  return cudaPeekAtLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 bool attn_tc_ok(const mla_dims& d) {
-  return kAttnTcReady && d.dtype == MLA_BF16 && d.n_h == 128 && d.d_c == 512 && d.d_R == 64;
+  return kAttnTcReady && d.dtype == MLA_BF16 && d.n_h <= 128 && d.d_c == 512 && d.d_R == 64;
 }
 
 }  // namespace
@@ -580,7 +610,7 @@ mla_status mla_decode(const mla_dims* dims, const mla_weights* w, const void* h,
   attn_event(g_attn_begin, c.st);
   if (tc_attn) {
     if ((s = launch_attn_decode_tc(reinterpret_cast<const __nv_bfloat16*>(qlat), cache, seqlen, tile_start, seg_start,
-                                   B, W, opart, ml, c.status, c.st)) != MLA_OK)
+                                   B, W, d.n_h, opart, ml, c.status, c.st)) != MLA_OK)
       return s;
   } else {
     const size_t shm = (row + 4 * d.d_c + 8) * sizeof(float);

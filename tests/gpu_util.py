@@ -71,3 +71,30 @@ def fill_cache(m, dims, Wd, cache, ws, seqs_h: dict, lengths, p, gen_seed=1234, 
             seq = torch.full((n,), b, dtype=torch.int32, device="cuda")
             pos = torch.arange(t0, t0 + n, dtype=torch.int32, device="cuda")
             m.cache_append(dims, wts, h, seq, pos, cache.handle, ws)
+
+
+def cache_value_check(got_bits: np.ndarray, Wh: dict, h: np.ndarray, pos: np.ndarray, dims) -> float:
+    """Checks stored bf16 cache rows against the exact rows [c^KV | RoPE(k^R)].
+
+    Bound per element: rounding to bf16 (half an ulp <= 2^-8 |x|) plus the
+    noise of an fp32 dot product of length K = d_model, taken as
+    16 sqrt(K) 2^-24 ||w o h||_2 (a generous multiple of the random-walk size of
+    fp32 summation error); a rotated k^R element carries the noise of both
+    members of its pair plus a few fp32 roundings of the rotation.
+    Returns the largest |error| / bound (must be <= 1)."""
+    from oracle import mla as om
+    c_kv, k_r = om.latent_rows(Wh, h, pos, dims)
+    exact = np.concatenate([c_kv, k_r], axis=1)
+    got = synth.bf16_bits_to_f32(got_bits).astype(np.float64)
+    K = dims.d_model
+    u = 2.0 ** -24
+    h2 = np.asarray(h, np.float64) ** 2
+    noise_c = np.sqrt(h2 @ (np.asarray(Wh["W_DKV"], np.float64) ** 2).T)
+    pre_r = np.asarray(h, np.float64) @ np.asarray(Wh["W_KR"], np.float64).T
+    noise_r = np.sqrt(h2 @ (np.asarray(Wh["W_KR"], np.float64) ** 2).T)
+    pair = noise_r.reshape(noise_r.shape[0], -1, 2).sum(-1).repeat(2, axis=1)
+    pair_mag = np.abs(pre_r).reshape(pre_r.shape[0], -1, 2).sum(-1).repeat(2, axis=1)
+    acc = 16.0 * np.sqrt(K) * u * np.concatenate([noise_c, pair], axis=1)
+    rot = np.concatenate([np.zeros_like(noise_c), 8 * u * pair_mag], axis=1)
+    bound = 2.0 ** -8 * np.abs(exact) + (1 + 2.0 ** -8) * acc + rot
+    return float(np.max(np.abs(got - exact) / bound))

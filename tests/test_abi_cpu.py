@@ -76,7 +76,7 @@ def test_host_argument_checks_without_gpu(m):
     dims = m.make_dims(synth.PRESETS["v2"].dims)
     A = 1 << 20  # 16-byte aligned fake address
     W = m.Weights(*[A] * 8)
-    C = m.Cache(A, A, None)
+    C = m.Cache(A, A, None, 1000)
     assert _call_decode(m, None, W, A, 4, C, A, A, A, 1 << 40) == -1
     assert _call_decode(m, dims, None, A, 4, C, A, A, A, 1 << 40) == -1
     assert _call_decode(m, dims, W, A, 0, C, A, A, A, 1 << 40) == -1
@@ -84,7 +84,8 @@ def test_host_argument_checks_without_gpu(m):
     W_bad = m.Weights(*[A] * 8)
     W_bad.W_UK = A + 8
     assert _call_decode(m, dims, W_bad, A, 4, C, A, A, A, 1 << 40) == -3
-    assert _call_decode(m, dims, W, A, 4, m.Cache(A + 4, A, None), A, A, A, 1 << 40) == -3
+    assert _call_decode(m, dims, W, A, 4, m.Cache(A + 4, A, None, 1000), A, A, A, 1 << 40) == -3
+    assert _call_decode(m, dims, W, A, 4, m.Cache(A, A, None, 0), A, A, A, 1 << 40) == -1   # n_rows required
     assert _call_decode(m, dims, W, A, 4, C, A, A, None, 1 << 40) == -4
     assert _call_decode(m, dims, W, A, 4, C, A, A, A, 1024) == -4
     assert _call_decode(m, dims, W, A, 4, C, A, A, A + 16, 1 << 40) == -3   # workspace wants 256-byte alignment
@@ -102,7 +103,7 @@ def test_prefill_and_append_argument_checks(m):
     dims = m.make_dims(synth.PRESETS["v2"].dims)
     A = 1 << 20
     W = m.Weights(*[A] * 8)
-    C = m.Cache(A, A, None)
+    C = m.Cache(A, A, None, 1000)
     lib = m.lib
     assert lib.mla_prefill(ctypes.byref(dims), ctypes.byref(W), A, 0, 0, ctypes.byref(C), 0, A, A, 1 << 40, None) == -1
     assert lib.mla_prefill(ctypes.byref(dims), ctypes.byref(W), A, 8, -1, ctypes.byref(C), 0, A, A, 1 << 40, None) == -1

@@ -2,8 +2,9 @@
 
 Cache layout and sequence-length indexing are checked bit-exactly: every
 cache row outside the rows written for (sequence, position) keeps its NaN
-poison pattern, and no poisoned row reaches u.  Row values must be within 1
-bf16 ulp of the oracle's rounded rows.  Outputs u must pass the gate
+poison pattern, and no poisoned row reaches u.  Row values must be within
+half a bf16 ulp of the exact row plus the fp32 accumulation noise bound
+(tests/gpu_util.cache_value_check).  Outputs u must pass the gate
 max|d| <= 1e-2 max|ref| and mean|d| <= 2e-3 max|ref| (bf16 storage), or a
 1e-4 bound on both for fp32 storage.
 """
@@ -68,14 +69,13 @@ def run_decode(m, preset, checked, lengths=None, pad=2, oracle="unabsorbed"):
     stats = {}
     for b in checked:
         hb = seqs_h[b]
-        c_kv, k_r = om.latent_rows(Wh, hb, np.arange(L[b] + 1.0), d)
-        rows_ref = np.concatenate([c_kv, k_r], axis=1)
         got = bits[ss[b]:ss[b] + L[b] + 1]
         if d.dtype == "bf16":
-            ref_bits = synth.to_bf16_bits(om.round_bf16_f64(rows_ref).astype(np.float32))
-            ulp = gu.bf16_ulp_diff(got, ref_bits)
-            assert ulp.max() <= 1, f"seq {b}: cache rows differ by {ulp.max()} ulp"
+            ratio = gu.cache_value_check(got, Wh, hb, np.arange(L[b] + 1.0), d)
+            assert ratio <= 1.0, f"seq {b}: cache row error at {ratio:.3g} of its bound"
         else:
+            c_kv, k_r = om.latent_rows(Wh, hb, np.arange(L[b] + 1.0), d)
+            rows_ref = np.concatenate([c_kv, k_r], axis=1)
             gotf = got.view(np.float32).astype(np.float64)
             assert np.max(np.abs(gotf - rows_ref)) <= 1e-5 * np.max(np.abs(rows_ref))
         u_ref = (om.decode_unabsorbed if oracle == "unabsorbed" else om.decode_absorbed)(Wh, hb, d)
