@@ -334,7 +334,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       // ---- epilogue of the piece: unnormalised O_r, m, l
       if (!mbar_wait(o_done, piece & 1, wc)) return;
       tc_fence_after();
-      const bool head = h < a.n_h;
       float* dst = a.o_part + (static_cast<long long>(p.slot) * a.n_h + h) * 512 + rank * 256;
       for (int c = 0; c < 256; c += 32) {
         uint32_t o[32];
