@@ -193,6 +193,22 @@ def blas_threads():
         return os.cpu_count()
 
 
+def reduce_max(x, world, device):
+    """Max of a per-rank number over all ranks (the slowest rank sets the time)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, units_per_rank, ms_per_step):
+    """Whole-job units per second: every rank processes `units_per_rank` per step."""
+    return world * units_per_rank / (ms_per_step * 1e-3)
+
+
 # ============================================================================ reference arm
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
@@ -289,11 +305,7 @@ def run_ours(args):
             dist.barrier()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -411,7 +423,7 @@ def run_ours(args):
                                   f"({pp.seqlen[0] + 1} tokens each) through the fp64 un-absorbed oracle"}
 
     traffic = traffic_record(ATTN_SOURCES)
-    value = world * B / (ms * 1e-3)
+    value = job_throughput(world, B, ms)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",

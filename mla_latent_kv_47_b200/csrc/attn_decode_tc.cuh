@@ -43,9 +43,9 @@ constexpr int kStages = 4;
 constexpr int kChunkBytes = 64 * 128;             // 64 token rows x 64 latent columns, bf16
 constexpr int kStageBytes = 5 * kChunkBytes;      // up to 5 chunks per CTA
 constexpr int kPBytes = 128 * 128;                // P: 128 heads x 64 tokens, bf16
-constexpr int kXBytes = 128 * 128;                // partner's partial S: 128 heads x 64 tokens, fp16
+constexpr int kXBytes = 128 * 128;                // partner's partial S: 128 heads x 64 tokens, fp16 (x2 buffers)
 constexpr int kBarBytes = 256;
-constexpr int kSmem = 1024 + kStages * kStageBytes + kPBytes + kXBytes + kBarBytes;
+constexpr int kSmem = 1024 + kStages * kStageBytes + kPBytes + 2 * kXBytes + kBarBytes;
 constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 320, kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kRow = 576;                         // d_c + d_R
@@ -87,15 +87,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   uint8_t* stages = smem;
   uint8_t* pbuf = stages + kStages * kStageBytes;
   uint8_t* xbuf = pbuf + kPBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(xbuf + kXBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(xbuf + 2 * kXBytes);
   uint64_t* empty = full + kStages;
   uint64_t* s_full = empty + kStages;
   uint64_t* s_free = s_full + 1;
   uint64_t* p_full = s_free + 1;
   uint64_t* p_free = p_full + 1;
-  uint64_t* x_full = p_free + 1;
-  uint64_t* x_free = x_full + 1;
-  uint64_t* q_full = x_free + 1;
+  uint64_t* x_full = p_free + 1;   // [2]
+  uint64_t* x_free = x_full + 2;   // [2]
+  uint64_t* q_full = x_free + 2;
   uint64_t* o_done = q_full + 1;
   uint64_t* drain = o_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -116,8 +116,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     mbar_init(s_free, 128);
     mbar_init(p_full, 128);
     mbar_init(p_free, 1);
-    mbar_init(x_full, 128);
-    mbar_init(x_free, 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&x_full[i], 4);  // one arrival per softmax warp of the partner
+      mbar_init(&x_free[i], 4);
+    }
     mbar_init(q_full, 128);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
@@ -133,6 +135,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   cluster_sync();  // the partner's barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();  // Q_lat and the new cache rows come from the preceding kernels
   WaitCtx wc{a.status, abort_flag};
 
   if (warp == 0) {
@@ -165,38 +168,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         if (!mbar_wait(q_full, piece & 1, wc)) return;
         tc_fence_after();
         const int nt = p.t1 - p.t0;
-        for (int k = 0; k <= nt; ++k) {
-          if (k < nt) {  // S(k) = Q_r C_r(k)^T
-            const int g = it + k;
+        // Event-driven issue: S(j) as soon as its tile landed and S(j-1) was read
+        // out (the softmax reads S one tile ahead), PV(j) as soon as P(j) is
+        // written; S first, so the softmax never waits behind a PV.
+        int ns = 0, npv = 0;
+        uint64_t t_idle = globaltimer();
+        while (npv < nt) {
+          bool issued = false;
+          if (ns < nt) {
+            const int g = it + ns;
             const int s = g % kStages;
-            if (!mbar_wait(&full[s], (g / kStages) & 1, wc)) return;
-            if (!mbar_wait(s_free, (g & 1) ^ 1, wc)) return;
-            tc_fence_after();
-            const uint32_t st = smem_u32(stages + s * kStageBytes);
-            for (int ci = 0; ci < nchunks; ++ci) {
+            if (mbar_try_wait(smem_u32(&full[s]), (g / kStages) & 1) && mbar_try_wait(smem_u32(s_free), (g & 1) ^ 1)) {
+              tc_fence_after();
+              const uint32_t st = smem_u32(stages + s * kStageBytes);
+              for (int ci = 0; ci < nchunks; ++ci) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  mma_ts(tmem + kTmemS, tmem + kTmemQ + ci * 32 + kk * 8,
+                         sdesc_sw128(st + ci * kChunkBytes + kk * 32, 16, 1024), idesc_s, (ci | kk) ? 1u : 0u);
+                }
+              }
+              mma_commit(s_full);
+              ++ns;
+              issued = true;
+            }
+          }
+          if (!issued && npv < ns) {
+            const int g = it + npv;
+            const int s = g % kStages;
+            if (mbar_try_wait(smem_u32(p_full), g & 1)) {
+              tc_fence_after();
+              const uint32_t st = smem_u32(stages + s * kStageBytes);
+              const uint32_t pb = smem_u32(pbuf);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
-                mma_ts(tmem + kTmemS, tmem + kTmemQ + ci * 32 + kk * 8,
-                       sdesc_sw128(st + ci * kChunkBytes + kk * 32, 16, 1024), idesc_s, (ci | kk) ? 1u : 0u);
+                mma_ss(tmem + kTmemO, sdesc_sw128(pb + kk * 32, 16, 1024), sdesc_sw128(st + kk * 2048, 8192, 1024),
+                       idesc_pv, (npv > 0 || kk > 0) ? 1u : 0u);
               }
+              mma_commit(p_free);
+              mma_commit(&empty[s]);
+              if (npv == nt - 1) mma_commit(o_done);
+              ++npv;
+              issued = true;
             }
-            mma_commit(s_full);
           }
-          if (k > 0) {  // O_r += P(k-1) C_r(k-1)
-            const int g = it + k - 1;
-            const int s = g % kStages;
-            if (!mbar_wait(p_full, g & 1, wc)) return;
-            tc_fence_after();
-            const uint32_t st = smem_u32(stages + s * kStageBytes);
-            const uint32_t pb = smem_u32(pbuf);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              mma_ss(tmem + kTmemO, sdesc_sw128(pb + kk * 32, 16, 1024), sdesc_sw128(st + kk * 2048, 8192, 1024),
-                     idesc_pv, (k > 1 || kk > 0) ? 1u : 0u);
-            }
-            mma_commit(p_free);
-            mma_commit(&empty[s]);
-            if (k == nt) mma_commit(o_done);
+          if (issued) {
+            t_idle = globaltimer();
+          } else if (*abort_flag) {
+            return;
+          } else if (globaltimer() - t_idle > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicOr(a.status, FAULT_WAIT_TIMEOUT);
+            return;
           }
         }
         it += nt;
@@ -215,6 +238,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     const uint32_t xfree_peer = mapa(smem_u32(x_free), peer);
     const uint32_t p_row = smem_u32(pbuf) + h * 128;
     const int sw = h & 7;
+    // Partial scores of global tile g: read from TMEM, rounded to fp16 into
+    // `out`, and sent to the partner's exchange buffer g & 1.  The partner is
+    // told once per warp (after the warp's stores, ordered by the warp barrier).
+    auto send = [&](int g, uint32_t (&out)[32]) -> bool {
+      if (!mbar_wait(s_full, g & 1, wc)) return false;
+      tc_fence_after();
+      uint32_t sr[64];
+      tmem_ld32(tl + kTmemS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tl + kTmemS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(s_free);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) out[j] = pack_half2(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1]));
+      const int slot = g & 1;
+      if (!mbar_wait<true>(&x_free[slot], ((g >> 1) & 1) ^ 1, wc)) return false;
+      const uint32_t dst = x_row_peer + slot * kXBytes;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        st_cluster_v4(dst + ((i ^ sw) << 4), make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(xfull_peer + slot * 8);
+      return true;
+    };
     int it = 0, piece = 0;
     for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
       if (*abort_flag) return;
@@ -238,46 +285,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       const int L1 = a.seqlen[p.b] + 1;
       float m_run = -INFINITY, l_run = 0.f;
       const int nt = p.t1 - p.t0;
+      uint32_t mine[32];
+      if (nt > 0 && !send(it, mine)) return;
       for (int k = 0; k < nt; ++k) {
         const int g = it + k;
         const int t = p.t0 + k;
-        // ---- partial scores of this CTA's columns
-        if (!mbar_wait(s_full, g & 1, wc)) return;
-        tc_fence_after();
-        uint32_t sr[64];
-        tmem_ld32(tl + kTmemS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(tl + kTmemS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(s_free);
-        uint32_t mine[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) mine[j] = pack_half2(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1]));
-        // ---- exchange with the partner CTA
-        if (!mbar_wait<true>(x_free, (g & 1) ^ 1, wc)) return;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          st_cluster_v4(x_row_peer + ((i ^ sw) << 4), make_uint4(mine[4 * i], mine[4 * i + 1], mine[4 * i + 2], mine[4 * i + 3]));
-        mbar_arrive_remote(xfull_peer);
-        if (!mbar_wait<true>(x_full, g & 1, wc)) return;
+        // the next tile's partial goes out before this tile's partner half is awaited,
+        // so the exchange latency overlaps the softmax of this tile
+        uint32_t nxt[32];
+        if (k + 1 < nt && !send(g + 1, nxt)) return;
+        const int slot = g & 1;
+        if (!mbar_wait<true>(&x_full[slot], (g >> 1) & 1, wc)) return;
         uint32_t theirs[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const uint4 v = ld_shared_v4(x_row + ((i ^ sw) << 4));
+          const uint4 v = ld_shared_v4(x_row + slot * kXBytes + ((i ^ sw) << 4));
           theirs[4 * i] = v.x; theirs[4 * i + 1] = v.y; theirs[4 * i + 2] = v.z; theirs[4 * i + 3] = v.w;
         }
-        mbar_arrive_remote(xfree_peer);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(xfree_peer + slot * 8);
         // ---- full scores (same bits in both CTAs), masked beyond the sequence
         const int valid = min(64, L1 - t * 64);
-        float sc[64];
         float mt = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const float2 x = unpack_half2(mine[j]), y = unpack_half2(theirs[j]);
           const float s0 = (2 * j < valid) ? x.x + y.x : -INFINITY;
           const float s1 = (2 * j + 1 < valid) ? x.y + y.y : -INFINITY;
-          sc[2 * j] = s0;
-          sc[2 * j + 1] = s1;
           mt = fmaxf(mt, fmaxf(s0, s1));
         }
         float m_new = m_run, alpha = 1.f;
@@ -293,7 +327,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         float lsum = 0.f;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(ex2_approx(sc[2 * j] - m_new), ex2_approx(sc[2 * j + 1] - m_new));
+          const float2 x = unpack_half2(mine[j]), y = unpack_half2(theirs[j]);
+          const float s0 = (2 * j < valid) ? x.x + y.x : -INFINITY;
+          const float s1 = (2 * j + 1 < valid) ? x.y + y.y : -INFINITY;
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(ex2_approx(s0 - m_new), ex2_approx(s1 - m_new));
           const float2 f = __bfloat1622float2(b2);
           lsum += f.x + f.y;
           pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
@@ -330,6 +367,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(p_full);
+        if (k + 1 < nt) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) mine[j] = nxt[j];
+        }
       }
       // ---- epilogue of the piece: unnormalised O_r, m, l
       if (!mbar_wait(o_done, piece & 1, wc)) return;
@@ -355,7 +396,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       ++piece;
     });
   }
-  // ---- teardown: every MMA retired, the partner no longer writes into this CTA
+  // ---- teardown: every MMA retired, the partner no longer writes into this CTA.
+  // The next kernel is released only now: its CTAs would otherwise sit on
+  // these SMs during the main loop.
+  if (threadIdx.x == 0) griddep_launch_dependents();
   if (warp == 1) {
     __syncwarp();
     if (lane == 0) {  // bounded, and not cut short by an abort: TMEM is freed only after the MMAs retire

@@ -109,17 +109,15 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   const uint32_t tmem = *tmem_slot;
   WaitCtx wc{args.status, abort_flag};
 
+  if (threadIdx.x == 0) griddep_launch_dependents();
   if (warp == 0) {
     if (elect_one()) {
       const uint64_t polA = policy_evict_first();
       const uint64_t polB = policy_evict_last();
       const uint32_t bytesA = A_MN ? 16384u : static_cast<uint32_t>(args.boxA_rows[seg]) * 128u;
       const uint32_t bytesB = static_cast<uint32_t>(args.boxB_rows) * 128u;
-      for (int i = 0; i < nk; ++i) {
+      auto load_a = [&](int i) {
         const int s = i % STAGES;
-        const uint32_t ph = (i / STAGES) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1, wc)) break;
-        mbar_arrive_expect_tx(&full[s], bytesA + bytesB);
         const int kb = kb0 + i;
         uint8_t* a = sA + s * L::kA;
         if (A_MN) {
@@ -131,7 +129,26 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         } else {
           tma_load_2d(a, &args.mapA[seg], &full[s], kb * 64, m0, polA);
         }
-        tma_load_2d(sB + s * L::kB, &args.mapB, &full[s], head * args.b_head_stride + kb * 64, nt * BN, polB);
+      };
+      auto load_b = [&](int i) {
+        const int s = i % STAGES;
+        tma_load_2d(sB + s * L::kB, &args.mapB, &full[s], head * args.b_head_stride + (kb0 + i) * 64, nt * BN, polB);
+      };
+      // Weights do not depend on earlier kernels: the first stages of A are
+      // fetched before waiting for the kernel that produces X.
+      const int pre = nk < STAGES ? nk : STAGES;
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(&full[i], bytesA + bytesB);
+        load_a(i);
+      }
+      griddep_wait();
+      for (int i = 0; i < pre; ++i) load_b(i);
+      for (int i = pre; i < nk; ++i) {
+        const int s = i % STAGES;
+        if (!mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, wc)) break;
+        mbar_arrive_expect_tx(&full[s], bytesA + bytesB);
+        load_a(i);
+        load_b(i);
       }
     }
   } else if (warp == 1) {
@@ -170,14 +187,17 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       const double inv_freq = epi_inv_freq(e, args.tok, m);
       bool do_epi = true;
       if (args.splits > 1) {
-        float* my = args.partials + (static_cast<long long>(tile_id) * args.splits + split) * (BN * 128);
+        // partial tile layout: [BN/4 column groups][128 rows][4], so a warp moves 512
+        // contiguous bytes per float4 access
+        float4* my = reinterpret_cast<float4*>(args.partials + (static_cast<long long>(tile_id) * args.splits + split) * (BN * 128));
 #pragma unroll 1
         for (int c = 0; c < BN; c += 16) {
           float v[16];
           tmem_ld16(trow + c, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) my[(c + j) * 128 + row] = v[j];
+          for (int q = 0; q < 4; ++q)
+            my[((c >> 2) + q) * 128 + row] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         }
         __threadfence();
         named_bar_sync(1, 128);
@@ -198,17 +218,28 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
           tmem_ld16(trow + c, v);
           tmem_wait_ld();
           if (args.splits > 1) {
+            // sum in split order (deterministic); own split from TMEM, the others from L2
             float acc[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+            const float4* base = reinterpret_cast<const float4*>(args.partials + static_cast<long long>(tile_id) * args.splits * (BN * 128));
+#pragma unroll 4
             for (int s = 0; s < args.splits; ++s) {
+              float4 t[4];
               if (s == split) {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) acc[j] += v[j];
+                for (int q = 0; q < 4; ++q) t[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
               } else {
-                const float* p = args.partials + (static_cast<long long>(tile_id) * args.splits + s) * (BN * 128);
+                const float4* p = base + static_cast<long long>(s) * (BN * 32);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) acc[j] += ld_cg_f32(p + (c + j) * 128 + row);
+                for (int q = 0; q < 4; ++q) t[q] = __ldcg(p + ((c >> 2) + q) * 128 + row);
+              }
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                acc[4 * q] += t[q].x;
+                acc[4 * q + 1] += t[q].y;
+                acc[4 * q + 2] += t[q].z;
+                acc[4 * q + 3] += t[q].w;
               }
             }
 #pragma unroll

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "attn_decode_tc.cuh"
+#include "attn_prefill_tc.cuh"
 #include "gemm_tc.cuh"
 #include "simt.cuh"
 
@@ -127,10 +128,30 @@ struct Ctx {
   int* status;
   cudaStream_t st;
   int num_sms;
+  bool pdl = false;  // chain the call's kernels with programmatic dependent launch
 };
 
+// Launches `kern` on the call's stream; with pdl the kernel may begin while
+// its predecessor drains (every kernel here calls griddep_wait() before it
+// reads or writes anything an earlier kernel touches).
+template <typename... KArgs, typename... Args>
+mla_status launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                  Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 template <int BN, bool AMN, int STAGES>
-mla_status launch_tc(const GemmArgs& a, dim3 grid, cudaStream_t st) {
+mla_status launch_tc(const GemmArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
   constexpr int smem = GemmSmem<BN, STAGES>::kBytes;
   auto kern = gemm_tc_kernel<BN, AMN, STAGES>;
   static bool attr_set = false;  // idempotent attribute set; races are harmless
@@ -139,17 +160,16 @@ mla_status launch_tc(const GemmArgs& a, dim3 grid, cudaStream_t st) {
       return MLA_ERR_CUDA;
     attr_set = true;
   }
-  kern<<<grid, 192, smem, st>>>(a);
-  return cudaPeekAtLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return launch(kern, grid, dim3(192), smem, st, pdl, a);
 }
 
 template <bool AMN>
-mla_status launch_tc_bn(int bn, const GemmArgs& a, dim3 grid, cudaStream_t st) {
+mla_status launch_tc_bn(int bn, const GemmArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
   switch (bn) {
-    case 32: return launch_tc<32, AMN, 5>(a, grid, st);
-    case 64: return launch_tc<64, AMN, 4>(a, grid, st);
-    case 128: return launch_tc<128, AMN, 3>(a, grid, st);
-    default: return launch_tc<256, AMN, 4>(a, grid, st);
+    case 32: return launch_tc<32, AMN, 5>(a, grid, st, pdl);
+    case 64: return launch_tc<64, AMN, 4>(a, grid, st, pdl);
+    case 128: return launch_tc<128, AMN, 3>(a, grid, st, pdl);
+    default: return launch_tc<256, AMN, 4>(a, grid, st, pdl);
   }
 }
 
@@ -208,7 +228,8 @@ mla_status run_gemm_tc(const Ctx& c, const GemmSpec& g) {
   a.partials = reinterpret_cast<float*>(c.ws + c.L.gpart);
   a.counters = reinterpret_cast<int*>(c.ws + c.L.counters);
   dim3 grid(m_tiles, n_tiles, splits);
-  return g.mode == GEMM_HEAD_MNMAJOR ? launch_tc_bn<true>(bn, a, grid, c.st) : launch_tc_bn<false>(bn, a, grid, c.st);
+  return g.mode == GEMM_HEAD_MNMAJOR ? launch_tc_bn<true>(bn, a, grid, c.st, c.pdl)
+                                     : launch_tc_bn<false>(bn, a, grid, c.st, c.pdl);
 }
 
 template <typename T>
@@ -382,7 +403,7 @@ void attn_event(cudaEvent_t e, cudaStream_t st) {
 
 mla_status launch_attn_decode_tc(const __nv_bfloat16* qlat, const mla_cache* cache, const int32_t* seqlen,
                                  const int* tile_start, const int* seg_start, int B, int W, int n_h, float* o_part,
-                                 float* ml, int* status, cudaStream_t st) {
+                                 float* ml, int* status, cudaStream_t st, bool pdl) {
   AttnArgs a;
   memset(&a, 0, sizeof(a));
   if (cache->n_rows > (1ll << 31) - 128) return MLA_ERR_UNSUPPORTED;  // tile rows are int32 TMA coordinates
@@ -405,8 +426,11 @@ mla_status launch_attn_decode_tc(const __nv_bfloat16* qlat, const mla_cache* cac
       return MLA_ERR_CUDA;
     attr_set = true;
   }
-  attn_decode_tc_kernel<<<2 * W, 192, attn::kSmem, st>>>(a);
-  return cudaPeekAtLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return launch(attn_decode_tc_kernel, dim3(2 * W), dim3(192), attn::kSmem, st, pdl, a);
+}
+
+bool prefill_tc_ok(const mla_dims& d) {
+  return d.dtype == MLA_BF16 && d.d_h == 128 && d.d_R == 64 && tc_gemm_ok(d);
 }
 
 bool attn_tc_ok(const mla_dims& d) {
@@ -527,15 +551,15 @@ mla_status mla_decode(const mla_dims* dims, const mla_weights* w, const void* h,
   tk.pos = seqlen;  // the new token of sequence b sits at position L_b
   (void)es;
 
-  if (cudaMemsetAsync(ws + c.L.counters, 0, kMaxCounters * sizeof(int), c.st) != cudaSuccess) return MLA_ERR_CUDA;
-
-  // ---- attention plan (device side: reads seqlen, no host sync)
+  // ---- attention plan (device side: reads seqlen, no host sync); also zeroes the split-K tickets
   const bool tc_attn = attn_tc_ok(d);
   const int tile_tokens = tc_attn ? kAttnTileTokens : 64;
   int W = tc_attn ? std::min(kMaxWorkers, c.num_sms / 2) : std::min(kMaxWorkers, c.num_sms * 2);
   if (W < 1) W = 1;
-  plan_kernel<<<1, 1024, 0, c.st>>>(seqlen, B, tile_tokens, W, tile_start, seg_start, c.status);
-  if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  c.pdl = tc_gemm_ok(d);
+  if ((s = launch(plan_kernel, dim3(1), dim3(1024), 0, c.st, c.pdl, seqlen, B, tile_tokens, W, tile_start, seg_start,
+                  c.status, reinterpret_cast<int*>(ws + c.L.counters), kMaxCounters)) != MLA_OK)
+    return s;
 
   // ---- a1 (+a2): down-projections from h, cache append of the new token
   {
@@ -610,7 +634,7 @@ mla_status mla_decode(const mla_dims* dims, const mla_weights* w, const void* h,
   attn_event(g_attn_begin, c.st);
   if (tc_attn) {
     if ((s = launch_attn_decode_tc(reinterpret_cast<const __nv_bfloat16*>(qlat), cache, seqlen, tile_start, seg_start,
-                                   B, W, d.n_h, opart, ml, c.status, c.st)) != MLA_OK)
+                                   B, W, d.n_h, opart, ml, c.status, c.st, c.pdl)) != MLA_OK)
       return s;
   } else {
     const size_t shm = (row + 4 * d.d_c + 8) * sizeof(float);
@@ -629,11 +653,12 @@ mla_status mla_decode(const mla_dims* dims, const mla_weights* w, const void* h,
   {
     dim3 grid(B, d.n_h);
     if (d.dtype == MLA_FP32)
-      combine_kernel<float><<<grid, 128, 0, c.st>>>(opart, ml, seg_start, d.n_h, d.d_c, static_cast<float*>(olat));
+      s = launch(combine_kernel<float>, grid, dim3(128), 0, c.st, c.pdl, opart, ml, seg_start, d.n_h, d.d_c,
+                 static_cast<float*>(olat));
     else
-      combine_kernel<__nv_bfloat16><<<grid, 128, 0, c.st>>>(opart, ml, seg_start, d.n_h, d.d_c,
-                                                           static_cast<__nv_bfloat16*>(olat));
-    if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
+      s = launch(combine_kernel<__nv_bfloat16>, grid, dim3(128), 0, c.st, c.pdl, opart, ml, seg_start, d.n_h, d.d_c,
+                 static_cast<__nv_bfloat16*>(olat));
+    if (s != MLA_OK) return s;
   }
   // ---- a7: absorbed W_UV on the latent output: o_i = W_UV_i o_lat_i
   {
@@ -798,7 +823,29 @@ extern "C" mla_status mla_prefill(const mla_dims* dims, const mla_weights* w, co
   }
   // ---- p4: causal attention per head
   attn_event(g_attn_begin, c.st);
-  {
+  if (prefill_tc_ok(d)) {
+    PrefillArgs a;
+    memset(&a, 0, sizeof(a));
+    if (!make_map_2d(&a.map_q, qp, static_cast<long long>(d.n_h) * dq, T, static_cast<long long>(d.n_h) * dq, 128) ||
+        !make_map_2d(&a.map_kc, kc, HD, S, HD, 128) || !make_map_2d(&a.map_kr, rows, row, S, row, 128) ||
+        !make_map_2d(&a.map_v, vv, HD, S, HD, 128))
+      return MLA_ERR_CUDA;
+    a.out = static_cast<__nv_bfloat16*>(att);
+    a.T = T;
+    a.start_pos = start_pos;
+    a.n_h = d.n_h;
+    a.n_qt = (T + pf::kQ - 1) / pf::kQ;
+    a.status = c.status;
+    static bool attr_set = false;
+    if (!attr_set) {
+      if (cudaFuncSetAttribute(attn_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pf::kSmem) !=
+          cudaSuccess)
+        return MLA_ERR_CUDA;
+      attr_set = true;
+    }
+    attn_prefill_tc_kernel<<<dim3(a.n_qt, d.n_h), 192, pf::kSmem, c.st>>>(a);
+    if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  } else {
     const size_t shm = (dq + 4 * d.d_h + 8) * sizeof(float);
     dim3 grid(T, d.n_h);
     if (d.dtype == MLA_FP32)

@@ -65,9 +65,13 @@ __host__ __device__ __forceinline__ long long worker_begin(int w, long long T, i
 }
 
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seqlen, int B, int tile_tokens, int W,
-                                                    int* tile_start, int* seg_start, int* status) {
+                                                    int* tile_start, int* seg_start, int* status, int* counters,
+                                                    int n_counters) {
   __shared__ long long s_scan[1024];
   __shared__ long long s_base;
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  for (int i = threadIdx.x; i < n_counters; i += 1024) counters[i] = 0;  // split-K tickets of this call
   // pass 1: cumulative tiles
   if (threadIdx.x == 0) s_base = 0;
   __syncthreads();
@@ -230,6 +234,8 @@ __global__ void __launch_bounds__(128) simt_decode_attn_kernel(
 template <typename T>
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ o_part, const float* __restrict__ ml_part,
                                                      const int* seg_start, int n_h, int d_c, T* __restrict__ olat) {
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch_dependents();
   const int b = blockIdx.x, h = blockIdx.y;
   const int s0 = seg_start[b], s1 = seg_start[b + 1];
   float M = -INFINITY;
