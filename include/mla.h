@@ -96,7 +96,10 @@ typedef struct {
 /* Bytes of workspace needed by mla_decode for batches up to `max_batch` and by
  * mla_cache_append / mla_prefill for up to `max_tokens` tokens per call.  The
  * workspace is caller-owned device memory (256-byte aligned); one workspace
- * must not be used by two calls that run at the same time. */
+ * must not be used by two calls that run at the same time.  Its first 256
+ * bytes hold the device status word: zero them once when the workspace is
+ * created (mla_get_device_status clears the word after reading a fault).  The
+ * rest may hold anything; the calls never read what they did not write. */
 size_t mla_workspace_bytes(const mla_dims* dims, int max_batch, int max_tokens);
 
 /* Cache append (the cache-write half of App. C): for t in [0, T),

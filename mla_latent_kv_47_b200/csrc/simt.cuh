@@ -52,11 +52,14 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const __grid_constant__ 
 }
 
 // ---------------------------------------------------------------- planner
-// Splits the attention work of a decode batch into W contiguous ranges of
-// tiles (`tile_tokens` tokens of one sequence each).  Outputs, for every
-// sequence b: tile_start[b] (cumulative tiles, [B+1]) and seg_start[b]
-// (cumulative number of (worker, sequence) pieces, [B+1]).  The piece of
-// worker w on sequence b is partial slot seg_start[b] + w - worker_of(tile_start[b]).
+// Splits the attention work of a decode batch into contiguous ranges of tiles
+// (`tile_tokens` tokens of one sequence each), one range per worker.  With T
+// tiles in all, the first We = min(W, T) workers each get at least one tile
+// and the rest none, so every worker counted for a sequence really writes its
+// partial slot.  Outputs, for every sequence b: tile_start[b] (cumulative
+// tiles, [B+1]) and seg_start[b] (cumulative number of (worker, sequence)
+// pieces, [B+1]).  The piece of worker w on sequence b is partial slot
+// seg_start[b] + w - worker_of(tile_start[b]).
 __host__ __device__ __forceinline__ int worker_of_tile(long long t, long long T, int W) {
   return static_cast<int>(((t + 1) * W + T - 1) / T) - 1;
 }
@@ -98,6 +101,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seqlen, int B
   }
   if (threadIdx.x == 0) tile_start[0] = 0;
   const long long T = s_base;
+  const int We = static_cast<int>(T < W ? T : W);  // workers that get tiles
   __syncthreads();
   // pass 2: pieces per sequence
   if (threadIdx.x == 0) s_base = 0;
@@ -108,7 +112,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seqlen, int B
     if (b < B) {
       const long long t0 = (b == 0) ? 0 : tile_start[b];
       const long long t1 = tile_start[b + 1];
-      v = worker_of_tile(t1 - 1, T, W) - worker_of_tile(t0, T, W) + 1;
+      v = worker_of_tile(t1 - 1, T, We) - worker_of_tile(t0, T, We) + 1;
     }
     s_scan[threadIdx.x] = v;
     __syncthreads();
@@ -137,7 +141,9 @@ template <typename F>
 __device__ __forceinline__ void for_each_piece(int w, int W, int B, const int* tile_start, const int* seg_start, F&& f) {
   const long long T = tile_start[B];
   if (T <= 0) return;
-  const long long r0 = worker_begin(w, T, W), r1 = worker_begin(w + 1, T, W);
+  const int We = static_cast<int>(T < W ? T : W);
+  if (w >= We) return;
+  const long long r0 = worker_begin(w, T, We), r1 = worker_begin(w + 1, T, We);
   if (r0 >= r1) return;
   int lo = 0, hi = B - 1;  // first b with tile_start[b+1] > r0
   while (lo < hi) {
@@ -150,7 +156,7 @@ __device__ __forceinline__ void for_each_piece(int w, int W, int B, const int* t
     p.b = b;
     p.t0 = static_cast<int>(max(r0, s0) - s0);
     p.t1 = static_cast<int>(min(r1, s1) - s0);
-    p.slot = seg_start[b] + (w - worker_of_tile(s0, T, W));
+    p.slot = seg_start[b] + (w - worker_of_tile(s0, T, We));
     f(p);
   }
 }
