@@ -153,6 +153,41 @@ const char* mla_status_string(mla_status s);
  * unknown id or invalid dims. */
 size_t mla_workspace_offset(const mla_dims* dims, int max_batch, int max_tokens, int which);
 
+/* ---------------------------------------------------------------------------
+ * Decode step that allocates nothing.  No counterpart in the paper: this is a
+ * deployment convenience around mla_decode.
+ *
+ * Some callers cannot allocate device memory when they call into this library,
+ * so they cannot hand it a workspace: for example an engine plugin that is given
+ * only its input and output buffers, or a latency-critical path where cudaMalloc
+ * (which can synchronise the whole device) is not allowed.  This entry point
+ * takes the same arguments as mla_decode minus the workspace and computes the
+ * same u.  Its scratch is one file-scope __device__ array of
+ * MLA_STATIC_SCRATCH_BYTES that every GPU which loads this library holds until
+ * the process exits; the call itself allocates nothing (no cudaMalloc, no
+ * cudaFree, no allocating library routine).
+ *
+ *  - Limit: the decode scratch of batch B must fit in the array.  At
+ *    DeepSeek-V2 dims it is about 0.35 MB x B (per-token intermediates)
+ *    + 0.26 MB x (B + SMs/2) (attention partials) + 0.15 MB x (split-K tile
+ *    width, 32..256), so B up to 101 on a 148-SM B200; V2-Lite dims allow far
+ *    larger batches.  A batch that does not fit returns MLA_ERR_WORKSPACE with
+ *    nothing enqueued.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current).  Make that first call outside any
+ *    stream capture.
+ *  - All calls share the one array, and it keeps the previous call's contents;
+ *    each call clears what must start at zero.  Calls whose work overlaps on the
+ *    GPU (several streams or host threads) race on the array.
+ *  - Faults found on the device are not reported (there is no workspace for
+ *    mla_get_device_status); the variant's status word is cleared at each call.
+ */
+#define MLA_STATIC_SCRATCH_BYTES (96u << 20)
+mla_status mla_decode_static(const mla_dims* dims, const mla_weights* w,
+                             const void* h, int B,
+                             const mla_cache* cache, const int32_t* seqlen,
+                             float* u, mla_stream_t stream);
+
 /* Diagnostic timing hook.  While set, every mla_decode / mla_prefill call
  * records CUDA event `begin` (a cudaEvent_t) on its stream just before the
  * launch of its attention kernel and `end` just after it, so a caller can time

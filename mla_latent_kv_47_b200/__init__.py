@@ -22,7 +22,8 @@ FAULT_CAPACITY, FAULT_WAIT_TIMEOUT, FAULT_PLAN = 1, 2, 4
 WS_CQ, WS_QC, WS_QLAT, WS_OLAT, WS_O = range(5)
 
 EXPORTS = ("mla_workspace_bytes", "mla_cache_append", "mla_decode", "mla_prefill",
-           "mla_get_device_status", "mla_status_string", "mla_workspace_offset", "mla_set_attention_events")
+           "mla_get_device_status", "mla_status_string", "mla_workspace_offset", "mla_set_attention_events",
+           "mla_decode_static")
 
 
 class MLAError(RuntimeError):
@@ -66,6 +67,8 @@ def _load():
     lib.mla_get_device_status.restype = i32
     lib.mla_status_string.argtypes = [i32]
     lib.mla_status_string.restype = ctypes.c_char_p
+    lib.mla_decode_static.argtypes = [P(Dims), P(Weights), vp, i32, P(Cache), vp, vp, vp]
+    lib.mla_decode_static.restype = i32
     lib.mla_set_attention_events.argtypes = [vp, vp]
     lib.mla_set_attention_events.restype = None
     return lib
@@ -161,6 +164,14 @@ def prefill(dims, weights, h, start_pos, cache, seq, u, workspace, stream=None):
     _check(_lib().mla_prefill(ctypes.byref(dims), ctypes.byref(weights), _ptr(h), int(h.shape[0]), int(start_pos),
                            ctypes.byref(cache), int(seq), _ptr(u), _ptr(workspace), workspace.numel(),
                            _stream(stream)), "mla_prefill")
+
+
+def decode_static(dims, weights, h, cache, seqlen, u, stream=None):
+    """mla_decode without a workspace: the library's static device scratch is used."""
+    assert seqlen.dtype == torch.int32 and u.dtype == torch.float32
+    _check(_lib().mla_decode_static(ctypes.byref(dims), ctypes.byref(weights), _ptr(h), int(h.shape[0]),
+                                    ctypes.byref(cache), _ptr(seqlen), _ptr(u), _stream(stream)),
+           "mla_decode_static")
 
 
 def device_status(workspace, stream=None):

@@ -38,7 +38,9 @@ int row_elems(const mla_dims& d) { return d.d_c + d.d_R; }
 
 int pick_bn(int N) { return N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256; }
 
-Layout make_layout(const mla_dims& d, int max_batch, int max_tokens) {
+// gpart_bn: widest split-K tile the call may use; workers: attention workers
+// (partial slots beyond the batch).
+Layout make_layout_sized(const mla_dims& d, int max_batch, int max_tokens, int gpart_bn, int workers) {
   Layout L{};
   const size_t es = elem_size(d);
   const size_t B = static_cast<size_t>(max_batch < 1 ? 1 : max_batch);
@@ -48,7 +50,7 @@ Layout make_layout(const mla_dims& d, int max_batch, int max_tokens) {
   auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, kAlign); return o; };
   L.status = take(256);
   L.counters = take(kMaxCounters * sizeof(int));
-  L.gpart = take(static_cast<size_t>(kMaxGemmCtas) * 256 * 128 * sizeof(float));
+  L.gpart = take(static_cast<size_t>(kMaxGemmCtas) * gpart_bn * 128 * sizeof(float));
   L.base_end = off;
   L.tile_start = take((B + 1) * sizeof(int));
   L.seg_start = take((B + 1) * sizeof(int));
@@ -57,8 +59,8 @@ Layout make_layout(const mla_dims& d, int max_batch, int max_tokens) {
   L.qlat = take(B * nh * row * es);
   L.olat = take(B * nh * d.d_c * es);
   L.o = take(B * nh * dh * es);
-  L.opart = take((B + kMaxWorkers) * nh * d.d_c * sizeof(float));
-  L.ml = take((B + kMaxWorkers) * nh * 2 * sizeof(float));
+  L.opart = take((B + workers) * nh * d.d_c * sizeof(float));
+  L.ml = take((B + workers) * nh * 2 * sizeof(float));
   L.decode_end = off;
   off = L.base_end;
   L.p_cq = take(T * (d.d_cq ? d.d_cq : 1) * es);
@@ -69,6 +71,10 @@ Layout make_layout(const mla_dims& d, int max_batch, int max_tokens) {
   L.p_out = take(T * nh * dh * es);
   L.prefill_end = off;
   return L;
+}
+
+Layout make_layout(const mla_dims& d, int max_batch, int max_tokens) {
+  return make_layout_sized(d, max_batch, max_tokens, 256, kMaxWorkers);
 }
 
 // ------------------------------------------------------------------ tensor maps
@@ -437,104 +443,19 @@ bool attn_tc_ok(const mla_dims& d) {
   return kAttnTcReady && d.dtype == MLA_BF16 && d.n_h <= 128 && d.d_c == 512 && d.d_R == 64;
 }
 
-}  // namespace
-
-// ====================================================================== C ABI
-extern "C" {
-
-void mla_set_attention_events(void* begin, void* end) {
-  g_attn_begin = static_cast<cudaEvent_t>(begin);
-  g_attn_end = static_cast<cudaEvent_t>(end);
+// Attention workers of a decode call: one 2-CTA cluster per SM pair on the
+// tensor-core path, two CTAs per SM on the CUDA-core path.
+int decode_workers(const mla_dims& d, int num_sms) {
+  const int W = attn_tc_ok(d) ? std::min(kMaxWorkers, num_sms / 2) : std::min(kMaxWorkers, num_sms * 2);
+  return W < 1 ? 1 : W;
 }
 
-size_t mla_workspace_bytes(const mla_dims* dims, int max_batch, int max_tokens) {
-  if (check_dims(dims) != MLA_OK) return 0;
-  const Layout L = make_layout(*dims, max_batch, max_tokens);
-  return std::max(L.decode_end, L.prefill_end);
-}
-
-size_t mla_workspace_offset(const mla_dims* dims, int max_batch, int max_tokens, int which) {
-  if (check_dims(dims) != MLA_OK) return static_cast<size_t>(-1);
-  const Layout L = make_layout(*dims, max_batch, max_tokens);
-  switch (which) {
-    case 0: return L.cq;
-    case 1: return L.qc;
-    case 2: return L.qlat;
-    case 3: return L.olat;
-    case 4: return L.o;
-    default: return static_cast<size_t>(-1);
-  }
-}
-
-const char* mla_status_string(mla_status s) {
-  switch (s) {
-    case MLA_OK: return "ok";
-    case MLA_ERR_INVALID_ARG: return "invalid argument";
-    case MLA_ERR_UNSUPPORTED: return "unsupported dims or dtype";
-    case MLA_ERR_MISALIGNED: return "pointer not 16-byte aligned (workspace: 256-byte)";
-    case MLA_ERR_WORKSPACE: return "workspace missing or too small";
-    case MLA_ERR_CUDA: return "CUDA error";
-    case MLA_ERR_DEVICE_FAULT: return "device fault reported by a kernel";
-  }
-  return "unknown status";
-}
-
-mla_status mla_get_device_status(void* workspace, mla_stream_t stream, int* detail) {
-  if (!workspace) return MLA_ERR_WORKSPACE;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  int v = 0;
-  // the status word is the first int of every layout
-  if (cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return MLA_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
-  if (detail) *detail = v;
-  if (v != 0) {
-    if (cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess) return MLA_ERR_CUDA;
-    if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
-    return MLA_ERR_DEVICE_FAULT;
-  }
-  return MLA_OK;
-}
-
-mla_status mla_cache_append(const mla_dims* dims, const mla_weights* w, const void* h, int T, const int32_t* seq_idx,
-                            const int32_t* pos, const mla_cache* cache, void* workspace, size_t workspace_bytes,
-                            mla_stream_t stream) {
-  mla_status s = check_dims(dims);
-  if (s != MLA_OK) return s;
-  if ((s = check_weights(dims, w)) != MLA_OK) return s;
-  if ((s = check_cache(cache)) != MLA_OK) return s;
-  if (T < 0) return MLA_ERR_INVALID_ARG;
-  if (T == 0) return MLA_OK;
-  if (!h || !seq_idx || !pos) return MLA_ERR_INVALID_ARG;
-  if (!aligned16(h)) return MLA_ERR_MISALIGNED;
-  Ctx c;
-  if ((s = make_ctx(c, dims, 1, 1, REGION_BASE, workspace, workspace_bytes, stream)) != MLA_OK) return s;
-  const mla_dims& d = *dims;
-  GemmSpec g;
-  g.K = d.d_model;
-  g.a_ld = d.d_model;
-  g.X = h;
-  g.x_cols = d.d_model;
-  g.x_ld = d.d_model;
-  g.N = T;
-  g.tok = cache_tokens(d, cache);
-  g.tok.pos = pos;
-  g.tok.seq = seq_idx;
-  add_cache_segments(g, d, w);
-  if (cudaMemsetAsync(c.ws + c.L.counters, 0, kMaxCounters * sizeof(int), c.st) != cudaSuccess) return MLA_ERR_CUDA;
-  return run_gemm(c, g);
-}
-
-mla_status mla_decode(const mla_dims* dims, const mla_weights* w, const void* h, int B, const mla_cache* cache,
-                      const int32_t* seqlen, float* u, void* workspace, size_t workspace_bytes, mla_stream_t stream) {
-  mla_status s = check_dims(dims);
-  if (s != MLA_OK) return s;
-  if ((s = check_weights(dims, w)) != MLA_OK) return s;
-  if ((s = check_cache(cache)) != MLA_OK) return s;
-  if (B <= 0 || !h || !seqlen || !u) return MLA_ERR_INVALID_ARG;
-  if (!aligned16(h) || !aligned16(u)) return MLA_ERR_MISALIGNED;
-  Ctx c;
-  if ((s = make_ctx(c, dims, B, 1, REGION_DECODE, workspace, workspace_bytes, stream)) != MLA_OK) return s;
-  const mla_dims& d = *dims;
+// The decode launch sequence (a1 .. a8 of the hot path) on an already checked
+// context; shared by mla_decode and the no-allocation variant.
+mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const mla_cache* cache,
+                      const int32_t* seqlen, float* u) {
+  const mla_dims& d = c.d;
+  mla_status s = MLA_OK;
   const int es = elem_size(d);
   const int row = row_elems(d);
   const long long HD = static_cast<long long>(d.n_h) * d.d_h;
@@ -554,8 +475,7 @@ mla_status mla_decode(const mla_dims* dims, const mla_weights* w, const void* h,
   // ---- attention plan (device side: reads seqlen, no host sync); also zeroes the split-K tickets
   const bool tc_attn = attn_tc_ok(d);
   const int tile_tokens = tc_attn ? kAttnTileTokens : 64;
-  int W = tc_attn ? std::min(kMaxWorkers, c.num_sms / 2) : std::min(kMaxWorkers, c.num_sms * 2);
-  if (W < 1) W = 1;
+  const int W = decode_workers(d, c.num_sms);
   c.pdl = tc_gemm_ok(d);
   if ((s = launch(plan_kernel, dim3(1), dim3(1024), 0, c.st, c.pdl, seqlen, B, tile_tokens, W, tile_start, seg_start,
                   c.status, reinterpret_cast<int*>(ws + c.L.counters), kMaxCounters)) != MLA_OK)
@@ -698,6 +618,106 @@ mla_status mla_decode(const mla_dims* dims, const mla_weights* w, const void* h,
     if ((s = run_gemm(c, g)) != MLA_OK) return s;
   }
   return MLA_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+void mla_set_attention_events(void* begin, void* end) {
+  g_attn_begin = static_cast<cudaEvent_t>(begin);
+  g_attn_end = static_cast<cudaEvent_t>(end);
+}
+
+size_t mla_workspace_bytes(const mla_dims* dims, int max_batch, int max_tokens) {
+  if (check_dims(dims) != MLA_OK) return 0;
+  const Layout L = make_layout(*dims, max_batch, max_tokens);
+  return std::max(L.decode_end, L.prefill_end);
+}
+
+size_t mla_workspace_offset(const mla_dims* dims, int max_batch, int max_tokens, int which) {
+  if (check_dims(dims) != MLA_OK) return static_cast<size_t>(-1);
+  const Layout L = make_layout(*dims, max_batch, max_tokens);
+  switch (which) {
+    case 0: return L.cq;
+    case 1: return L.qc;
+    case 2: return L.qlat;
+    case 3: return L.olat;
+    case 4: return L.o;
+    default: return static_cast<size_t>(-1);
+  }
+}
+
+const char* mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "ok";
+    case MLA_ERR_INVALID_ARG: return "invalid argument";
+    case MLA_ERR_UNSUPPORTED: return "unsupported dims or dtype";
+    case MLA_ERR_MISALIGNED: return "pointer not 16-byte aligned (workspace: 256-byte)";
+    case MLA_ERR_WORKSPACE: return "workspace missing or too small";
+    case MLA_ERR_CUDA: return "CUDA error";
+    case MLA_ERR_DEVICE_FAULT: return "device fault reported by a kernel";
+  }
+  return "unknown status";
+}
+
+mla_status mla_get_device_status(void* workspace, mla_stream_t stream, int* detail) {
+  if (!workspace) return MLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  // the status word is the first int of every layout
+  if (cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+  if (detail) *detail = v;
+  if (v != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess) return MLA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+    return MLA_ERR_DEVICE_FAULT;
+  }
+  return MLA_OK;
+}
+
+mla_status mla_cache_append(const mla_dims* dims, const mla_weights* w, const void* h, int T, const int32_t* seq_idx,
+                            const int32_t* pos, const mla_cache* cache, void* workspace, size_t workspace_bytes,
+                            mla_stream_t stream) {
+  mla_status s = check_dims(dims);
+  if (s != MLA_OK) return s;
+  if ((s = check_weights(dims, w)) != MLA_OK) return s;
+  if ((s = check_cache(cache)) != MLA_OK) return s;
+  if (T < 0) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (!h || !seq_idx || !pos) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h)) return MLA_ERR_MISALIGNED;
+  Ctx c;
+  if ((s = make_ctx(c, dims, 1, 1, REGION_BASE, workspace, workspace_bytes, stream)) != MLA_OK) return s;
+  const mla_dims& d = *dims;
+  GemmSpec g;
+  g.K = d.d_model;
+  g.a_ld = d.d_model;
+  g.X = h;
+  g.x_cols = d.d_model;
+  g.x_ld = d.d_model;
+  g.N = T;
+  g.tok = cache_tokens(d, cache);
+  g.tok.pos = pos;
+  g.tok.seq = seq_idx;
+  add_cache_segments(g, d, w);
+  if (cudaMemsetAsync(c.ws + c.L.counters, 0, kMaxCounters * sizeof(int), c.st) != cudaSuccess) return MLA_ERR_CUDA;
+  return run_gemm(c, g);
+}
+
+mla_status mla_decode(const mla_dims* dims, const mla_weights* w, const void* h, int B, const mla_cache* cache,
+                      const int32_t* seqlen, float* u, void* workspace, size_t workspace_bytes, mla_stream_t stream) {
+  mla_status s = check_dims(dims);
+  if (s != MLA_OK) return s;
+  if ((s = check_weights(dims, w)) != MLA_OK) return s;
+  if ((s = check_cache(cache)) != MLA_OK) return s;
+  if (B <= 0 || !h || !seqlen || !u) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(u)) return MLA_ERR_MISALIGNED;
+  Ctx c;
+  if ((s = make_ctx(c, dims, B, 1, REGION_DECODE, workspace, workspace_bytes, stream)) != MLA_OK) return s;
+  return decode_run(c, w, h, B, cache, seqlen, u);
 }
 
 }  // extern "C"
@@ -877,4 +897,60 @@ extern "C" mla_status mla_prefill(const mla_dims* dims, const mla_weights* w, co
     if ((s = run_gemm(c, g)) != MLA_OK) return s;
   }
   return MLA_OK;
+}
+
+// ====================================================================== decode without a workspace
+// Scratch of mla_decode_static: one file-scope device array per GPU that loads
+// this library, held until the process exits.  Host code must not pass the
+// array's name to a kernel (on the host it is only a stand-in); the device
+// address comes from cudaGetSymbolAddress, looked up once per device.
+namespace {
+
+static __device__ __align__(256) uint8_t g_static_scratch[MLA_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+mla_status static_scratch_address(int dev, void** out) {
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return MLA_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" mla_status mla_decode_static(const mla_dims* dims, const mla_weights* w, const void* h, int B,
+                                        const mla_cache* cache, const int32_t* seqlen, float* u,
+                                        mla_stream_t stream) {
+  mla_status s = check_dims(dims);
+  if (s != MLA_OK) return s;
+  if ((s = check_weights(dims, w)) != MLA_OK) return s;
+  if ((s = check_cache(cache)) != MLA_OK) return s;
+  if (B <= 0 || !h || !seqlen || !u) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(u)) return MLA_ERR_MISALIGNED;
+  Ctx c;
+  c.d = *dims;
+  c.st = reinterpret_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&c.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MLA_ERR_CUDA;
+  // exactly the space this batch uses on this device: split-K tiles of the
+  // batch's width, attention partials for B + (workers on this GPU) slots
+  c.L = make_layout_sized(*dims, B, 1, pick_bn(B), decode_workers(*dims, c.num_sms));
+  if (c.L.decode_end > MLA_STATIC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((s = static_scratch_address(dev, &scratch)) != MLA_OK) return s;
+  c.ws = static_cast<uint8_t*>(scratch);
+  c.status = reinterpret_cast<int*>(c.ws + c.L.status);
+  // the array keeps the previous call's contents: the status word is cleared
+  // here, the split-K tickets by the first kernel of the sequence
+  if (cudaMemsetAsync(c.status, 0, sizeof(int), c.st) != cudaSuccess) return MLA_ERR_CUDA;
+  return decode_run(c, w, h, B, cache, seqlen, u);
 }
