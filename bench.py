@@ -327,11 +327,13 @@ def run_ours(args):
             torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
+        launches0 = m.kernel_launches()
         t_start.record()
         for i in range(K):
             m.set_attention_events(ev_b[i], ev_e[i])
             step()
         t_end.record()
+        launches = m.kernel_launches() - launches0
         torch.cuda.synchronize()
     m.set_attention_events(None, None)
     barrier()
@@ -441,7 +443,7 @@ def run_ours(args):
                           "frac": roof_ms / ms, "latent_cache_gbs": cache_bytes / (ms * 1e-3) / 1e9},
         "e2e": {"value": world * B / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": K * (8 if d.d_cq else 7),
+        "gpu_launches": launches,
         "clocks": clk.summary(),
         "cpu_baseline": cpu_baseline,
         "prefill": prefill,

@@ -188,6 +188,11 @@ mla_status mla_decode_static(const mla_dims* dims, const mla_weights* w,
                              const mla_cache* cache, const int32_t* seqlen,
                              float* u, mla_stream_t stream);
 
+/* Diagnostic: number of kernels this library has launched in this process
+ * (all entry points, all threads).  The difference across a call counts the
+ * call's kernel launches. */
+unsigned long long mla_kernel_launches(void);
+
 /* Diagnostic timing hook.  While set, every mla_decode / mla_prefill call
  * records CUDA event `begin` (a cudaEvent_t) on its stream just before the
  * launch of its attention kernel and `end` just after it, so a caller can time

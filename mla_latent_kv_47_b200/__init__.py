@@ -23,7 +23,7 @@ WS_CQ, WS_QC, WS_QLAT, WS_OLAT, WS_O = range(5)
 
 EXPORTS = ("mla_workspace_bytes", "mla_cache_append", "mla_decode", "mla_prefill",
            "mla_get_device_status", "mla_status_string", "mla_workspace_offset", "mla_set_attention_events",
-           "mla_decode_static")
+           "mla_decode_static", "mla_kernel_launches")
 
 
 class MLAError(RuntimeError):
@@ -69,6 +69,8 @@ def _load():
     lib.mla_status_string.restype = ctypes.c_char_p
     lib.mla_decode_static.argtypes = [P(Dims), P(Weights), vp, i32, P(Cache), vp, vp, vp]
     lib.mla_decode_static.restype = i32
+    lib.mla_kernel_launches.argtypes = []
+    lib.mla_kernel_launches.restype = ctypes.c_ulonglong
     lib.mla_set_attention_events.argtypes = [vp, vp]
     lib.mla_set_attention_events.restype = None
     return lib
@@ -185,3 +187,8 @@ def set_attention_events(begin=None, end=None):
     """Bracket the attention kernel of the next calls with two torch.cuda.Event objects (None clears)."""
     _lib().mla_set_attention_events(ctypes.c_void_p(begin.cuda_event) if begin is not None else None,
                                  ctypes.c_void_p(end.cuda_event) if end is not None else None)
+
+
+def kernel_launches() -> int:
+    """Kernels launched by the library so far in this process (diagnostic)."""
+    return int(_lib().mla_kernel_launches())

@@ -55,7 +55,7 @@ __device__ __forceinline__ int tok_seq(const TokenMap& t, int n) {
 __device__ __forceinline__ double rope_inv_freq(int i, int d_R, double log2_base) {
   return exp2(-(2.0 * i / d_R) * log2_base);
 }
-__device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float& c, float& s) {
+__device__ __noinline__ void rope_cos_sin(int pos, double inv_freq, float& c, float& s) {
   const double two_pi_hi = 6.283185307179586;
   const double two_pi_lo = 2.4492935982947064e-16;
   double phi = static_cast<double>(pos) * inv_freq;
@@ -143,6 +143,53 @@ __device__ __forceinline__ void epi_apply(const Epi& e, const TokenMap& tk, int 
       store_elem<T>(e.out, static_cast<long long>(n) * e.ld + hh * e.hs + e.col0 + j, y * e.scale, e.out_f32);
       break;
     }
+  }
+}
+
+// Per-kind form of epi_apply, so that a chunk of outputs is dispatched once
+// (one switch per chunk instead of per element keeps the epilogue code small).
+template <int KIND, typename T>
+__device__ __forceinline__ void epi_one(const Epi& e, const TokenMap& tk, int m, int n, int head, float y, float yp,
+                                        double inv_freq, int* status) {
+  if (KIND == EPI_STORE) {
+    store_elem<T>(e.out, static_cast<long long>(n) * e.ld + e.col0 + m, y * e.scale, e.out_f32);
+  } else if (KIND == EPI_PER_HEAD) {
+    store_elem<T>(e.out, static_cast<long long>(n) * e.ld + head * e.hs + m, y * e.scale, e.out_f32);
+  } else if (KIND == EPI_HEADS) {
+    const int hh = m / e.dh, j = m % e.dh;
+    store_elem<T>(e.out, static_cast<long long>(n) * e.ld + hh * e.hs + e.col0 + j, y * e.scale, e.out_f32);
+  } else if (KIND == EPI_CACHE_CKV) {
+    const long long row = cache_row(tk, n, status);
+    if (row >= 0) store_elem<T>(tk.cache, row * tk.row_elems + m, y, 0);
+  } else {
+    epi_apply<T>(e, tk, m, n, head, y, yp, inv_freq, status);  // rotary kinds
+  }
+}
+
+// Applies the epilogue to outputs (m, n0 + j), j < NV, held by this thread;
+// whole warps call it (the rotary partner is a lane shuffle away).
+template <int KIND, int NV, typename T>
+__device__ __forceinline__ void epi_chunk(const Epi& e, const TokenMap& tk, int m, int n0, int head, const float* v,
+                                          int n_end, bool m_ok, double inv_freq, int* status) {
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const bool rot = (KIND == EPI_QLAT_ROPE || KIND == EPI_CACHE_KR || KIND == EPI_QP_ROPE);
+    const float yp = rot ? __shfl_xor_sync(0xffffffffu, v[j], 1) : 0.f;
+    if (n0 + j < n_end && m_ok) epi_one<KIND, T>(e, tk, m, n0 + j, head, v[j], yp, inv_freq, status);
+  }
+}
+
+template <int NV, typename T>
+__device__ __forceinline__ void epi_dispatch(const Epi& e, const TokenMap& tk, int m, int n0, int head, const float* v,
+                                             int n_end, bool m_ok, double inv_freq, int* status) {
+  switch (e.kind) {
+    case EPI_STORE: epi_chunk<EPI_STORE, NV, T>(e, tk, m, n0, head, v, n_end, m_ok, inv_freq, status); break;
+    case EPI_PER_HEAD: epi_chunk<EPI_PER_HEAD, NV, T>(e, tk, m, n0, head, v, n_end, m_ok, inv_freq, status); break;
+    case EPI_HEADS: epi_chunk<EPI_HEADS, NV, T>(e, tk, m, n0, head, v, n_end, m_ok, inv_freq, status); break;
+    case EPI_CACHE_CKV: epi_chunk<EPI_CACHE_CKV, NV, T>(e, tk, m, n0, head, v, n_end, m_ok, inv_freq, status); break;
+    case EPI_QLAT_ROPE: epi_chunk<EPI_QLAT_ROPE, NV, T>(e, tk, m, n0, head, v, n_end, m_ok, inv_freq, status); break;
+    case EPI_CACHE_KR: epi_chunk<EPI_CACHE_KR, NV, T>(e, tk, m, n0, head, v, n_end, m_ok, inv_freq, status); break;
+    default: epi_chunk<EPI_QP_ROPE, NV, T>(e, tk, m, n0, head, v, n_end, m_ok, inv_freq, status); break;
   }
 }
 

@@ -9,8 +9,9 @@
 // full-rate M=128 MMAs and the kernel streams the weights at HBM speed.
 // Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
 // issues tcgen05.mma, warps 2-5 run the epilogue (one TMEM lane per thread).
-// Split-K: CTAs of one output tile write fp32 partials; the last one to finish
-// (an atomic ticket, no waiting) sums them in split order and runs the epilogue.
+// Split-K: CTAs of one output tile write fp32 partials; a second, wide kernel
+// (gemm_splitk_epilogue_kernel) sums them in split order and runs the epilogue,
+// so the reduction is spread over the whole GPU instead of one CTA per tile.
 #pragma once
 #include "epilogue.cuh"
 
@@ -40,23 +41,27 @@ struct GemmArgs {
   int kb_total;                // K / 64
   int kb_per_split;
   int splits;
-  float* partials;             // [tiles][splits][BN][128] fp32 (splits > 1)
-  int* counters;               // [tiles] tickets, zero before the launch; reset by the last CTA
+  float* partials;             // [tiles][splits][BN/4][128][4] fp32 (splits > 1)
   int* status;
   TokenMap tok;
 };
 
-template <int BN, int STAGES>
+// One pipeline stage holds KBB consecutive 64-wide K blocks of A (128 rows)
+// and of X (BN rows): fewer, larger stages mean fewer barrier round trips and
+// longer runs of each weight row in flight.
+template <int BN, int STAGES, int KBB>
 struct GemmSmem {
-  static constexpr int kA = 16384;        // 128 rows x 128 B
-  static constexpr int kB = BN * 128;     // BN rows x 128 B
+  static constexpr int kSlabA = 16384;     // 128 rows x 128 B
+  static constexpr int kSlabB = BN * 128;  // BN rows x 128 B
+  static constexpr int kA = KBB * kSlabA;
+  static constexpr int kB = KBB * kSlabB;
   static constexpr int kStage = kA + kB;
   static constexpr int kBytes = 1024 + STAGES * kStage + 256;
 };
 
-template <int BN, bool A_MN, int STAGES>
+template <int BN, bool A_MN, int STAGES, int KBB>
 __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ GemmArgs args) {
-  using L = GemmSmem<BN, STAGES>;
+  using L = GemmSmem<BN, STAGES, KBB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
@@ -66,7 +71,6 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   uint64_t* accum = empty + STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* last_flag = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -85,7 +89,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   }
   const int kb0 = split * args.kb_per_split;
   const int kb1 = min(args.kb_total, kb0 + args.kb_per_split);
-  const int nk = kb1 - kb0;
+  const int nkb = kb1 - kb0;                 // K blocks of this CTA
+  const int nk = (nkb + KBB - 1) / KBB;      // pipeline stages of this CTA
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -116,10 +121,11 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       const uint64_t polB = policy_evict_last();
       const uint32_t bytesA = A_MN ? 16384u : static_cast<uint32_t>(args.boxA_rows[seg]) * 128u;
       const uint32_t bytesB = static_cast<uint32_t>(args.boxB_rows) * 128u;
-      auto load_a = [&](int i) {
+      auto stage_kbs = [&](int i) { return min(KBB, nkb - i * KBB); };
+      auto load_a = [&](int i, int j) {
         const int s = i % STAGES;
-        const int kb = kb0 + i;
-        uint8_t* a = sA + s * L::kA;
+        const int kb = kb0 + i * KBB + j;
+        uint8_t* a = sA + s * L::kA + j * L::kSlabA;
         if (A_MN) {
           const int y = head * args.head_rows + kb * 64;
           tma_load_2d(a, &args.mapA[0], &full[s], m0, y, polA);
@@ -130,25 +136,29 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
           tma_load_2d(a, &args.mapA[seg], &full[s], kb * 64, m0, polA);
         }
       };
-      auto load_b = [&](int i) {
+      auto load_b = [&](int i, int j) {
         const int s = i % STAGES;
-        tma_load_2d(sB + s * L::kB, &args.mapB, &full[s], head * args.b_head_stride + (kb0 + i) * 64, nt * BN, polB);
+        tma_load_2d(sB + s * L::kB + j * L::kSlabB, &args.mapB, &full[s],
+                    head * args.b_head_stride + (kb0 + i * KBB + j) * 64, nt * BN, polB);
       };
       // Weights do not depend on earlier kernels: the first stages of A are
       // fetched before waiting for the kernel that produces X.
       const int pre = nk < STAGES ? nk : STAGES;
       for (int i = 0; i < pre; ++i) {
-        mbar_arrive_expect_tx(&full[i], bytesA + bytesB);
-        load_a(i);
+        mbar_arrive_expect_tx(&full[i], stage_kbs(i) * (bytesA + bytesB));
+        for (int j = 0; j < stage_kbs(i); ++j) load_a(i, j);
       }
       griddep_wait();
-      for (int i = 0; i < pre; ++i) load_b(i);
+      for (int i = 0; i < pre; ++i)
+        for (int j = 0; j < stage_kbs(i); ++j) load_b(i, j);
       for (int i = pre; i < nk; ++i) {
         const int s = i % STAGES;
         if (!mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, wc)) break;
-        mbar_arrive_expect_tx(&full[s], bytesA + bytesB);
-        load_a(i);
-        load_b(i);
+        mbar_arrive_expect_tx(&full[s], stage_kbs(i) * (bytesA + bytesB));
+        for (int j = 0; j < stage_kbs(i); ++j) {
+          load_a(i, j);
+          load_b(i, j);
+        }
       }
     }
   } else if (warp == 1) {
@@ -159,13 +169,16 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         const uint32_t ph = (i / STAGES) & 1;
         if (!mbar_wait(&full[s], ph, wc)) break;
         tc_fence_after();
-        const uint32_t a_base = smem_u32(sA + s * L::kA);
-        const uint32_t b_base = smem_u32(sB + s * L::kB);
+        const int kbs = min(KBB, nkb - i * KBB);
+        for (int j = 0; j < kbs; ++j) {
+          const uint32_t a_base = smem_u32(sA + s * L::kA + j * L::kSlabA);
+          const uint32_t b_base = smem_u32(sB + s * L::kB + j * L::kSlabB);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint64_t ad = A_MN ? sdesc_sw128(a_base + k * 2048, 8192, 1024) : sdesc_sw128(a_base + k * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(b_base + k * 32, 16, 1024);
-          mma_ss(tmem, ad, bd, idesc, (i > 0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = A_MN ? sdesc_sw128(a_base + k * 2048, 8192, 1024) : sdesc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b_base + k * 32, 16, 1024);
+            mma_ss(tmem, ad, bd, idesc, (i > 0 || j > 0 || k > 0) ? 1u : 0u);
+          }
         }
         mma_commit(&empty[s]);
       }
@@ -182,13 +195,12 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     if (!*abort_flag) {
       const Epi& e = args.epi[seg];
       const int m = m0 + row;
-      const int rows_valid = args.seg_rows[seg];
+      const bool m_ok = m < args.seg_rows[seg];
       const int tile_id = mt + gridDim.x * nt;
-      const double inv_freq = epi_inv_freq(e, args.tok, m);
-      bool do_epi = true;
       if (args.splits > 1) {
-        // partial tile layout: [BN/4 column groups][128 rows][4], so a warp moves 512
-        // contiguous bytes per float4 access
+        // split-K: store this split's partial tile ([BN/4 column groups][128 rows][4],
+        // so a warp moves 512 contiguous bytes per float4); gemm_splitk_epilogue_kernel
+        // sums the splits in order and applies the epilogue
         float4* my = reinterpret_cast<float4*>(args.partials + (static_cast<long long>(tile_id) * args.splits + split) * (BN * 128));
 #pragma unroll 1
         for (int c = 0; c < BN; c += 16) {
@@ -199,58 +211,14 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
           for (int q = 0; q < 4; ++q)
             my[((c >> 2) + q) * 128 + row] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         }
-        __threadfence();
-        named_bar_sync(1, 128);
-        if (threadIdx.x == 64) {
-          const int old = atomicAdd(&args.counters[tile_id], 1);
-          const int last = (old == args.splits - 1);
-          if (last) args.counters[tile_id] = 0;
-          *last_flag = last;
-        }
-        named_bar_sync(1, 128);
-        do_epi = *last_flag != 0;
-        if (do_epi) __threadfence();
-      }
-      if (do_epi) {
+      } else {
+        const double inv_freq = epi_inv_freq(e, args.tok, m);
 #pragma unroll 1
         for (int c = 0; c < BN; c += 16) {
           float v[16];
           tmem_ld16(trow + c, v);
           tmem_wait_ld();
-          if (args.splits > 1) {
-            // sum in split order (deterministic); own split from TMEM, the others from L2
-            float acc[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-            const float4* base = reinterpret_cast<const float4*>(args.partials + static_cast<long long>(tile_id) * args.splits * (BN * 128));
-#pragma unroll 4
-            for (int s = 0; s < args.splits; ++s) {
-              float4 t[4];
-              if (s == split) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) t[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-              } else {
-                const float4* p = base + static_cast<long long>(s) * (BN * 32);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) t[q] = __ldcg(p + ((c >> 2) + q) * 128 + row);
-              }
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                acc[4 * q] += t[q].x;
-                acc[4 * q + 1] += t[q].y;
-                acc[4 * q + 2] += t[q].z;
-                acc[4 * q + 3] += t[q].w;
-              }
-            }
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = acc[j];
-          }
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float yp = __shfl_xor_sync(0xffffffffu, v[j], 1);
-            const int n = nt * BN + c + j;
-            if (n < args.N && m < rows_valid) epi_apply<__nv_bfloat16>(e, args.tok, m, n, head, v[j], yp, inv_freq, args.status);
-          }
+          epi_dispatch<16, __nv_bfloat16>(e, args.tok, m, nt * BN + c, head, v, args.N, m_ok, inv_freq, args.status);
         }
       }
     }
@@ -260,6 +228,43 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// Sums the split-K partials of every output tile in split order and applies
+// the epilogue.  Grid (output tiles, BN/4): block x owns tile x, block y a
+// group of 4 columns; thread = row of the tile (so the rotary partner row is a
+// lane shuffle away).  All splits' loads of a thread are independent, so they
+// are in flight together.
+template <int BN>
+__global__ void __launch_bounds__(128) gemm_splitk_epilogue_kernel(const __grid_constant__ GemmArgs args) {
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  const int mt = blockIdx.x, cg = blockIdx.y, row = threadIdx.x;
+  int seg = 0, head = 0, m0;
+  if (args.mode == GEMM_DENSE) {
+    while (seg + 1 < args.nseg && mt >= args.seg_tile0[seg + 1]) ++seg;
+    m0 = (mt - args.seg_tile0[seg]) * 128;
+  } else {
+    const int tph = args.seg_tile0[1];
+    head = mt / tph;
+    m0 = (mt % tph) * 128;
+  }
+  const float4* p = reinterpret_cast<const float4*>(args.partials + static_cast<long long>(mt) * args.splits * (BN * 128)) +
+                    cg * 128 + row;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+  for (int s = 0; s < args.splits; ++s) {
+    const float4 t = __ldcg(p + static_cast<long long>(s) * (BN * 32));
+    acc.x += t.x;
+    acc.y += t.y;
+    acc.z += t.z;
+    acc.w += t.w;
+  }
+  const Epi& e = args.epi[seg];
+  const int m = m0 + row;
+  const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+  epi_dispatch<4, __nv_bfloat16>(e, args.tok, m, cg * 4, head, v, args.N, m < args.seg_rows[seg], epi_inv_freq(e, args.tok, m),
+                                 args.status);
 }
 
 }  // namespace mla

@@ -3,6 +3,7 @@
 // point.  Every arithmetic step runs in the kernels of this directory.
 #include "mla.h"
 
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -137,6 +138,8 @@ struct Ctx {
   bool pdl = false;  // chain the call's kernels with programmatic dependent launch
 };
 
+std::atomic<unsigned long long> g_kernel_launches{0};  // diagnostic: kernels launched by this library
+
 // Launches `kern` on the call's stream; with pdl the kernel may begin while
 // its predecessor drains (every kernel here calls griddep_wait() before it
 // reads or writes anything an earlier kernel touches).
@@ -153,13 +156,19 @@ mla_status launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
+  g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
-template <int BN, bool AMN, int STAGES>
+// Tile width, pipeline depth, K blocks per stage and CTA target of one GEMM launch.
+struct GemmConfig {
+  int bn, stages, kbb, target_ctas;
+};
+
+template <int BN, bool AMN, int STAGES, int KBB>
 mla_status launch_tc(const GemmArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
-  constexpr int smem = GemmSmem<BN, STAGES>::kBytes;
-  auto kern = gemm_tc_kernel<BN, AMN, STAGES>;
+  constexpr int smem = GemmSmem<BN, STAGES, KBB>::kBytes;
+  auto kern = gemm_tc_kernel<BN, AMN, STAGES, KBB>;
   static bool attr_set = false;  // idempotent attribute set; races are harmless
   if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -169,20 +178,32 @@ mla_status launch_tc(const GemmArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
   return launch(kern, grid, dim3(192), smem, st, pdl, a);
 }
 
+// The instantiated configurations (bn, stages, K blocks per stage).
 template <bool AMN>
-mla_status launch_tc_bn(int bn, const GemmArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
-  switch (bn) {
-    case 32: return launch_tc<32, AMN, 5>(a, grid, st, pdl);
-    case 64: return launch_tc<64, AMN, 4>(a, grid, st, pdl);
-    case 128: return launch_tc<128, AMN, 3>(a, grid, st, pdl);
-    default: return launch_tc<256, AMN, 4>(a, grid, st, pdl);
-  }
+mla_status launch_tc_cfg(const GemmConfig& k, const GemmArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
+#define MLA_GEMM_CFG(BN, S, KB) \
+  if (k.bn == BN && k.stages == S && k.kbb == KB) return launch_tc<BN, AMN, S, KB>(a, grid, st, pdl);
+  MLA_GEMM_CFG(32, 5, 1) MLA_GEMM_CFG(64, 4, 1) MLA_GEMM_CFG(128, 3, 1) MLA_GEMM_CFG(256, 4, 1)
+  MLA_GEMM_CFG(32, 4, 2) MLA_GEMM_CFG(64, 4, 2) MLA_GEMM_CFG(32, 2, 4) MLA_GEMM_CFG(64, 2, 4)
+  MLA_GEMM_CFG(64, 2, 2) MLA_GEMM_CFG(32, 2, 2) MLA_GEMM_CFG(128, 2, 2)
+#undef MLA_GEMM_CFG
+  return MLA_ERR_UNSUPPORTED;
 }
 
-mla_status run_gemm_tc(const Ctx& c, const GemmSpec& g) {
+// Default configuration for N tokens: weight-streaming shapes (N <= 64) take
+// two K blocks per stage and four stages (one CTA per SM), larger N the
+// 128/256-wide tiles.
+GemmConfig choose_gemm_config(int N, int num_sms) {
+  if (N <= 32) return {32, 5, 1, 2 * num_sms};
+  if (N <= 64) return {64, 4, 1, 2 * num_sms};
+  if (N <= 128) return {128, 3, 1, 2 * num_sms};
+  return {256, 4, 1, num_sms};
+}
+
+mla_status run_gemm_tc(const Ctx& c, const GemmSpec& g, const GemmConfig& cfg) {
   GemmArgs a;
   memset(&a, 0, sizeof(a));
-  const int bn = pick_bn(g.N);
+  const int bn = cfg.bn;
   const int n_tiles = (g.N + bn - 1) / bn;
   a.mode = g.mode;
   a.N = g.N;
@@ -223,19 +244,29 @@ mla_status run_gemm_tc(const Ctx& c, const GemmSpec& g) {
   if (!make_map_2d(&a.mapB, g.X, g.x_cols, g.N, g.x_ld, a.boxB_rows)) return MLA_ERR_CUDA;
   // split-K so that small tile counts still cover the SMs
   const int tiles = m_tiles * n_tiles;
+  const int target = std::min(cfg.target_ctas, kMaxGemmCtas);
   int splits = 1;
-  if (n_tiles == 1 && tiles < kMaxGemmCtas && tiles <= kMaxCounters) {
-    splits = std::max(1, std::min(a.kb_total / 2, kMaxGemmCtas / tiles));
+  if (n_tiles == 1 && tiles < target && tiles <= kMaxCounters) {
+    splits = std::max(1, std::min(a.kb_total / (2 * cfg.kbb), target / tiles));
   }
   int kbps = (a.kb_total + splits - 1) / splits;
+  kbps = (kbps + cfg.kbb - 1) / cfg.kbb * cfg.kbb;  // whole stages per split
   splits = (a.kb_total + kbps - 1) / kbps;
   a.splits = splits;
   a.kb_per_split = kbps;
   a.partials = reinterpret_cast<float*>(c.ws + c.L.gpart);
-  a.counters = reinterpret_cast<int*>(c.ws + c.L.counters);
   dim3 grid(m_tiles, n_tiles, splits);
-  return g.mode == GEMM_HEAD_MNMAJOR ? launch_tc_bn<true>(bn, a, grid, c.st, c.pdl)
-                                     : launch_tc_bn<false>(bn, a, grid, c.st, c.pdl);
+  mla_status s = g.mode == GEMM_HEAD_MNMAJOR ? launch_tc_cfg<true>(cfg, a, grid, c.st, c.pdl)
+                                            : launch_tc_cfg<false>(cfg, a, grid, c.st, c.pdl);
+  if (s != MLA_OK || splits == 1) return s;
+  // split-K: a wide second kernel sums the partials in split order and runs the epilogue
+  const dim3 rgrid(m_tiles, bn / 4);
+  switch (bn) {
+    case 32: return launch(gemm_splitk_epilogue_kernel<32>, rgrid, dim3(128), 0, c.st, c.pdl, a);
+    case 64: return launch(gemm_splitk_epilogue_kernel<64>, rgrid, dim3(128), 0, c.st, c.pdl, a);
+    case 128: return launch(gemm_splitk_epilogue_kernel<128>, rgrid, dim3(128), 0, c.st, c.pdl, a);
+    default: return launch(gemm_splitk_epilogue_kernel<256>, rgrid, dim3(128), 0, c.st, c.pdl, a);
+  }
 }
 
 template <typename T>
@@ -276,6 +307,7 @@ mla_status run_gemm_simt(const Ctx& c, const GemmSpec& g) {
   a.tok = g.tok;
   a.status = c.status;
   dim3 grid((M + 31) / 32, (g.N + 7) / 8, g.heads);
+  g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
   simt_gemm_kernel<T><<<grid, dim3(32, 8), 0, c.st>>>(a);
   return cudaPeekAtLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
@@ -286,7 +318,7 @@ bool tc_gemm_ok(const mla_dims& d) {
 }
 
 mla_status run_gemm(const Ctx& c, const GemmSpec& g) {
-  if (tc_gemm_ok(c.d)) return run_gemm_tc(c, g);
+  if (tc_gemm_ok(c.d)) return run_gemm_tc(c, g, choose_gemm_config(g.N, c.num_sms));
   return c.d.dtype == MLA_FP32 ? run_gemm_simt<float>(c, g) : run_gemm_simt<__nv_bfloat16>(c, g);
 }
 
@@ -559,6 +591,7 @@ mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const 
   } else {
     const size_t shm = (row + 4 * d.d_c + 8) * sizeof(float);
     dim3 grid(W, d.n_h);
+    g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
     if (d.dtype == MLA_FP32)
       simt_decode_attn_kernel<float><<<grid, 128, shm, c.st>>>(
           static_cast<const float*>(qlat), static_cast<const float*>(cache->base), cache->seq_start, seqlen,
@@ -624,6 +657,8 @@ mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const 
 
 // ====================================================================== C ABI
 extern "C" {
+
+unsigned long long mla_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }
 
 void mla_set_attention_events(void* begin, void* end) {
   g_attn_begin = static_cast<cudaEvent_t>(begin);
@@ -813,6 +848,7 @@ extern "C" mla_status mla_prefill(const mla_dims* dims, const mla_weights* w, co
   // ---- the sequence's cache rows (prefix + new) as one contiguous block
   {
     const int blocks = std::min<long long>(4096, (static_cast<long long>(S) * row + 255) / 256);
+    g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
     if (d.dtype == MLA_FP32)
       gather_rows_kernel<float><<<blocks, 256, 0, c.st>>>(static_cast<const float*>(cache->base), cache->seq_start,
                                                           seq, S, row, static_cast<float*>(rows));
@@ -863,11 +899,13 @@ extern "C" mla_status mla_prefill(const mla_dims* dims, const mla_weights* w, co
         return MLA_ERR_CUDA;
       attr_set = true;
     }
+    g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
     attn_prefill_tc_kernel<<<dim3(a.n_qt, d.n_h), 192, pf::kSmem, c.st>>>(a);
     if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
   } else {
     const size_t shm = (dq + 4 * d.d_h + 8) * sizeof(float);
     dim3 grid(T, d.n_h);
+    g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
     if (d.dtype == MLA_FP32)
       simt_prefill_attn_kernel<float><<<grid, 128, shm, c.st>>>(
           static_cast<const float*>(qp), static_cast<const float*>(kc), static_cast<const float*>(vv),
