@@ -17,17 +17,24 @@
 //   CTA 1: columns c[256,512)        (4 chunks),     O columns [256,512)
 // Each CTA TMA-loads only its own columns of a tile, so the pair reads every
 // cache byte exactly once.  Each computes a partial score S_r = Q_r C_r^T
-// (tcgen05.mma, M = 128 heads, N = 64 tokens, Q_r held in TMEM), sends it to
-// its partner through distributed shared memory as fp16, and forms
-// S = fp16(S_0) + fp16(S_1): both CTAs round both halves the same way, so
-// their softmax, P and running max are bit-identical.  The online softmax runs
-// one thread per head (no cross-thread reductions) with a lazily refreshed
-// max: O is rescaled only when a tile's max exceeds the running one by more
-// than 2^8.  P (bf16) goes to shared memory and O_r += P C_r (N = 256, the
+// (tcgen05.mma, M = 128 heads, N = 64 tokens, Q_r held in TMEM) and both CTAs
+// form S = fp16(S_0) + fp16(S_1) from the same rounded halves, so their
+// softmax, P and running max are bit-identical.  O_r += P C_r (N = 256, the
 // same cache tile read as an MN-major operand) accumulates in TMEM.
 //
-// Warp roles (192 threads per CTA): warp 0 TMA, warp 1 TMEM owner and MMA
-// issuer, warps 2-5 softmax / epilogue (thread = head = TMEM lane).
+// Warp roles (320 threads per CTA); each tile flows through them in order:
+//   warp 0     TMA producer (3-stage ring of tiles)
+//   warp 1     TMEM owner and MMA issuer: S as soon as a tile landed and the
+//              S buffer was read out, PV as soon as a P buffer is written
+//   warps 2-5  exchange: read S from TMEM, round it to fp16, push it into the
+//              partner's shared memory with st.async (its bytes complete the
+//              partner's barrier, so the sender neither fences nor waits) and
+//              keep a copy for this CTA's softmax
+//   warps 6-9  softmax: add the two halves, online softmax with a lazily
+//              refreshed max (O is rescaled only when a tile's max exceeds the
+//              running one by more than 2^8), P (bf16) into one of two shared
+//              buffers, and the per-piece epilogue
+// In both groups thread = head = TMEM lane (warp w owns lanes 32 (w mod 4) ..).
 #pragma once
 #include "mla.h"
 #include "ptx.cuh"
@@ -39,13 +46,16 @@ constexpr int kAttnTileTokens = 64;
 constexpr bool kAttnTcReady = true;
 
 namespace attn {
-constexpr int kStages = 4;
+constexpr int kStages = 3;
+constexpr int kThreads = 320;
 constexpr int kChunkBytes = 64 * 128;             // 64 token rows x 64 latent columns, bf16
 constexpr int kStageBytes = 5 * kChunkBytes;      // up to 5 chunks per CTA
+constexpr int kXBytes = 128 * 128;                // one half of S: 128 heads x 64 tokens, fp16
 constexpr int kPBytes = 128 * 128;                // P: 128 heads x 64 tokens, bf16
-constexpr int kXBytes = 128 * 128;                // partner's partial S: 128 heads x 64 tokens, fp16 (x2 buffers)
 constexpr int kBarBytes = 256;
-constexpr int kSmem = 1024 + kStages * kStageBytes + kPBytes + 2 * kXBytes + kBarBytes;
+// stages | own S half x2 | partner's S half x2 | P x2 | barriers
+constexpr int kSmem = 1024 + kStages * kStageBytes + 4 * kXBytes + 2 * kPBytes + kBarBytes;
+// TMEM columns: O half [0,256), S [256,320), Q half (bf16 pairs) [320,480)
 constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 320, kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kRow = 576;                         // d_c + d_R
@@ -79,23 +89,26 @@ __device__ __forceinline__ float2 unpack_half2(uint32_t v) {
   return __half22float2(*reinterpret_cast<const __half2*>(&v));
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     attn_decode_tc_kernel(const __grid_constant__ AttnArgs a) {
   using namespace attn;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* stages = smem;
-  uint8_t* pbuf = stages + kStages * kStageBytes;
-  uint8_t* xbuf = pbuf + kPBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(xbuf + 2 * kXBytes);
+  uint8_t* xown = stages + kStages * kStageBytes;   // [2] this CTA's half of S (fp16)
+  uint8_t* xpeer = xown + 2 * kXBytes;              // [2] the partner's half, written by the partner
+  uint8_t* pbuf = xpeer + 2 * kXBytes;              // [2] P (bf16), MMA A operand
+  uint64_t* full = reinterpret_cast<uint64_t*>(pbuf + 2 * kPBytes);
   uint64_t* empty = full + kStages;
   uint64_t* s_full = empty + kStages;
   uint64_t* s_free = s_full + 1;
-  uint64_t* p_full = s_free + 1;
-  uint64_t* p_free = p_full + 1;
-  uint64_t* x_full = p_free + 1;   // [2]
-  uint64_t* x_free = x_full + 2;   // [2]
-  uint64_t* q_full = x_free + 2;
+  uint64_t* xo_full = s_free + 1;    // [2] own half stored (exchange -> softmax)
+  uint64_t* xo_free = xo_full + 2;   // [2] own half consumed (softmax -> exchange)
+  uint64_t* x_full = xo_free + 2;    // [2] partner's half landed (st.async bytes)
+  uint64_t* x_free = x_full + 2;     // [2] partner's half consumed (arrivals from the partner's softmax)
+  uint64_t* p_full = x_free + 2;     // [2]
+  uint64_t* p_free = p_full + 2;     // [2]
+  uint64_t* q_full = p_free + 2;
   uint64_t* o_done = q_full + 1;
   uint64_t* drain = o_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -114,17 +127,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 128);
-    mbar_init(p_full, 128);
-    mbar_init(p_free, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&x_full[i], 4);  // one arrival per softmax warp of the partner
-      mbar_init(&x_free[i], 4);
+      mbar_init(&xo_full[i], 4);  // one arrival per exchange warp
+      mbar_init(&xo_free[i], 4);  // one arrival per softmax warp
+      mbar_init(&x_full[i], 1);   // armed once per phase with the expected bytes
+      mbar_init(&x_free[i], 4);   // one arrival per softmax warp of the partner
+      mbar_init(&p_full[i], 128);
+      mbar_init(&p_free[i], 1);
     }
     mbar_init(q_full, 128);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // phase 0 of both exchange slots expects the partner's 16 KB
+    mbar_arrive_expect_tx(&x_full[0], kXBytes);
+    mbar_arrive_expect_tx(&x_full[1], kXBytes);
   }
   if (warp == 0 && lane == 0) prefetch_tmap(&a.map_cache);
   if (warp == 1) {
@@ -132,7 +150,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     tmem_relinquish();
   }
   __syncthreads();
-  cluster_sync();  // the partner's barriers exist before any remote arrive
+  cluster_sync();  // the partner's barriers exist (and are armed) before any remote access
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   griddep_wait();  // Q_lat and the new cache rows come from the preceding kernels
@@ -168,11 +186,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         if (!mbar_wait(q_full, piece & 1, wc)) return;
         tc_fence_after();
         const int nt = p.t1 - p.t0;
-        // Event-driven issue: S(j) as soon as its tile landed and S(j-1) was read
-        // out (the softmax reads S one tile ahead), PV(j) as soon as P(j) is
-        // written; S first, so the softmax never waits behind a PV.
+        // S first, so the exchange never waits behind a PV.
         int ns = 0, npv = 0;
-        uint64_t t_idle = globaltimer();
+        uint32_t spins = 0;
+        uint64_t t_idle = 0;
         while (npv < nt) {
           bool issued = false;
           if (ns < nt) {
@@ -196,30 +213,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           if (!issued && npv < ns) {
             const int g = it + npv;
             const int s = g % kStages;
-            if (mbar_try_wait(smem_u32(p_full), g & 1)) {
+            const int b = g & 1;
+            if (mbar_try_wait(smem_u32(&p_full[b]), (g >> 1) & 1)) {
               tc_fence_after();
               const uint32_t st = smem_u32(stages + s * kStageBytes);
-              const uint32_t pb = smem_u32(pbuf);
+              const uint32_t pb = smem_u32(pbuf + b * kPBytes);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 mma_ss(tmem + kTmemO, sdesc_sw128(pb + kk * 32, 16, 1024), sdesc_sw128(st + kk * 2048, 8192, 1024),
                        idesc_pv, (npv > 0 || kk > 0) ? 1u : 0u);
               }
-              mma_commit(p_free);
+              mma_commit(&p_free[b]);
               mma_commit(&empty[s]);
               if (npv == nt - 1) mma_commit(o_done);
               ++npv;
               issued = true;
             }
           }
+          // idle bookkeeping every 256 empty polls: abort, and the wait limit
           if (issued) {
-            t_idle = globaltimer();
-          } else if (*abort_flag) {
-            return;
-          } else if (globaltimer() - t_idle > kWaitLimitNs) {
-            *abort_flag = 1;
-            atomicOr(a.status, FAULT_WAIT_TIMEOUT);
-            return;
+            spins = 0;
+          } else if ((++spins & 255u) == 0) {
+            if (*abort_flag) return;
+            const uint64_t now = globaltimer();
+            if (spins == 256) {
+              t_idle = now;
+            } else if (now - t_idle > kWaitLimitNs) {
+              *abort_flag = 1;
+              atomicOr(a.status, FAULT_WAIT_TIMEOUT);
+              return;
+            }
           }
         }
         it += nt;
@@ -227,45 +250,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       });
       mma_commit(drain);
     }
-  } else {
-    // ------------------------------------------------------------ softmax + epilogue
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ exchange
     const int q4 = warp & 3;
     const int h = q4 * 32 + lane;  // head = TMEM lane
     const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    const uint32_t x_row = smem_u32(xbuf) + h * 128;
-    const uint32_t x_row_peer = mapa(smem_u32(xbuf), peer) + h * 128;
-    const uint32_t xfull_peer = mapa(smem_u32(x_full), peer);
-    const uint32_t xfree_peer = mapa(smem_u32(x_free), peer);
-    const uint32_t p_row = smem_u32(pbuf) + h * 128;
     const int sw = h & 7;
-    // Partial scores of global tile g: read from TMEM, rounded to fp16 into
-    // `out`, and sent to the partner's exchange buffer g & 1.  The partner is
-    // told once per warp (after the warp's stores, ordered by the warp barrier).
-    auto send = [&](int g, uint32_t (&out)[32]) -> bool {
-      if (!mbar_wait(s_full, g & 1, wc)) return false;
-      tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(tl + kTmemS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tl + kTmemS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(s_free);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) out[j] = pack_half2(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1]));
-      const int slot = g & 1;
-      if (!mbar_wait<true>(&x_free[slot], ((g >> 1) & 1) ^ 1, wc)) return false;
-      const uint32_t dst = x_row_peer + slot * kXBytes;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        st_cluster_v4(dst + ((i ^ sw) << 4), make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]));
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(xfull_peer + slot * 8);
-      return true;
-    };
-    int it = 0, piece = 0;
+    const uint32_t own_row = smem_u32(xown) + h * 128;
+    const uint32_t peer_row = mapa(smem_u32(xpeer), peer) + h * 128;
+    const uint32_t xfull_peer = mapa(smem_u32(x_full), peer);
+    int it = 0;
     for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
       if (*abort_flag) return;
-      // ---- this CTA's half of Q_lat[b, h] into TMEM (MMA A operand)
+      // ---- this CTA's half of Q_lat[b, h] into TMEM (MMA A operand).  The
+      // previous piece's last S has been read out, so no MMA still reads Q.
       const bool head = h < a.n_h;
       const __nv_bfloat16* qrow = a.qlat + (static_cast<long long>(p.b) * a.n_h + (head ? h : 0)) * kRow;
       for (int ci = 0; ci < nchunks; ++ci) {
@@ -282,37 +280,92 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(q_full);
 
+      const int nt = p.t1 - p.t0;
+      for (int k = 0; k < nt; ++k) {
+        const int g = it + k;
+        const int slot = g & 1;
+        const uint32_t ph = (g >> 1) & 1;
+        if (!mbar_wait(s_full, g & 1, wc)) return;
+        tc_fence_after();
+        uint32_t sr[64];
+        tmem_ld32(tl + kTmemS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(tl + kTmemS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(s_free);
+        uint32_t hx[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) hx[j] = pack_half2(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1]));
+        // partner first: its copy has the longer way to go
+        if (!mbar_wait<true>(&x_free[slot], ph ^ 1, wc)) return;
+        const uint32_t dst = peer_row + slot * kXBytes;
+        const uint32_t bar = xfull_peer + slot * 8;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          st_async_v4(dst + ((i ^ sw) << 4), make_uint4(hx[4 * i], hx[4 * i + 1], hx[4 * i + 2], hx[4 * i + 3]), bar);
+        if (!mbar_wait(&xo_free[slot], ph ^ 1, wc)) return;
+        const uint32_t od = own_row + slot * kXBytes;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          st_shared_v4(od + ((i ^ sw) << 4), make_uint4(hx[4 * i], hx[4 * i + 1], hx[4 * i + 2], hx[4 * i + 3]));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xo_full[slot]);
+      }
+      it += nt;
+    });
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int q4 = warp & 3;
+    const int h = q4 * 32 + lane;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const int sw = h & 7;
+    const bool leader = warp == 6;  // re-arms the exchange barriers
+    const uint32_t own_row = smem_u32(xown) + h * 128;
+    const uint32_t peer_row = smem_u32(xpeer) + h * 128;
+    const uint32_t p_row = smem_u32(pbuf) + h * 128;
+    const uint32_t xfree_peer = mapa(smem_u32(x_free), peer);
+    int it = 0, piece = 0;
+    for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
+      if (*abort_flag) return;
+      const bool head = h < a.n_h;
       const int L1 = a.seqlen[p.b] + 1;
       float m_run = -INFINITY, l_run = 0.f;
       const int nt = p.t1 - p.t0;
-      uint32_t mine[32];
-      if (nt > 0 && !send(it, mine)) return;
       for (int k = 0; k < nt; ++k) {
         const int g = it + k;
         const int t = p.t0 + k;
-        // the next tile's partial goes out before this tile's partner half is awaited,
-        // so the exchange latency overlaps the softmax of this tile
-        uint32_t nxt[32];
-        if (k + 1 < nt && !send(g + 1, nxt)) return;
         const int slot = g & 1;
-        if (!mbar_wait<true>(&x_full[slot], (g >> 1) & 1, wc)) return;
-        uint32_t theirs[32];
+        const uint32_t ph = (g >> 1) & 1;
+        if (!mbar_wait(&xo_full[slot], ph, wc)) return;
+        if (!mbar_wait<true>(&x_full[slot], ph, wc)) return;
+        // ---- full scores (same bits in both CTAs), masked beyond the sequence
+        float sc[64];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const uint4 v = ld_shared_v4(x_row + slot * kXBytes + ((i ^ sw) << 4));
-          theirs[4 * i] = v.x; theirs[4 * i + 1] = v.y; theirs[4 * i + 2] = v.z; theirs[4 * i + 3] = v.w;
+          const uint4 u = ld_shared_v4(own_row + slot * kXBytes + ((i ^ sw) << 4));
+          const uint4 v = ld_shared_v4(peer_row + slot * kXBytes + ((i ^ sw) << 4));
+          const uint32_t uu[4] = {u.x, u.y, u.z, u.w}, vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 x = unpack_half2(uu[e]), y = unpack_half2(vv[e]);
+            sc[8 * i + 2 * e] = x.x + y.x;
+            sc[8 * i + 2 * e + 1] = x.y + y.y;
+          }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(xfree_peer + slot * 8);
-        // ---- full scores (same bits in both CTAs), masked beyond the sequence
+        if (lane == 0) {
+          mbar_arrive(&xo_free[slot]);
+          // the slot's next phase expects the partner's next 16 KB; armed
+          // before the slot is released, so no byte can land ahead of it
+          if (leader) mbar_arrive_expect_tx(&x_full[slot], kXBytes);
+          mbar_arrive_remote(xfree_peer + slot * 8);
+        }
         const int valid = min(64, L1 - t * 64);
         float mt = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float2 x = unpack_half2(mine[j]), y = unpack_half2(theirs[j]);
-          const float s0 = (2 * j < valid) ? x.x + y.x : -INFINITY;
-          const float s1 = (2 * j + 1 < valid) ? x.y + y.y : -INFINITY;
-          mt = fmaxf(mt, fmaxf(s0, s1));
+        for (int j = 0; j < 64; ++j) {
+          if (j >= valid) sc[j] = -INFINITY;
+          mt = fmaxf(mt, sc[j]);
         }
         float m_new = m_run, alpha = 1.f;
         bool rescale = false;
@@ -327,20 +380,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         float lsum = 0.f;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float2 x = unpack_half2(mine[j]), y = unpack_half2(theirs[j]);
-          const float s0 = (2 * j < valid) ? x.x + y.x : -INFINITY;
-          const float s1 = (2 * j + 1 < valid) ? x.y + y.y : -INFINITY;
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(ex2_approx(s0 - m_new), ex2_approx(s1 - m_new));
+          const __nv_bfloat162 b2 =
+              __floats2bfloat162_rn(ex2_approx(sc[2 * j] - m_new), ex2_approx(sc[2 * j + 1] - m_new));
           const float2 f = __bfloat1622float2(b2);
           lsum += f.x + f.y;
           pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
         }
         l_run = l_run * alpha + lsum;
         m_run = m_new;
-        // ---- previous PV done: P buffer free, O settled
-        if (!mbar_wait(p_free, (g & 1) ^ 1, wc)) return;
-        tc_fence_after();
+        const int b = g & 1;
+        // ---- P buffer b is free once PV(g-2) retired
+        if (!mbar_wait(&p_free[b], ph ^ 1, wc)) return;
         if (__any_sync(0xffffffffu, rescale)) {
+          // O must hold PV(g-1) before it is scaled (k >= 1 here, so g >= 1)
+          if (!mbar_wait(&p_free[b ^ 1], ((g - 1) >> 1) & 1, wc)) return;
+          tc_fence_after();
           for (int c = 0; c < 256; c += 32) {
             uint32_t o[32];
             tmem_ld32(tl + kTmemO + c, o);
@@ -361,16 +415,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             *reinterpret_cast<uint4*>(st + (c16 >> 3) * kChunkBytes + row * 128 + (c16 & 7) * 16) = make_uint4(0, 0, 0, 0);
           }
         }
+        const uint32_t pr = p_row + b * kPBytes;
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          st_shared_v4(p_row + ((i ^ sw) << 4), make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
+          st_shared_v4(pr + ((i ^ sw) << 4), make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(p_full);
-        if (k + 1 < nt) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) mine[j] = nxt[j];
-        }
+        mbar_arrive(&p_full[b]);
       }
       // ---- epilogue of the piece: unnormalised O_r, m, l
       if (!mbar_wait(o_done, piece & 1, wc)) return;

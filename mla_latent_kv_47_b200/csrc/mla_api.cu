@@ -464,7 +464,7 @@ mla_status launch_attn_decode_tc(const __nv_bfloat16* qlat, const mla_cache* cac
       return MLA_ERR_CUDA;
     attr_set = true;
   }
-  return launch(attn_decode_tc_kernel, dim3(2 * W), dim3(192), attn::kSmem, st, pdl, a);
+  return launch(attn_decode_tc_kernel, dim3(2 * W), dim3(attn::kThreads), attn::kSmem, st, pdl, a);
 }
 
 bool prefill_tc_ok(const mla_dims& d) {

@@ -243,6 +243,16 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint4 v) {
                "r"(v.w)
                : "memory");
 }
+// 16-byte store into another CTA's shared memory that completes 16 transaction
+// bytes on that CTA's mbarrier (both addresses from mapa).  Nothing on the
+// sending side waits for it; the receiver's barrier phase completes once all
+// expected bytes landed.
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint4 v, uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1,%2,%3,%4}, [%5];" ::"r"(
+                   cluster_addr),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(cluster_bar)
+               : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
