@@ -22,19 +22,21 @@
 // softmax, P and running max are bit-identical.  O_r += P C_r (N = 256, the
 // same cache tile read as an MN-major operand) accumulates in TMEM.
 //
-// Warp roles (320 threads per CTA); each tile flows through them in order:
-//   warp 0     TMA producer (3-stage ring of tiles)
-//   warp 1     TMEM owner and MMA issuer: S as soon as a tile landed and the
-//              S buffer was read out, PV as soon as a P buffer is written
-//   warps 2-5  exchange: read S from TMEM, round it to fp16, push it into the
-//              partner's shared memory with st.async (its bytes complete the
-//              partner's barrier, so the sender neither fences nor waits) and
-//              keep a copy for this CTA's softmax
-//   warps 6-9  softmax: add the two halves, online softmax with a lazily
-//              refreshed max (O is rescaled only when a tile's max exceeds the
-//              running one by more than 2^8), P (bf16) into one of two shared
-//              buffers, and the per-piece epilogue
-// In both groups thread = head = TMEM lane (warp w owns lanes 32 (w mod 4) ..).
+// Warp roles (448 threads per CTA); each tile flows through them in order:
+//   warp 0      TMA producer (4-stage ring of tiles)
+//   warp 1      TMEM owner and MMA issuer: S as soon as a tile landed and the
+//               S buffer was read out, PV as soon as P is written
+//   warps 2-5   exchange: read S from TMEM, round it to fp16, push it into the
+//               partner's shared memory with st.async (its bytes complete the
+//               partner's barrier, so the sender neither fences nor waits) and
+//               park this CTA's rounded half in TMEM for the softmax
+//   warps 6-13  softmax, two warps per head: warps 6-9 take tokens 0-31 and
+//               warps 10-13 tokens 32-63 of a tile, each for the heads of its
+//               lane quarter; they agree on the tile max through shared memory.  Online
+//               softmax with a lazily refreshed max (O is rescaled only when a
+//               tile's max exceeds the running one by more than 2^8), P (bf16)
+//               into shared memory, and the per-piece epilogue
+// thread = head = TMEM lane (warp w owns lanes 32 (w mod 4) ..).
 #pragma once
 #include "mla.h"
 #include "ptx.cuh"
@@ -46,17 +48,19 @@ constexpr int kAttnTileTokens = 64;
 constexpr bool kAttnTcReady = true;
 
 namespace attn {
-constexpr int kStages = 3;
-constexpr int kThreads = 320;
+constexpr int kStages = 4;
+constexpr int kThreads = 448;
 constexpr int kChunkBytes = 64 * 128;             // 64 token rows x 64 latent columns, bf16
 constexpr int kStageBytes = 5 * kChunkBytes;      // up to 5 chunks per CTA
 constexpr int kXBytes = 128 * 128;                // one half of S: 128 heads x 64 tokens, fp16
 constexpr int kPBytes = 128 * 128;                // P: 128 heads x 64 tokens, bf16
-constexpr int kBarBytes = 256;
-// stages | own S half x2 | partner's S half x2 | P x2 | barriers
-constexpr int kSmem = 1024 + kStages * kStageBytes + 4 * kXBytes + 2 * kPBytes + kBarBytes;
-// TMEM columns: O half [0,256), S [256,320), Q half (bf16 pairs) [320,480)
-constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 320, kTmemCols = 512;
+constexpr int kRedBytes = (2 * 2 + 1) * 128 * 4;  // tile max of each token half (two slots), l of half 1
+constexpr int kBarBytes = 512;
+// stages | partner's S half x2 | P | max / sum exchange | barriers
+constexpr int kSmem = 1024 + kStages * kStageBytes + 2 * kXBytes + kPBytes + kRedBytes + kBarBytes;
+// TMEM columns: O half [0,256), S [256,320), Q half (bf16 pairs) [320,480),
+// this CTA's fp16-rounded S half (pairs) [480,512)
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 320, kTmemX = 480, kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kRow = 576;                         // d_c + d_R
 }  // namespace attn
@@ -95,23 +99,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* stages = smem;
-  uint8_t* xown = stages + kStages * kStageBytes;   // [2] this CTA's half of S (fp16)
-  uint8_t* xpeer = xown + 2 * kXBytes;              // [2] the partner's half, written by the partner
-  uint8_t* pbuf = xpeer + 2 * kXBytes;              // [2] P (bf16), MMA A operand
-  uint64_t* full = reinterpret_cast<uint64_t*>(pbuf + 2 * kPBytes);
+  uint8_t* xpeer = stages + kStages * kStageBytes;  // [2] the partner's half of S (fp16), written by the partner
+  uint8_t* pbuf = xpeer + 2 * kXBytes;              // P (bf16), MMA A operand
+  float* red = reinterpret_cast<float*>(pbuf + kPBytes);  // [2 slots][2 halves][128] tile max, then [128] l
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + kRedBytes);
   uint64_t* empty = full + kStages;
   uint64_t* s_full = empty + kStages;
   uint64_t* s_free = s_full + 1;
-  uint64_t* xo_full = s_free + 1;    // [2] own half stored (exchange -> softmax)
-  uint64_t* xo_free = xo_full + 2;   // [2] own half consumed (softmax -> exchange)
-  uint64_t* x_full = xo_free + 2;    // [2] partner's half landed (st.async bytes)
+  uint64_t* xo_full = s_free + 1;    // own rounded half parked in TMEM (exchange -> softmax)
+  uint64_t* xo_free = xo_full + 1;   // own half read out (softmax -> exchange)
+  uint64_t* x_full = xo_free + 1;    // [2] partner's half landed (st.async bytes)
   uint64_t* x_free = x_full + 2;     // [2] partner's half consumed (arrivals from the partner's softmax)
-  uint64_t* p_full = x_free + 2;     // [2]
-  uint64_t* p_free = p_full + 2;     // [2]
-  uint64_t* q_full = p_free + 2;
+  uint64_t* p_full = x_free + 2;
+  uint64_t* p_free = p_full + 1;
+  uint64_t* q_full = p_free + 1;
   uint64_t* o_done = q_full + 1;
   uint64_t* drain = o_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* m_bar = drain + 1;       // [2 slots][4 quarters] both token halves posted their tile max
+  uint64_t* l_bar = m_bar + 8;       // [4 quarters] token half 1 posted its l at the end of a piece
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(l_bar + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t rank = cluster_ctarank();
@@ -127,17 +133,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 128);
+    mbar_init(xo_full, 4);      // one arrival per exchange warp
+    mbar_init(xo_free, 8);      // one arrival per softmax warp
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&xo_full[i], 4);  // one arrival per exchange warp
-      mbar_init(&xo_free[i], 4);  // one arrival per softmax warp
       mbar_init(&x_full[i], 1);   // armed once per phase with the expected bytes
-      mbar_init(&x_free[i], 4);   // one arrival per softmax warp of the partner
-      mbar_init(&p_full[i], 128);
-      mbar_init(&p_free[i], 1);
+      mbar_init(&x_free[i], 8);   // one arrival per softmax warp of the partner
     }
+    mbar_init(p_full, 256);
+    mbar_init(p_free, 1);
     mbar_init(q_full, 128);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&m_bar[i], 2);  // one arrival per warp of the pair
+    for (int i = 0; i < 4; ++i) mbar_init(&l_bar[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
     // phase 0 of both exchange slots expects the partner's 16 KB
@@ -180,6 +188,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     if (elect_one()) {
       constexpr uint32_t idesc_s = idesc_bf16(128, 64, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(128, 256, false, true);
+      const uint32_t pb = smem_u32(pbuf);
       int it = 0, piece = 0;
       for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
         if (*abort_flag) return;
@@ -213,17 +222,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           if (!issued && npv < ns) {
             const int g = it + npv;
             const int s = g % kStages;
-            const int b = g & 1;
-            if (mbar_try_wait(smem_u32(&p_full[b]), (g >> 1) & 1)) {
+            if (mbar_try_wait(smem_u32(p_full), g & 1)) {
               tc_fence_after();
               const uint32_t st = smem_u32(stages + s * kStageBytes);
-              const uint32_t pb = smem_u32(pbuf + b * kPBytes);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 mma_ss(tmem + kTmemO, sdesc_sw128(pb + kk * 32, 16, 1024), sdesc_sw128(st + kk * 2048, 8192, 1024),
                        idesc_pv, (npv > 0 || kk > 0) ? 1u : 0u);
               }
-              mma_commit(&p_free[b]);
+              mma_commit(p_free);
               mma_commit(&empty[s]);
               if (npv == nt - 1) mma_commit(o_done);
               ++npv;
@@ -256,7 +263,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     const int h = q4 * 32 + lane;  // head = TMEM lane
     const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int sw = h & 7;
-    const uint32_t own_row = smem_u32(xown) + h * 128;
     const uint32_t peer_row = mapa(smem_u32(xpeer), peer) + h * 128;
     const uint32_t xfull_peer = mapa(smem_u32(x_full), peer);
     int it = 0;
@@ -287,15 +293,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         const uint32_t ph = (g >> 1) & 1;
         if (!mbar_wait(s_full, g & 1, wc)) return;
         tc_fence_after();
-        uint32_t sr[64];
-        tmem_ld32(tl + kTmemS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(tl + kTmemS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(s_free);
         uint32_t hx[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) hx[j] = pack_half2(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1]));
+        for (int half = 0; half < 2; ++half) {
+          uint32_t sr[32];
+          tmem_ld32(tl + kTmemS + half * 32, sr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            hx[half * 16 + j] = pack_half2(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1]));
+        }
+        tc_fence_before();
+        mbar_arrive(s_free);
         // partner first: its copy has the longer way to go
         if (!mbar_wait<true>(&x_free[slot], ph ^ 1, wc)) return;
         const uint32_t dst = peer_row + slot * kXBytes;
@@ -303,27 +312,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           st_async_v4(dst + ((i ^ sw) << 4), make_uint4(hx[4 * i], hx[4 * i + 1], hx[4 * i + 2], hx[4 * i + 3]), bar);
-        if (!mbar_wait(&xo_free[slot], ph ^ 1, wc)) return;
-        const uint32_t od = own_row + slot * kXBytes;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          st_shared_v4(od + ((i ^ sw) << 4), make_uint4(hx[4 * i], hx[4 * i + 1], hx[4 * i + 2], hx[4 * i + 3]));
+        // own half into TMEM once the softmax has read the previous one
+        if (!mbar_wait(xo_free, (g & 1) ^ 1, wc)) return;
+        tc_fence_after();
+        tmem_st32(tl + kTmemX, hx);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&xo_full[slot]);
+        if (lane == 0) mbar_arrive(xo_full);
       }
       it += nt;
     });
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int q4 = warp & 3;
+    const int hf = (warp - 6) >> 2;  // token half of the tile: [32 hf, 32 hf + 32)
     const int h = q4 * 32 + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int sw = h & 7;
-    const bool leader = warp == 6;  // re-arms the exchange barriers
-    const uint32_t own_row = smem_u32(xown) + h * 128;
+    const bool leader = warp == 6;   // re-arms the exchange barriers
     const uint32_t peer_row = smem_u32(xpeer) + h * 128;
     const uint32_t p_row = smem_u32(pbuf) + h * 128;
     const uint32_t xfree_peer = mapa(smem_u32(x_free), peer);
+    float* l_other = red + 4 * 128;
     int it = 0, piece = 0;
     for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
       if (*abort_flag) return;
@@ -336,37 +347,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         const int t = p.t0 + k;
         const int slot = g & 1;
         const uint32_t ph = (g >> 1) & 1;
-        if (!mbar_wait(&xo_full[slot], ph, wc)) return;
+        if (!mbar_wait(xo_full, g & 1, wc)) return;
         if (!mbar_wait<true>(&x_full[slot], ph, wc)) return;
-        // ---- full scores (same bits in both CTAs), masked beyond the sequence
-        float sc[64];
+        tc_fence_after();
+        // ---- full scores of this warp's 32 tokens (same bits in both CTAs)
+        uint32_t own[16];
+        tmem_ld16(tl + kTmemX + hf * 16, *reinterpret_cast<float(*)[16]>(own));
+        uint4 pv[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 u = ld_shared_v4(own_row + slot * kXBytes + ((i ^ sw) << 4));
-          const uint4 v = ld_shared_v4(peer_row + slot * kXBytes + ((i ^ sw) << 4));
-          const uint32_t uu[4] = {u.x, u.y, u.z, u.w}, vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 x = unpack_half2(uu[e]), y = unpack_half2(vv[e]);
-            sc[8 * i + 2 * e] = x.x + y.x;
-            sc[8 * i + 2 * e + 1] = x.y + y.y;
-          }
-        }
+        for (int i = 0; i < 4; ++i) pv[i] = ld_shared_v4(peer_row + slot * kXBytes + (((hf * 4 + i) ^ sw) << 4));
+        tmem_wait_ld();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&xo_free[slot]);
+          mbar_arrive(xo_free);
           // the slot's next phase expects the partner's next 16 KB; armed
           // before the slot is released, so no byte can land ahead of it
           if (leader) mbar_arrive_expect_tx(&x_full[slot], kXBytes);
           mbar_arrive_remote(xfree_peer + slot * 8);
         }
-        const int valid = min(64, L1 - t * 64);
-        float mt = -INFINITY;
+        const int valid = min(64, L1 - t * 64) - hf * 32;  // valid tokens of this half (may be <= 0)
+        float sc[32];
+        float mh = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          if (j >= valid) sc[j] = -INFINITY;
-          mt = fmaxf(mt, sc[j]);
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t vv[4] = {pv[i].x, pv[i].y, pv[i].z, pv[i].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 8 * i + 2 * e;
+            const float2 x = unpack_half2(own[4 * i + e]), y = unpack_half2(vv[e]);
+            sc[j] = j < valid ? x.x + y.x : -INFINITY;
+            sc[j + 1] = j + 1 < valid ? x.y + y.y : -INFINITY;
+            mh = fmaxf(mh, fmaxf(sc[j], sc[j + 1]));
+          }
         }
+        // tile max over both halves (a barrier wait that gives up, unlike bar.sync,
+        // so a partner warp that aborted cannot strand this one)
+        red[(slot * 2 + hf) * 128 + h] = mh;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&m_bar[slot * 4 + q4]);
+        if (!mbar_wait(&m_bar[slot * 4 + q4], ph, wc)) return;
+        const float mt = fmaxf(mh, red[(slot * 2 + (hf ^ 1)) * 128 + h]);
         float m_new = m_run, alpha = 1.f;
         bool rescale = false;
         if (k == 0) {
@@ -376,10 +397,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           alpha = ex2_approx(m_run - m_new);
           rescale = true;
         }
-        uint32_t pk[32];
+        uint32_t pk[16];
         float lsum = 0.f;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < 16; ++j) {
           const __nv_bfloat162 b2 =
               __floats2bfloat162_rn(ex2_approx(sc[2 * j] - m_new), ex2_approx(sc[2 * j + 1] - m_new));
           const float2 f = __bfloat1622float2(b2);
@@ -388,14 +409,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         }
         l_run = l_run * alpha + lsum;
         m_run = m_new;
-        const int b = g & 1;
-        // ---- P buffer b is free once PV(g-2) retired
-        if (!mbar_wait(&p_free[b], ph ^ 1, wc)) return;
+        // ---- PV(g-1) retired: the P buffer is free and O settled
+        if (!mbar_wait(p_free, (g & 1) ^ 1, wc)) return;
+        tc_fence_after();
         if (__any_sync(0xffffffffu, rescale)) {
-          // O must hold PV(g-1) before it is scaled (k >= 1 here, so g >= 1)
-          if (!mbar_wait(&p_free[b ^ 1], ((g - 1) >> 1) & 1, wc)) return;
-          tc_fence_after();
-          for (int c = 0; c < 256; c += 32) {
+          for (int c = hf * 128; c < hf * 128 + 128; c += 32) {
             uint32_t o[32];
             tmem_ld32(tl + kTmemO + c, o);
             tmem_wait_ld();
@@ -405,29 +423,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           }
           tmem_wait_st();
         }
-        if (valid < 64) {
+        if (valid + hf * 32 < 64) {
           // rows past the sequence may hold anything (even NaN); 0 * NaN would
           // poison O, so the rows this CTA multiplies into O are zeroed
+          const int v64 = valid + hf * 32;
           uint8_t* st = stages + (g % kStages) * kStageBytes;
-          const int n16 = (64 - valid) * 32;
-          for (int idx = h; idx < n16; idx += 128) {
-            const int row = valid + (idx >> 5), c16 = idx & 31;
+          const int n16 = (64 - v64) * 32;
+          for (int idx = hf * 128 + h; idx < n16; idx += 256) {
+            const int row = v64 + (idx >> 5), c16 = idx & 31;
             *reinterpret_cast<uint4*>(st + (c16 >> 3) * kChunkBytes + row * 128 + (c16 & 7) * 16) = make_uint4(0, 0, 0, 0);
           }
         }
-        const uint32_t pr = p_row + b * kPBytes;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          st_shared_v4(pr + ((i ^ sw) << 4), make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
+        for (int i = 0; i < 4; ++i)
+          st_shared_v4(p_row + (((hf * 4 + i) ^ sw) << 4), make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&p_full[b]);
+        mbar_arrive(p_full);
       }
-      // ---- epilogue of the piece: unnormalised O_r, m, l
+      // ---- epilogue of the piece: unnormalised O_r (this warp's 128 columns), m, l
       if (!mbar_wait(o_done, piece & 1, wc)) return;
       tc_fence_after();
       float* dst = a.o_part + (static_cast<long long>(p.slot) * a.n_h + h) * 512 + rank * 256;
-      for (int c = 0; c < 256; c += 32) {
+      for (int c = hf * 128; c < hf * 128 + 128; c += 32) {
         uint32_t o[32];
         tmem_ld32(tl + kTmemO + c, o);
         tmem_wait_ld();
@@ -438,9 +456,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
                                                                 __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
         }
       }
-      if (rank == 0 && head) {
+      if (hf == 1) {
+        l_other[h] = l_run;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&l_bar[q4]);
+      } else if (!mbar_wait(&l_bar[q4], piece & 1, wc)) {
+        return;
+      }
+      if (rank == 0 && hf == 0 && head) {
         a.ml_part[(static_cast<long long>(p.slot) * a.n_h + h) * 2] = m_run;
-        a.ml_part[(static_cast<long long>(p.slot) * a.n_h + h) * 2 + 1] = l_run;
+        a.ml_part[(static_cast<long long>(p.slot) * a.n_h + h) * 2 + 1] = l_run + l_other[h];
       }
       tc_fence_before();
       it += nt;

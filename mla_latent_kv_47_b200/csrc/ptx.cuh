@@ -88,10 +88,10 @@ struct WaitCtx {
 
 // Waits until the phase with `parity` of `bar` completed.  Returns false (and
 // sets FAULT_WAIT_TIMEOUT) after kWaitLimitNs, or at once if the CTA aborted.
-template <bool kCluster = false>
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
-  const uint32_t a = smem_u32(bar);
-  if (kCluster ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity)) return true;
+// The first probe is inline; only a barrier that is not yet complete pays for
+// the call into the polling loop.
+template <bool kCluster>
+__device__ __noinline__ bool mbar_wait_slow(uint32_t a, uint32_t parity, const WaitCtx& w) {
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
     if (kCluster ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity)) return true;
@@ -104,6 +104,12 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Wai
       }
     }
   }
+}
+template <bool kCluster = false>
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+  const uint32_t a = smem_u32(bar);
+  if (kCluster ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity)) return true;
+  return mbar_wait_slow<kCluster>(a, parity, w);
 }
 
 // ------------------------------------------------------------------ TMA
