@@ -29,7 +29,9 @@
 //   warps 2-5   exchange: read S from TMEM, round it to fp16, push it into the
 //               partner's shared memory with st.async (its bytes complete the
 //               partner's barrier, so the sender neither fences nor waits) and
-//               park this CTA's rounded half in TMEM for the softmax
+//               park this CTA's rounded half in TMEM for the softmax.  The
+//               partner hands a slot back the same way: a 4-byte st.async per
+//               softmax warp that completes this CTA's slot-free barrier.
 //   warps 6-13  softmax, two warps per head: warps 6-9 take tokens 0-31 and
 //               warps 10-13 tokens 32-63 of a tile, each for the heads of its
 //               lane quarter; they agree on the tile max through shared memory.  Online
@@ -117,7 +119,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   uint64_t* drain = o_done + 1;
   uint64_t* m_bar = drain + 1;       // [2 slots][4 quarters] both token halves posted their tile max
   uint64_t* l_bar = m_bar + 8;       // [4 quarters] token half 1 posted its l at the end of a piece
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(l_bar + 4);
+  uint32_t* sig = reinterpret_cast<uint32_t*>(l_bar + 4);  // [2 slots][8] landing words of the partner's slot-free signals
+  uint32_t* tmem_slot = sig + 16;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t rank = cluster_ctarank();
@@ -137,7 +140,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     mbar_init(xo_free, 8);      // one arrival per softmax warp
     for (int i = 0; i < 2; ++i) {
       mbar_init(&x_full[i], 1);   // armed once per phase with the expected bytes
-      mbar_init(&x_free[i], 8);   // one arrival per softmax warp of the partner
+      mbar_init(&x_free[i], 1);   // armed by the exchange before each use; 8 x 4 signal bytes from the partner
     }
     mbar_init(p_full, 256);
     mbar_init(p_free, 1);
@@ -265,6 +268,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     const int sw = h & 7;
     const uint32_t peer_row = mapa(smem_u32(xpeer), peer) + h * 128;
     const uint32_t xfull_peer = mapa(smem_u32(x_full), peer);
+    const bool arm = warp == 2 && lane == 0;
     int it = 0;
     for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
       if (*abort_flag) return;
@@ -307,6 +311,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         mbar_arrive(s_free);
         // partner first: its copy has the longer way to go
         if (!mbar_wait<true>(&x_free[slot], ph ^ 1, wc)) return;
+        // the partner returns this use of the slot with 8 signals of 4 bytes;
+        // armed before this warp's data goes out, so no signal can precede it
+        if (arm) mbar_arrive_expect_tx(&x_free[slot], 32);
         const uint32_t dst = peer_row + slot * kXBytes;
         const uint32_t bar = xfull_peer + slot * 8;
 #pragma unroll
@@ -323,6 +330,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       }
       it += nt;
     });
+    // The partner's signals for the last use of each slot land in this CTA's
+    // shared memory: they must have arrived before the CTA may exit.
+    if (arm && !*abort_flag) {
+      for (int s2 = 0; s2 < 2; ++s2) {
+        const int uses = (it + 1 - s2) / 2;
+        if (uses > 0 && !mbar_wait<true>(&x_free[s2], (uses - 1) & 1, wc)) break;
+      }
+    }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int q4 = warp & 3;
@@ -334,6 +349,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     const uint32_t peer_row = smem_u32(xpeer) + h * 128;
     const uint32_t p_row = smem_u32(pbuf) + h * 128;
     const uint32_t xfree_peer = mapa(smem_u32(x_free), peer);
+    const uint32_t sig_peer = mapa(smem_u32(sig), peer) + (warp - 6) * 4;
     float* l_other = red + 4 * 128;
     int it = 0, piece = 0;
     for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
@@ -364,7 +380,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           // the slot's next phase expects the partner's next 16 KB; armed
           // before the slot is released, so no byte can land ahead of it
           if (leader) mbar_arrive_expect_tx(&x_full[slot], kXBytes);
-          mbar_arrive_remote(xfree_peer + slot * 8);
         }
         const int valid = min(64, L1 - t * 64) - hf * 32;  // valid tokens of this half (may be <= 0)
         float sc[32];
@@ -381,6 +396,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
             mh = fmaxf(mh, fmaxf(sc[j], sc[j + 1]));
           }
         }
+        // every value read from the partner's half is consumed: hand the slot back
+        __syncwarp();
+        if (lane == 0) st_async_b32(sig_peer + slot * 32, 0u, xfree_peer + slot * 8);
         // tile max over both halves (a barrier wait that gives up, unlike bar.sync,
         // so a partner warp that aborted cannot strand this one)
         red[(slot * 2 + hf) * 128 + h] = mh;
