@@ -343,7 +343,8 @@ def run_ours(args):
     assert code == 0, ("decode fault", code, detail)
 
     if args.profile:
-        print(json.dumps({"profile_run": True, "ms_per_step": ms, "attn_ms": attn_ms}), flush=True)
+        print(json.dumps({"profile_run": True, "ms_per_step": ms, "attn_ms": attn_ms,
+                          "launches_before_timing": launches0, "launches_per_step": launches // K}), flush=True)
         return 0
     # ---- end to end: host (pinned) inputs in, host output back, every step
     h_host = h_new.cpu().pin_memory()

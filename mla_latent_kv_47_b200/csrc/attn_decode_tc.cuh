@@ -32,13 +32,15 @@
 //               park this CTA's rounded half in TMEM for the softmax.  The
 //               partner hands a slot back the same way: a 4-byte st.async per
 //               softmax warp that completes this CTA's slot-free barrier.
-//   warps 6-13  softmax, two warps per head: warps 6-9 take tokens 0-31 and
-//               warps 10-13 tokens 32-63 of a tile, each for the heads of its
-//               lane quarter; they agree on the tile max through shared memory.  Online
-//               softmax with a lazily refreshed max (O is rescaled only when a
-//               tile's max exceeds the running one by more than 2^8), P (bf16)
-//               into shared memory, and the per-piece epilogue
-// thread = head = TMEM lane (warp w owns lanes 32 (w mod 4) ..).
+//   warps 6-13  softmax: warp 6+i and warp 10+i share lane quarter i mod 4,
+//               16 heads each; two threads per head (tokens 0-31 and 32-63 of
+//               the tile, via the 16-lane TMEM access shape), so a head's tile
+//               max is one shuffle.  Online softmax with a lazily refreshed
+//               max (O is rescaled only when a tile's max exceeds the running
+//               one by more than 2^8), P (bf16) into shared memory, and the
+//               per-piece epilogue
+// The exchange warps use thread = head = TMEM lane (warp w owns lanes
+// 32 (w mod 4) ..).
 #pragma once
 #include "mla.h"
 #include "ptx.cuh"
@@ -56,10 +58,9 @@ constexpr int kChunkBytes = 64 * 128;             // 64 token rows x 64 latent c
 constexpr int kStageBytes = 5 * kChunkBytes;      // up to 5 chunks per CTA
 constexpr int kXBytes = 128 * 128;                // one half of S: 128 heads x 64 tokens, fp16
 constexpr int kPBytes = 128 * 128;                // P: 128 heads x 64 tokens, bf16
-constexpr int kRedBytes = (2 * 2 + 1) * 128 * 4;  // tile max of each token half (two slots), l of half 1
 constexpr int kBarBytes = 512;
-// stages | partner's S half x2 | P | max / sum exchange | barriers
-constexpr int kSmem = 1024 + kStages * kStageBytes + 2 * kXBytes + kPBytes + kRedBytes + kBarBytes;
+// stages | partner's S half x2 | P | barriers
+constexpr int kSmem = 1024 + kStages * kStageBytes + 2 * kXBytes + kPBytes + kBarBytes;
 // TMEM columns: O half [0,256), S [256,320), Q half (bf16 pairs) [320,480),
 // this CTA's fp16-rounded S half (pairs) [480,512)
 constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 320, kTmemX = 480, kTmemCols = 512;
@@ -103,8 +104,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   uint8_t* stages = smem;
   uint8_t* xpeer = stages + kStages * kStageBytes;  // [2] the partner's half of S (fp16), written by the partner
   uint8_t* pbuf = xpeer + 2 * kXBytes;              // P (bf16), MMA A operand
-  float* red = reinterpret_cast<float*>(pbuf + kPBytes);  // [2 slots][2 halves][128] tile max, then [128] l
-  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + kRedBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(pbuf + kPBytes);
   uint64_t* empty = full + kStages;
   uint64_t* s_full = empty + kStages;
   uint64_t* s_free = s_full + 1;
@@ -117,9 +117,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   uint64_t* q_full = p_free + 1;
   uint64_t* o_done = q_full + 1;
   uint64_t* drain = o_done + 1;
-  uint64_t* m_bar = drain + 1;       // [2 slots][4 quarters] both token halves posted their tile max
-  uint64_t* l_bar = m_bar + 8;       // [4 quarters] token half 1 posted its l at the end of a piece
-  uint32_t* sig = reinterpret_cast<uint32_t*>(l_bar + 4);  // [2 slots][8] landing words of the partner's slot-free signals
+  uint32_t* sig = reinterpret_cast<uint32_t*>(drain + 1);  // [2 slots][8] landing words of the partner's slot-free signals
   uint32_t* tmem_slot = sig + 16;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -142,13 +140,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       mbar_init(&x_full[i], 1);   // armed once per phase with the expected bytes
       mbar_init(&x_free[i], 1);   // armed by the exchange before each use; 8 x 4 signal bytes from the partner
     }
-    mbar_init(p_full, 256);
+    mbar_init(p_full, 8);       // one arrival per softmax warp
     mbar_init(p_free, 1);
     mbar_init(q_full, 128);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&m_bar[i], 2);  // one arrival per warp of the pair
-    for (int i = 0; i < 4; ++i) mbar_init(&l_bar[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
     // phase 0 of both exchange slots expects the partner's 16 KB
@@ -198,31 +194,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         if (!mbar_wait(q_full, piece & 1, wc)) return;
         tc_fence_after();
         const int nt = p.t1 - p.t0;
-        // S first, so the exchange never waits behind a PV.
+        // PV first: it gates the softmax of the next tile, while S only has
+        // to be ready by the time the exchange warps come back for it.
         int ns = 0, npv = 0;
         uint32_t spins = 0;
         uint64_t t_idle = 0;
         while (npv < nt) {
           bool issued = false;
-          if (ns < nt) {
-            const int g = it + ns;
-            const int s = g % kStages;
-            if (mbar_try_wait(smem_u32(&full[s]), (g / kStages) & 1) && mbar_try_wait(smem_u32(s_free), (g & 1) ^ 1)) {
-              tc_fence_after();
-              const uint32_t st = smem_u32(stages + s * kStageBytes);
-              for (int ci = 0; ci < nchunks; ++ci) {
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                  mma_ts(tmem + kTmemS, tmem + kTmemQ + ci * 32 + kk * 8,
-                         sdesc_sw128(st + ci * kChunkBytes + kk * 32, 16, 1024), idesc_s, (ci | kk) ? 1u : 0u);
-                }
-              }
-              mma_commit(s_full);
-              ++ns;
-              issued = true;
-            }
-          }
-          if (!issued && npv < ns) {
+          if (npv < ns) {
             const int g = it + npv;
             const int s = g % kStages;
             if (mbar_try_wait(smem_u32(p_full), g & 1)) {
@@ -237,6 +216,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
               mma_commit(&empty[s]);
               if (npv == nt - 1) mma_commit(o_done);
               ++npv;
+              issued = true;
+            }
+          }
+          if (!issued && ns < nt) {
+            const int g = it + ns;
+            const int s = g % kStages;
+            if (mbar_try_wait(smem_u32(&full[s]), (g / kStages) & 1) && mbar_try_wait(smem_u32(s_free), (g & 1) ^ 1)) {
+              tc_fence_after();
+              const uint32_t st = smem_u32(stages + s * kStageBytes);
+              for (int ci = 0; ci < nchunks; ++ci) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  mma_ts(tmem + kTmemS, tmem + kTmemQ + ci * 32 + kk * 8,
+                         sdesc_sw128(st + ci * kChunkBytes + kk * 32, 16, 1024), idesc_s, (ci | kk) ? 1u : 0u);
+                }
+              }
+              mma_commit(s_full);
+              ++ns;
               issued = true;
             }
           }
@@ -341,22 +338,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int q4 = warp & 3;
-    const int hf = (warp - 6) >> 2;  // token half of the tile: [32 hf, 32 hf + 32)
-    const int h = q4 * 32 + lane;
-    const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const int hs = (warp - 6) >> 2;  // which 16 heads of the lane quarter
+    const int th = lane >> 4;        // token half of the tile: [32 th, 32 th + 32)
+    const int h = q4 * 32 + hs * 16 + (lane & 15);
+    const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32 + hs * 16) << 16);
     const int sw = h & 7;
     const bool leader = warp == 6;   // re-arms the exchange barriers
     const uint32_t peer_row = smem_u32(xpeer) + h * 128;
     const uint32_t p_row = smem_u32(pbuf) + h * 128;
     const uint32_t xfree_peer = mapa(smem_u32(x_free), peer);
     const uint32_t sig_peer = mapa(smem_u32(sig), peer) + (warp - 6) * 4;
-    float* l_other = red + 4 * 128;
     int it = 0, piece = 0;
     for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
       if (*abort_flag) return;
       const bool head = h < a.n_h;
       const int L1 = a.seqlen[p.b] + 1;
-      float m_run = -INFINITY, l_run = 0.f;
+      float m_run = -INFINITY, l_run = 0.f;  // l_run: this thread's token half only
       const int nt = p.t1 - p.t0;
       for (int k = 0; k < nt; ++k) {
         const int g = it + k;
@@ -366,12 +363,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         if (!mbar_wait(xo_full, g & 1, wc)) return;
         if (!mbar_wait<true>(&x_full[slot], ph, wc)) return;
         tc_fence_after();
-        // ---- full scores of this warp's 32 tokens (same bits in both CTAs)
+        // ---- full scores of this thread's 32 tokens (same bits in both CTAs)
         uint32_t own[16];
-        tmem_ld16(tl + kTmemX + hf * 16, *reinterpret_cast<float(*)[16]>(own));
+        tmem_ld16x2(tl + kTmemX, own);
         uint4 pv[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) pv[i] = ld_shared_v4(peer_row + slot * kXBytes + (((hf * 4 + i) ^ sw) << 4));
+        for (int i = 0; i < 4; ++i) pv[i] = ld_shared_v4(peer_row + slot * kXBytes + (((th * 4 + i) ^ sw) << 4));
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
@@ -381,31 +378,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           // before the slot is released, so no byte can land ahead of it
           if (leader) mbar_arrive_expect_tx(&x_full[slot], kXBytes);
         }
-        const int valid = min(64, L1 - t * 64) - hf * 32;  // valid tokens of this half (may be <= 0)
+        const int valid = min(64, L1 - t * 64) - th * 32;  // valid tokens of this half (may be <= 0)
         float sc[32];
-        float mh = -INFINITY;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint32_t vv[4] = {pv[i].x, pv[i].y, pv[i].z, pv[i].w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int j = 8 * i + 2 * e;
             const float2 x = unpack_half2(own[4 * i + e]), y = unpack_half2(vv[e]);
-            sc[j] = j < valid ? x.x + y.x : -INFINITY;
-            sc[j + 1] = j + 1 < valid ? x.y + y.y : -INFINITY;
-            mh = fmaxf(mh, fmaxf(sc[j], sc[j + 1]));
+            sc[8 * i + 2 * e] = x.x + y.x;
+            sc[8 * i + 2 * e + 1] = x.y + y.y;
           }
         }
         // every value read from the partner's half is consumed: hand the slot back
         __syncwarp();
         if (lane == 0) st_async_b32(sig_peer + slot * 32, 0u, xfree_peer + slot * 8);
-        // tile max over both halves (a barrier wait that gives up, unlike bar.sync,
-        // so a partner warp that aborted cannot strand this one)
-        red[(slot * 2 + hf) * 128 + h] = mh;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&m_bar[slot * 4 + q4]);
-        if (!mbar_wait(&m_bar[slot * 4 + q4], ph, wc)) return;
-        const float mt = fmaxf(mh, red[(slot * 2 + (hf ^ 1)) * 128 + h]);
+        if (__any_sync(0xffffffffu, valid < 32)) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j >= valid) sc[j] = -INFINITY;
+        }
+        float mh = sc[0];
+#pragma unroll
+        for (int j = 1; j < 32; ++j) mh = fmaxf(mh, sc[j]);
+        const float mt = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));  // the head's other token half
         float m_new = m_run, alpha = 1.f;
         bool rescale = false;
         if (k == 0) {
@@ -419,10 +415,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         float lsum = 0.f;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const __nv_bfloat162 b2 =
-              __floats2bfloat162_rn(ex2_approx(sc[2 * j] - m_new), ex2_approx(sc[2 * j + 1] - m_new));
-          const float2 f = __bfloat1622float2(b2);
-          lsum += f.x + f.y;
+          const float p0 = ex2_approx(sc[2 * j] - m_new), p1 = ex2_approx(sc[2 * j + 1] - m_new);
+          lsum += p0 + p1;
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
           pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
         }
         l_run = l_run * alpha + lsum;
@@ -431,59 +426,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         if (!mbar_wait(p_free, (g & 1) ^ 1, wc)) return;
         tc_fence_after();
         if (__any_sync(0xffffffffu, rescale)) {
-          for (int c = hf * 128; c < hf * 128 + 128; c += 32) {
-            uint32_t o[32];
-            tmem_ld32(tl + kTmemO + c, o);
+          for (int c = 0; c < 256; c += 32) {
+            uint32_t o[16];
+            tmem_ld16x2(tl + kTmemO + c, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tl + kTmemO + c, o);
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st16x2(tl + kTmemO + c, o);
           }
           tmem_wait_st();
         }
-        if (valid + hf * 32 < 64) {
+        const int v64 = valid + th * 32;
+        if (v64 < 64) {
           // rows past the sequence may hold anything (even NaN); 0 * NaN would
           // poison O, so the rows this CTA multiplies into O are zeroed
-          const int v64 = valid + hf * 32;
           uint8_t* st = stages + (g % kStages) * kStageBytes;
           const int n16 = (64 - v64) * 32;
-          for (int idx = hf * 128 + h; idx < n16; idx += 256) {
+          for (int idx = (warp - 6) * 32 + lane; idx < n16; idx += 256) {
             const int row = v64 + (idx >> 5), c16 = idx & 31;
             *reinterpret_cast<uint4*>(st + (c16 >> 3) * kChunkBytes + row * 128 + (c16 & 7) * 16) = make_uint4(0, 0, 0, 0);
           }
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          st_shared_v4(p_row + (((hf * 4 + i) ^ sw) << 4), make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
+          st_shared_v4(p_row + (((th * 4 + i) ^ sw) << 4), make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(p_full);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
       }
-      // ---- epilogue of the piece: unnormalised O_r (this warp's 128 columns), m, l
+      // ---- epilogue of the piece: unnormalised O_r, m, l
       if (!mbar_wait(o_done, piece & 1, wc)) return;
       tc_fence_after();
-      float* dst = a.o_part + (static_cast<long long>(p.slot) * a.n_h + h) * 512 + rank * 256;
-      for (int c = hf * 128; c < hf * 128 + 128; c += 32) {
-        uint32_t o[32];
-        tmem_ld32(tl + kTmemO + c, o);
+      float* dst = a.o_part + (static_cast<long long>(p.slot) * a.n_h + h) * 512 + rank * 256 + th * 16;
+      for (int c = 0; c < 256; c += 32) {
+        uint32_t o[16];
+        tmem_ld16x2(tl + kTmemO + c, o);
         tmem_wait_ld();
         if (head) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
+          for (int i = 0; i < 4; ++i)
             reinterpret_cast<float4*>(dst + c)[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
                                                                 __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
         }
       }
-      if (hf == 1) {
-        l_other[h] = l_run;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&l_bar[q4]);
-      } else if (!mbar_wait(&l_bar[q4], piece & 1, wc)) {
-        return;
-      }
-      if (rank == 0 && hf == 0 && head) {
+      const float l_head = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+      if (rank == 0 && th == 0 && head) {
         a.ml_part[(static_cast<long long>(p.slot) * a.n_h + h) * 2] = m_run;
-        a.ml_part[(static_cast<long long>(p.slot) * a.n_h + h) * 2 + 1] = l_run + l_other[h];
+        a.ml_part[(static_cast<long long>(p.slot) * a.n_h + h) * 2 + 1] = l_head;
       }
       tc_fence_before();
       it += nt;
