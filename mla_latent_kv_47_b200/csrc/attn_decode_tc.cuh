@@ -38,7 +38,8 @@
 //               max is one shuffle.  Online softmax with a lazily refreshed
 //               max (O is rescaled only when a tile's max exceeds the running
 //               one by more than 2^8), P (bf16) into shared memory, and the
-//               per-piece epilogue
+//               per-piece epilogue.  P alternates between two buffers, so P(j+1)
+//               is written while PV(j) still reads P(j).
 // The exchange warps use thread = head = TMEM lane (warp w owns lanes
 // 32 (w mod 4) ..).
 #pragma once
@@ -59,8 +60,8 @@ constexpr int kStageBytes = 5 * kChunkBytes;      // up to 5 chunks per CTA
 constexpr int kXBytes = 128 * 128;                // one half of S: 128 heads x 64 tokens, fp16
 constexpr int kPBytes = 128 * 128;                // P: 128 heads x 64 tokens, bf16
 constexpr int kBarBytes = 512;
-// stages | partner's S half x2 | P | barriers
-constexpr int kSmem = 1024 + kStages * kStageBytes + 2 * kXBytes + kPBytes + kBarBytes;
+// stages | partner's S half x2 | P x2 | barriers
+constexpr int kSmem = 1024 + kStages * kStageBytes + 2 * kXBytes + 2 * kPBytes + kBarBytes;
 // TMEM columns: O half [0,256), S [256,320), Q half (bf16 pairs) [320,480),
 // this CTA's fp16-rounded S half (pairs) [480,512)
 constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 320, kTmemX = 480, kTmemCols = 512;
@@ -103,8 +104,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   uint8_t* smem = align1024(smem_raw);
   uint8_t* stages = smem;
   uint8_t* xpeer = stages + kStages * kStageBytes;  // [2] the partner's half of S (fp16), written by the partner
-  uint8_t* pbuf = xpeer + 2 * kXBytes;              // P (bf16), MMA A operand
-  uint64_t* full = reinterpret_cast<uint64_t*>(pbuf + kPBytes);
+  uint8_t* pbuf = xpeer + 2 * kXBytes;              // [2] P (bf16), MMA A operand
+  uint64_t* full = reinterpret_cast<uint64_t*>(pbuf + 2 * kPBytes);
   uint64_t* empty = full + kStages;
   uint64_t* s_full = empty + kStages;
   uint64_t* s_free = s_full + 1;
@@ -112,9 +113,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   uint64_t* xo_free = xo_full + 1;   // own half read out (softmax -> exchange)
   uint64_t* x_full = xo_free + 1;    // [2] partner's half landed (st.async bytes)
   uint64_t* x_free = x_full + 2;     // [2] partner's half consumed (arrivals from the partner's softmax)
-  uint64_t* p_full = x_free + 2;
-  uint64_t* p_free = p_full + 1;
-  uint64_t* q_full = p_free + 1;
+  uint64_t* p_full = x_free + 2;     // [2]
+  uint64_t* p_free = p_full + 2;     // [2]
+  uint64_t* q_full = p_free + 2;
   uint64_t* o_done = q_full + 1;
   uint64_t* drain = o_done + 1;
   uint32_t* sig = reinterpret_cast<uint32_t*>(drain + 1);  // [2 slots][8] landing words of the partner's slot-free signals
@@ -140,8 +141,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       mbar_init(&x_full[i], 1);   // armed once per phase with the expected bytes
       mbar_init(&x_free[i], 1);   // armed by the exchange before each use; 8 x 4 signal bytes from the partner
     }
-    mbar_init(p_full, 8);       // one arrival per softmax warp
-    mbar_init(p_free, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&p_full[i], 8);   // one arrival per softmax warp
+      mbar_init(&p_free[i], 1);
+    }
     mbar_init(q_full, 128);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
@@ -187,7 +190,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     if (elect_one()) {
       constexpr uint32_t idesc_s = idesc_bf16(128, 64, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(128, 256, false, true);
-      const uint32_t pb = smem_u32(pbuf);
       int it = 0, piece = 0;
       for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
         if (*abort_flag) return;
@@ -204,15 +206,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           if (npv < ns) {
             const int g = it + npv;
             const int s = g % kStages;
-            if (mbar_try_wait(smem_u32(p_full), g & 1)) {
+            const int b = g & 1;
+            if (mbar_test_wait(smem_u32(&p_full[b]), (g >> 1) & 1)) {
               tc_fence_after();
               const uint32_t st = smem_u32(stages + s * kStageBytes);
+              const uint32_t pb = smem_u32(pbuf + b * kPBytes);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 mma_ss(tmem + kTmemO, sdesc_sw128(pb + kk * 32, 16, 1024), sdesc_sw128(st + kk * 2048, 8192, 1024),
                        idesc_pv, (npv > 0 || kk > 0) ? 1u : 0u);
               }
-              mma_commit(p_free);
+              mma_commit(&p_free[b]);
               mma_commit(&empty[s]);
               if (npv == nt - 1) mma_commit(o_done);
               ++npv;
@@ -222,7 +226,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           if (!issued && ns < nt) {
             const int g = it + ns;
             const int s = g % kStages;
-            if (mbar_try_wait(smem_u32(&full[s]), (g / kStages) & 1) && mbar_try_wait(smem_u32(s_free), (g & 1) ^ 1)) {
+            if (mbar_test_wait(smem_u32(&full[s]), (g / kStages) & 1) && mbar_test_wait(smem_u32(s_free), (g & 1) ^ 1)) {
               tc_fence_after();
               const uint32_t st = smem_u32(stages + s * kStageBytes);
               for (int ci = 0; ci < nchunks; ++ci) {
@@ -422,10 +426,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         }
         l_run = l_run * alpha + lsum;
         m_run = m_new;
-        // ---- PV(g-1) retired: the P buffer is free and O settled
-        if (!mbar_wait(p_free, (g & 1) ^ 1, wc)) return;
+        // ---- P buffer b is free once PV(g-2) retired
+        const int b = g & 1;
+        if (!mbar_wait(&p_free[b], ph ^ 1, wc)) return;
         tc_fence_after();
         if (__any_sync(0xffffffffu, rescale)) {
+          // O must hold PV(g-1) before it is scaled (k >= 1 here, so g >= 1)
+          if (!mbar_wait(&p_free[b ^ 1], ((g - 1) >> 1) & 1, wc)) return;
+          tc_fence_after();
           for (int c = 0; c < 256; c += 32) {
             uint32_t o[16];
             tmem_ld16x2(tl + kTmemO + c, o);
@@ -449,11 +457,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          st_shared_v4(p_row + (((th * 4 + i) ^ sw) << 4), make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
+          st_shared_v4(p_row + b * kPBytes + (((th * 4 + i) ^ sw) << 4),
+                       make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive(&p_full[b]);
       }
       // ---- epilogue of the piece: unnormalised O_r, m, l
       if (!mbar_wait(o_done, piece & 1, wc)) return;
