@@ -41,6 +41,7 @@ struct TokenMap {
   int row_elems;             // d_c + d_R
   int d_c, d_R;
   double log2_base;          // log2(rope_base)
+  const float2* rope;        // NULL, or (cos, sin) of pair i at token n: rope[n * d_R / 2 + i]
 };
 
 __device__ __forceinline__ int tok_pos(const TokenMap& t, int n) { return t.pos ? t.pos[n] : t.pos_base + n; }
@@ -63,6 +64,19 @@ __device__ __noinline__ void rope_cos_sin(int pos, double inv_freq, float& c, fl
   double r = fma(-k, two_pi_hi, phi);
   r = fma(-k, two_pi_lo, r);
   sincosf(static_cast<float>(r), &s, &c);
+}
+
+// (cos, sin) of pair i at token n: from the call's table when there is one,
+// else computed here.  Both give the same bits (the table is filled by
+// rope_table_kernel with rope_cos_sin).
+__device__ __forceinline__ void rope_cs(const TokenMap& t, int n, int i, double inv_freq, float& c, float& s) {
+  if (t.rope) {
+    const float2 v = t.rope[static_cast<long long>(n) * (t.d_R >> 1) + i];
+    c = v.x;
+    s = v.y;
+  } else {
+    rope_cos_sin(tok_pos(t, n), inv_freq, c, s);
+  }
 }
 
 // Rotated value of component j (of an interleaved pair) given its own value y
@@ -109,7 +123,7 @@ __device__ __forceinline__ void epi_apply(const Epi& e, const TokenMap& tk, int 
     case EPI_QLAT_ROPE: {
       const int hh = m / tk.d_R, j = m % tk.d_R;
       float c, s;
-      rope_cos_sin(tok_pos(tk, n), inv_freq, c, s);
+      rope_cs(tk, n, j >> 1, inv_freq, c, s);
       const float r = rope_apply(j, y, yp, c, s);
       store_elem<T>(e.out, static_cast<long long>(n) * e.ld + hh * e.hs + tk.d_c + j, r * e.scale, e.out_f32);
       break;
@@ -125,7 +139,7 @@ __device__ __forceinline__ void epi_apply(const Epi& e, const TokenMap& tk, int 
     case EPI_CACHE_KR: {
       const long long row = cache_row(tk, n, status);
       float c, s;
-      rope_cos_sin(tok_pos(tk, n), inv_freq, c, s);
+      rope_cs(tk, n, m >> 1, inv_freq, c, s);
       const float r = rope_apply(m, y, yp, c, s);
       if (row >= 0) store_elem<T>(tk.cache, row * tk.row_elems + tk.d_c + m, r, 0);
       break;
@@ -133,7 +147,7 @@ __device__ __forceinline__ void epi_apply(const Epi& e, const TokenMap& tk, int 
     case EPI_QP_ROPE: {
       const int hh = m / tk.d_R, j = m % tk.d_R;
       float c, s;
-      rope_cos_sin(tok_pos(tk, n), inv_freq, c, s);
+      rope_cs(tk, n, j >> 1, inv_freq, c, s);
       const float r = rope_apply(j, y, yp, c, s);
       store_elem<T>(e.out, static_cast<long long>(n) * e.ld + hh * e.hs + e.col0 + j, r * e.scale, e.out_f32);
       break;
@@ -146,50 +160,100 @@ __device__ __forceinline__ void epi_apply(const Epi& e, const TokenMap& tk, int 
   }
 }
 
-// Per-kind form of epi_apply, so that a chunk of outputs is dispatched once
-// (one switch per chunk instead of per element keeps the epilogue code small).
-template <int KIND, typename T>
-__device__ __forceinline__ void epi_one(const Epi& e, const TokenMap& tk, int m, int n, int head, float y, float yp,
-                                        double inv_freq, int* status) {
-  if (KIND == EPI_STORE) {
-    store_elem<T>(e.out, static_cast<long long>(n) * e.ld + e.col0 + m, y * e.scale, e.out_f32);
-  } else if (KIND == EPI_PER_HEAD) {
-    store_elem<T>(e.out, static_cast<long long>(n) * e.ld + head * e.hs + m, y * e.scale, e.out_f32);
-  } else if (KIND == EPI_HEADS) {
-    const int hh = m / e.dh, j = m % e.dh;
-    store_elem<T>(e.out, static_cast<long long>(n) * e.ld + hh * e.hs + e.col0 + j, y * e.scale, e.out_f32);
+// ---- staged epilogue of the tensor-core GEMM.
+// Phase 1 (thread = output row m of the tile): each output's final value
+// (scale, RoPE) goes into a staging tile in shared memory, column-major
+// ([n][128 rows]), so consecutive rows of one token sit side by side.
+// Phase 2 (all epilogue threads): runs of 16 bytes (8 bf16 or 4 fp32 rows of
+// one token) are copied to their destination with one vector store each.
+// Every kind maps a run of 8 consecutive rows to 8 consecutive destination
+// elements (head blocks are multiples of 8 rows), so one address per run.
+
+template <int KIND>
+__device__ __forceinline__ float epi_value(const Epi& e, const TokenMap& tk, int m, int n, float y, float yp,
+                                           double inv_freq) {
+  if (KIND == EPI_QLAT_ROPE || KIND == EPI_QP_ROPE) {
+    const int j = m % tk.d_R;
+    float c, s;
+    rope_cs(tk, n, j >> 1, inv_freq, c, s);
+    return rope_apply(j, y, yp, c, s) * e.scale;
+  } else if (KIND == EPI_CACHE_KR) {
+    float c, s;
+    rope_cs(tk, n, m >> 1, inv_freq, c, s);
+    return rope_apply(m, y, yp, c, s);
   } else if (KIND == EPI_CACHE_CKV) {
-    const long long row = cache_row(tk, n, status);
-    if (row >= 0) store_elem<T>(tk.cache, row * tk.row_elems + m, y, 0);
+    return y;
   } else {
-    epi_apply<T>(e, tk, m, n, head, y, yp, inv_freq, status);  // rotary kinds
+    return y * e.scale;
   }
 }
 
-// Applies the epilogue to outputs (m, n0 + j), j < NV, held by this thread;
-// whole warps call it (the rotary partner is a lane shuffle away).
-template <int KIND, int NV, typename T>
-__device__ __forceinline__ void epi_chunk(const Epi& e, const TokenMap& tk, int m, int n0, int head, const float* v,
-                                          int n_end, bool m_ok, double inv_freq, int* status) {
+// Phase 1 for NV consecutive columns n0.. held by this thread (whole warps
+// call it: the rotary partner row is a lane shuffle away).  Columns at or
+// past n_end are staged as zero and never stored.
+template <int KIND, int NV>
+__device__ __forceinline__ void epi_stage_kind(const Epi& e, const TokenMap& tk, int m, int n0, int n_end,
+                                               const float* v, double inv_freq, uint8_t* stage, int nl0, int ml) {
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
-    const bool rot = (KIND == EPI_QLAT_ROPE || KIND == EPI_CACHE_KR || KIND == EPI_QP_ROPE);
+    constexpr bool rot = (KIND == EPI_QLAT_ROPE || KIND == EPI_CACHE_KR || KIND == EPI_QP_ROPE);
     const float yp = rot ? __shfl_xor_sync(0xffffffffu, v[j], 1) : 0.f;
-    if (n0 + j < n_end && m_ok) epi_one<KIND, T>(e, tk, m, n0 + j, head, v[j], yp, inv_freq, status);
+    const float r = (n0 + j < n_end) ? epi_value<KIND>(e, tk, m, n0 + j, v[j], yp, inv_freq) : 0.f;
+    const int idx = (nl0 + j) * 128 + ml;
+    if (e.out_f32) {
+      reinterpret_cast<float*>(stage)[idx] = r;
+    } else {
+      reinterpret_cast<__nv_bfloat16*>(stage)[idx] = __float2bfloat16_rn(r);
+    }
   }
 }
 
-template <int NV, typename T>
-__device__ __forceinline__ void epi_dispatch(const Epi& e, const TokenMap& tk, int m, int n0, int head, const float* v,
-                                             int n_end, bool m_ok, double inv_freq, int* status) {
+template <int NV>
+__device__ __forceinline__ void epi_stage(const Epi& e, const TokenMap& tk, int m, int n0, int n_end, const float* v,
+                                          double inv_freq, uint8_t* stage, int nl0, int ml) {
   switch (e.kind) {
-    case EPI_STORE: epi_chunk<EPI_STORE, NV, T>(e, tk, m, n0, head, v, n_end, m_ok, inv_freq, status); break;
-    case EPI_PER_HEAD: epi_chunk<EPI_PER_HEAD, NV, T>(e, tk, m, n0, head, v, n_end, m_ok, inv_freq, status); break;
-    case EPI_HEADS: epi_chunk<EPI_HEADS, NV, T>(e, tk, m, n0, head, v, n_end, m_ok, inv_freq, status); break;
-    case EPI_CACHE_CKV: epi_chunk<EPI_CACHE_CKV, NV, T>(e, tk, m, n0, head, v, n_end, m_ok, inv_freq, status); break;
-    case EPI_QLAT_ROPE: epi_chunk<EPI_QLAT_ROPE, NV, T>(e, tk, m, n0, head, v, n_end, m_ok, inv_freq, status); break;
-    case EPI_CACHE_KR: epi_chunk<EPI_CACHE_KR, NV, T>(e, tk, m, n0, head, v, n_end, m_ok, inv_freq, status); break;
-    default: epi_chunk<EPI_QP_ROPE, NV, T>(e, tk, m, n0, head, v, n_end, m_ok, inv_freq, status); break;
+    case EPI_QLAT_ROPE: epi_stage_kind<EPI_QLAT_ROPE, NV>(e, tk, m, n0, n_end, v, inv_freq, stage, nl0, ml); break;
+    case EPI_QP_ROPE: epi_stage_kind<EPI_QP_ROPE, NV>(e, tk, m, n0, n_end, v, inv_freq, stage, nl0, ml); break;
+    case EPI_CACHE_KR: epi_stage_kind<EPI_CACHE_KR, NV>(e, tk, m, n0, n_end, v, inv_freq, stage, nl0, ml); break;
+    case EPI_CACHE_CKV: epi_stage_kind<EPI_CACHE_CKV, NV>(e, tk, m, n0, n_end, v, inv_freq, stage, nl0, ml); break;
+    default: epi_stage_kind<EPI_STORE, NV>(e, tk, m, n0, n_end, v, inv_freq, stage, nl0, ml); break;
+  }
+}
+
+// Destination of the run of rows m.. (a multiple of 8) of token n, or nullptr
+// when the token's cache row is out of bounds (recorded in the status word).
+__device__ __forceinline__ uint8_t* epi_addr(const Epi& e, const TokenMap& tk, int m, int n, int head, int* status) {
+  const int es = e.out_f32 ? 4 : 2;
+  long long idx;
+  switch (e.kind) {
+    case EPI_QLAT_ROPE: idx = static_cast<long long>(n) * e.ld + (m / tk.d_R) * e.hs + tk.d_c + m % tk.d_R; break;
+    case EPI_QP_ROPE: idx = static_cast<long long>(n) * e.ld + (m / tk.d_R) * e.hs + e.col0 + m % tk.d_R; break;
+    case EPI_HEADS: idx = static_cast<long long>(n) * e.ld + (m / e.dh) * e.hs + e.col0 + m % e.dh; break;
+    case EPI_PER_HEAD: idx = static_cast<long long>(n) * e.ld + head * e.hs + m; break;
+    case EPI_CACHE_CKV:
+    case EPI_CACHE_KR: {
+      const long long row = cache_row(tk, n, status);
+      if (row < 0) return nullptr;
+      return static_cast<uint8_t*>(tk.cache) + (row * tk.row_elems + (e.kind == EPI_CACHE_KR ? tk.d_c : 0) + m) * 2;
+    }
+    default: idx = static_cast<long long>(n) * e.ld + e.col0 + m; break;
+  }
+  return static_cast<uint8_t*>(e.out) + idx * es;
+}
+
+// Phase 2: the staged tile (tokens n_base .. n_base + n_cols - 1, rows m0 ..
+// m0 + 127) to global memory, 16 bytes per store; thread tid of nthr.
+__device__ __forceinline__ void epi_flush(const Epi& e, const TokenMap& tk, int m0, int rows_valid, int n_base, int n_cols,
+                                          int n_end, int head, const uint8_t* stage, int tid, int nthr, int* status) {
+  const int vec = e.out_f32 ? 4 : 8;  // rows per 16-byte run
+  const int runs = 128 / vec;
+  const int es = e.out_f32 ? 4 : 2;
+  for (int id = tid; id < n_cols * runs; id += nthr) {
+    const int nl = id / runs, ml = (id % runs) * vec;
+    const int n = n_base + nl, m = m0 + ml;
+    if (n >= n_end || m >= rows_valid) continue;
+    uint8_t* dst = epi_addr(e, tk, m, n, head, status);
+    if (dst) *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(stage + (nl * 128 + ml) * es);
   }
 }
 
@@ -200,6 +264,23 @@ __device__ __forceinline__ double epi_inv_freq(const Epi& e, const TokenMap& tk,
   if (!epi_needs_rope(e.kind)) return 0.0;
   const int j = (e.kind == EPI_CACHE_KR) ? m : (m % tk.d_R);
   return rope_inv_freq(j >> 1, tk.d_R, tk.log2_base);
+}
+
+// (cos, sin) of every rotary pair of the call's T tokens, for the epilogues
+// of the GEMMs that follow (one evaluation per (token, pair) instead of one per
+// output element).
+__global__ void __launch_bounds__(256) rope_table_kernel(const TokenMap tk, int T, float2* out) {
+  griddep_wait();  // positions may be written, and the previous call's epilogues may still read `out`
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  const int half = tk.d_R >> 1;
+  const long long total = static_cast<long long>(T) * half;
+  for (long long idx = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x; idx < total;
+       idx += static_cast<long long>(gridDim.x) * 256) {
+    const int n = static_cast<int>(idx / half), i = static_cast<int>(idx % half);
+    float c, s;
+    rope_cos_sin(tok_pos(tk, n), rope_inv_freq(i, tk.d_R, tk.log2_base), c, s);
+    out[idx] = make_float2(c, s);
+  }
 }
 
 }  // namespace mla

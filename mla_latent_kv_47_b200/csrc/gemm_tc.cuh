@@ -46,22 +46,25 @@ struct GemmArgs {
   TokenMap tok;
 };
 
-// One pipeline stage holds KBB consecutive 64-wide K blocks of A (128 rows)
-// and of X (BN rows): fewer, larger stages mean fewer barrier round trips and
-// longer runs of each weight row in flight.
-template <int BN, int STAGES, int KBB>
+// One pipeline stage holds KBB consecutive 64-wide K blocks of A (MT tiles of
+// 128 rows) and of X (BN rows): fewer, larger stages mean fewer barrier round
+// trips and longer runs of each weight row in flight.
+template <int BN, int STAGES, int KBB, int MT = 1>
 struct GemmSmem {
   static constexpr int kSlabA = 16384;     // 128 rows x 128 B
   static constexpr int kSlabB = BN * 128;  // BN rows x 128 B
-  static constexpr int kA = KBB * kSlabA;
+  static constexpr int kA = KBB * MT * kSlabA;
   static constexpr int kB = KBB * kSlabB;
   static constexpr int kStage = kA + kB;
   static constexpr int kBytes = 1024 + STAGES * kStage + 256;
 };
 
-template <int BN, bool A_MN, int STAGES, int KBB>
+// MT > 1 (per-head modes, no split-K): one CTA computes MT consecutive
+// 128-row tiles of a head against the same X block, one TMEM accumulator each.
+template <int BN, bool A_MN, int STAGES, int KBB, int MT = 1>
 __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ GemmArgs args) {
-  using L = GemmSmem<BN, STAGES, KBB>;
+  using L = GemmSmem<BN, STAGES, KBB, MT>;
+  static_assert(STAGES * L::kStage >= BN * 128 * 4, "the pipeline stages must hold an fp32 staging tile");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
@@ -74,7 +77,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+  constexpr uint32_t kTmemCols = BN * MT < 32 ? 32 : BN * MT;
+  static_assert(BN * MT <= 512 && (BN * MT & (BN * MT - 1)) == 0, "TMEM columns: a power of two <= 512");
 
   // ---- which tile
   const int mt = blockIdx.x, nt = blockIdx.y, split = blockIdx.z;
@@ -84,8 +88,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     m0 = (mt - args.seg_tile0[seg]) * 128;
   } else {
     const int tph = args.seg_tile0[1];
-    head = mt / tph;
-    m0 = (mt % tph) * 128;
+    head = (mt * MT) / tph;
+    m0 = ((mt * MT) % tph) * 128;
   }
   const int kb0 = split * args.kb_per_split;
   const int kb1 = min(args.kb_total, kb0 + args.kb_per_split);
@@ -119,21 +123,25 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     if (elect_one()) {
       const uint64_t polA = policy_evict_first();
       const uint64_t polB = policy_evict_last();
-      const uint32_t bytesA = A_MN ? 16384u : static_cast<uint32_t>(args.boxA_rows[seg]) * 128u;
+      const uint32_t bytesA = MT * (A_MN ? 16384u : static_cast<uint32_t>(args.boxA_rows[seg]) * 128u);
       const uint32_t bytesB = static_cast<uint32_t>(args.boxB_rows) * 128u;
       auto stage_kbs = [&](int i) { return min(KBB, nkb - i * KBB); };
       auto load_a = [&](int i, int j) {
         const int s = i % STAGES;
         const int kb = kb0 + i * KBB + j;
-        uint8_t* a = sA + s * L::kA + j * L::kSlabA;
-        if (A_MN) {
-          const int y = head * args.head_rows + kb * 64;
-          tma_load_2d(a, &args.mapA[0], &full[s], m0, y, polA);
-          tma_load_2d(a + 8192, &args.mapA[0], &full[s], m0 + 64, y, polA);
-        } else if (args.mode == GEMM_HEAD_KMAJOR) {
-          tma_load_2d(a, &args.mapA[0], &full[s], kb * 64, head * args.head_rows + m0, polA);
-        } else {
-          tma_load_2d(a, &args.mapA[seg], &full[s], kb * 64, m0, polA);
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          uint8_t* a = sA + s * L::kA + (j * MT + t) * L::kSlabA;
+          const int mr = m0 + t * 128;
+          if (A_MN) {
+            const int y = head * args.head_rows + kb * 64;
+            tma_load_2d(a, &args.mapA[0], &full[s], mr, y, polA);
+            tma_load_2d(a + 8192, &args.mapA[0], &full[s], mr + 64, y, polA);
+          } else if (args.mode == GEMM_HEAD_KMAJOR) {
+            tma_load_2d(a, &args.mapA[0], &full[s], kb * 64, head * args.head_rows + mr, polA);
+          } else {
+            tma_load_2d(a, &args.mapA[seg], &full[s], kb * 64, mr, polA);
+          }
         }
       };
       auto load_b = [&](int i, int j) {
@@ -171,13 +179,16 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         tc_fence_after();
         const int kbs = min(KBB, nkb - i * KBB);
         for (int j = 0; j < kbs; ++j) {
-          const uint32_t a_base = smem_u32(sA + s * L::kA + j * L::kSlabA);
           const uint32_t b_base = smem_u32(sB + s * L::kB + j * L::kSlabB);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = A_MN ? sdesc_sw128(a_base + k * 2048, 8192, 1024) : sdesc_sw128(a_base + k * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(b_base + k * 32, 16, 1024);
-            mma_ss(tmem, ad, bd, idesc, (i > 0 || j > 0 || k > 0) ? 1u : 0u);
+          for (int t = 0; t < MT; ++t) {
+            const uint32_t a_base = smem_u32(sA + s * L::kA + (j * MT + t) * L::kSlabA);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t ad = A_MN ? sdesc_sw128(a_base + k * 2048, 8192, 1024) : sdesc_sw128(a_base + k * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(b_base + k * 32, 16, 1024);
+              mma_ss(tmem + t * BN, ad, bd, idesc, (i > 0 || j > 0 || k > 0) ? 1u : 0u);
+            }
           }
         }
         mma_commit(&empty[s]);
@@ -195,7 +206,6 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     if (!*abort_flag) {
       const Epi& e = args.epi[seg];
       const int m = m0 + row;
-      const bool m_ok = m < args.seg_rows[seg];
       const int tile_id = mt + gridDim.x * nt;
       if (args.splits > 1) {
         // split-K: store this split's partial tile ([BN/4 column groups][128 rows][4],
@@ -212,13 +222,23 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
             my[((c >> 2) + q) * 128 + row] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         }
       } else {
-        const double inv_freq = epi_inv_freq(e, args.tok, m);
+        // the pipeline stages are idle now (every MMA retired): they hold the staging tile
+        uint8_t* stage = sA;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
-          float v[16];
-          tmem_ld16(trow + c, v);
-          tmem_wait_ld();
-          epi_dispatch<16, __nv_bfloat16>(e, args.tok, m, nt * BN + c, head, v, args.N, m_ok, inv_freq, args.status);
+        for (int t = 0; t < MT; ++t) {
+          const int mr = m + t * 128;
+          const double inv_freq = epi_inv_freq(e, args.tok, mr);
+#pragma unroll 1
+          for (int c = 0; c < BN; c += 16) {
+            float v[16];
+            tmem_ld16(trow + t * BN + c, v);
+            tmem_wait_ld();
+            epi_stage<16>(e, args.tok, mr, nt * BN + c, args.N, v, inv_freq, stage, c, row);
+          }
+          named_bar_sync(1, 128);
+          epi_flush(e, args.tok, m0 + t * 128, args.seg_rows[seg], nt * BN, BN, args.N, head, stage, threadIdx.x - 64, 128,
+                    args.status);
+          if (t + 1 < MT) named_bar_sync(1, 128);  // the staging tile is refilled
         }
       }
     }
@@ -260,11 +280,13 @@ __global__ void __launch_bounds__(128) gemm_splitk_epilogue_kernel(const __grid_
     acc.z += t.z;
     acc.w += t.w;
   }
+  __shared__ __align__(16) uint8_t stage[4 * 128 * 4];
   const Epi& e = args.epi[seg];
   const int m = m0 + row;
   const float v[4] = {acc.x, acc.y, acc.z, acc.w};
-  epi_dispatch<4, __nv_bfloat16>(e, args.tok, m, cg * 4, head, v, args.N, m < args.seg_rows[seg], epi_inv_freq(e, args.tok, m),
-                                 args.status);
+  epi_stage<4>(e, args.tok, m, cg * 4, args.N, v, epi_inv_freq(e, args.tok, m), stage, 0, row);
+  __syncthreads();
+  epi_flush(e, args.tok, m0, args.seg_rows[seg], cg * 4, 4, args.N, head, stage, threadIdx.x, 128, args.status);
 }
 
 }  // namespace mla

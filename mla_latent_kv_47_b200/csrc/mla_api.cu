@@ -30,8 +30,8 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // number of key tokens); a call uses only its own region.
 struct Layout {
   size_t status, counters, gpart, base_end;
-  size_t tile_start, seg_start, cq, qc, qlat, olat, o, opart, ml, decode_end;
-  size_t p_cq, p_qp, p_rows, p_kc, p_v, p_out, prefill_end;
+  size_t tile_start, seg_start, rope, cq, qc, qlat, olat, o, opart, ml, decode_end;
+  size_t p_rope, p_cq, p_qp, p_rows, p_kc, p_v, p_out, prefill_end;
 };
 
 int elem_size(const mla_dims& d) { return d.dtype == MLA_FP32 ? 4 : 2; }
@@ -55,6 +55,7 @@ Layout make_layout_sized(const mla_dims& d, int max_batch, int max_tokens, int g
   L.base_end = off;
   L.tile_start = take((B + 1) * sizeof(int));
   L.seg_start = take((B + 1) * sizeof(int));
+  L.rope = take(B * (d.d_R / 2 + 1) * 2 * sizeof(float));
   L.cq = take(B * (d.d_cq ? d.d_cq : 1) * es);
   L.qc = take(B * nh * dh * es);
   L.qlat = take(B * nh * row * es);
@@ -64,6 +65,7 @@ Layout make_layout_sized(const mla_dims& d, int max_batch, int max_tokens, int g
   L.ml = take((B + workers) * nh * 2 * sizeof(float));
   L.decode_end = off;
   off = L.base_end;
+  L.p_rope = take(T * (d.d_R / 2 + 1) * 2 * sizeof(float));
   L.p_cq = take(T * (d.d_cq ? d.d_cq : 1) * es);
   L.p_qp = take(T * nh * (dh + d.d_R) * es);
   L.p_rows = take(T * row * es);
@@ -160,15 +162,16 @@ mla_status launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
-// Tile width, pipeline depth, K blocks per stage and CTA target of one GEMM launch.
+// Tile width, pipeline depth, K blocks per stage, CTA target and 128-row tiles
+// per CTA (per-head modes) of one GEMM launch.
 struct GemmConfig {
-  int bn, stages, kbb, target_ctas;
+  int bn, stages, kbb, target_ctas, mt = 1;
 };
 
-template <int BN, bool AMN, int STAGES, int KBB>
+template <int BN, bool AMN, int STAGES, int KBB, int MT = 1>
 mla_status launch_tc(const GemmArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
-  constexpr int smem = GemmSmem<BN, STAGES, KBB>::kBytes;
-  auto kern = gemm_tc_kernel<BN, AMN, STAGES, KBB>;
+  constexpr int smem = GemmSmem<BN, STAGES, KBB, MT>::kBytes;
+  auto kern = gemm_tc_kernel<BN, AMN, STAGES, KBB, MT>;
   static bool attr_set = false;  // idempotent attribute set; races are harmless
   if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -181,6 +184,8 @@ mla_status launch_tc(const GemmArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
 // The instantiated configurations (bn, stages, K blocks per stage).
 template <bool AMN>
 mla_status launch_tc_cfg(const GemmConfig& k, const GemmArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
+  if (k.mt == 4 && k.bn == 64 && k.stages == 2 && k.kbb == 1) return launch_tc<64, AMN, 2, 1, 4>(a, grid, st, pdl);
+  if (k.mt != 1) return MLA_ERR_UNSUPPORTED;
 #define MLA_GEMM_CFG(BN, S, KB) \
   if (k.bn == BN && k.stages == S && k.kbb == KB) return launch_tc<BN, AMN, S, KB>(a, grid, st, pdl);
   MLA_GEMM_CFG(32, 5, 1) MLA_GEMM_CFG(64, 4, 1) MLA_GEMM_CFG(128, 3, 1) MLA_GEMM_CFG(256, 4, 1)
@@ -213,7 +218,7 @@ mla_status run_gemm_tc(const Ctx& c, const GemmSpec& g, const GemmConfig& cfg) {
   a.b_head_stride = g.b_head_stride;
   a.status = c.status;
   a.tok = g.tok;
-  int m_tiles = 0;
+  int m_tiles = 0, mt_per_cta = 1;
   if (g.mode == GEMM_DENSE) {
     a.nseg = g.nseg;
     for (int s = 0; s < g.nseg; ++s) {
@@ -233,6 +238,7 @@ mla_status run_gemm_tc(const Ctx& c, const GemmSpec& g, const GemmConfig& cfg) {
     a.seg_rows[0] = g.rows[0];
     a.epi[0] = g.epi[0];
     m_tiles = tph * g.heads;
+    if (cfg.mt > 1 && tph % cfg.mt == 0) mt_per_cta = cfg.mt;
     if (g.mode == GEMM_HEAD_MNMAJOR) {
       a.boxA_rows[0] = 64;
       if (!make_map_2d(&a.mapA[0], g.A[0], g.a_ld, g.a_total_rows, g.a_ld, 64)) return MLA_ERR_CUDA;
@@ -246,7 +252,7 @@ mla_status run_gemm_tc(const Ctx& c, const GemmSpec& g, const GemmConfig& cfg) {
   const int tiles = m_tiles * n_tiles;
   const int target = std::min(cfg.target_ctas, kMaxGemmCtas);
   int splits = 1;
-  if (n_tiles == 1 && tiles < target && tiles <= kMaxCounters) {
+  if (mt_per_cta == 1 && n_tiles == 1 && tiles < target && tiles <= kMaxCounters) {
     splits = std::max(1, std::min(a.kb_total / (2 * cfg.kbb), target / tiles));
   }
   int kbps = (a.kb_total + splits - 1) / splits;
@@ -255,9 +261,11 @@ mla_status run_gemm_tc(const Ctx& c, const GemmSpec& g, const GemmConfig& cfg) {
   a.splits = splits;
   a.kb_per_split = kbps;
   a.partials = reinterpret_cast<float*>(c.ws + c.L.gpart);
-  dim3 grid(m_tiles, n_tiles, splits);
-  mla_status s = g.mode == GEMM_HEAD_MNMAJOR ? launch_tc_cfg<true>(cfg, a, grid, c.st, c.pdl)
-                                            : launch_tc_cfg<false>(cfg, a, grid, c.st, c.pdl);
+  dim3 grid(m_tiles / mt_per_cta, n_tiles, splits);
+  GemmConfig k = cfg;
+  k.mt = mt_per_cta;
+  mla_status s = g.mode == GEMM_HEAD_MNMAJOR ? launch_tc_cfg<true>(k, a, grid, c.st, c.pdl)
+                                            : launch_tc_cfg<false>(k, a, grid, c.st, c.pdl);
   if (s != MLA_OK || splits == 1) return s;
   // split-K: a wide second kernel sums the partials in split order and runs the epilogue
   const dim3 rgrid(m_tiles, bn / 4);
@@ -314,11 +322,17 @@ mla_status run_gemm_simt(const Ctx& c, const GemmSpec& g) {
 
 bool tc_gemm_ok(const mla_dims& d) {
   return d.dtype == MLA_BF16 && d.d_model % 64 == 0 && d.d_cq % 64 == 0 && d.d_c % 128 == 0 && d.d_h == 128 &&
-         (d.n_h * d.d_h) % 64 == 0 && d.d_R % 2 == 0 && d.d_R <= 128;
+         (d.n_h * d.d_h) % 64 == 0 && d.d_R % 8 == 0 && d.d_R <= 128;
 }
 
 mla_status run_gemm(const Ctx& c, const GemmSpec& g) {
-  if (tc_gemm_ok(c.d)) return run_gemm_tc(c, g, choose_gemm_config(g.N, c.num_sms));
+  if (tc_gemm_ok(c.d)) {
+    GemmConfig cfg = choose_gemm_config(g.N, c.num_sms);
+    // per-head weight blocks of several 128-row tiles (W_UK^T: d_c rows per head)
+    // share one X block: a CTA per head streams them all, one accumulator each
+    if (g.mode != GEMM_DENSE && g.N <= 64 && g.rows[0] % 512 == 0) cfg = {64, 2, 1, c.num_sms, 4};
+    return run_gemm_tc(c, g, cfg);
+  }
   return c.d.dtype == MLA_FP32 ? run_gemm_simt<float>(c, g) : run_gemm_simt<__nv_bfloat16>(c, g);
 }
 
@@ -392,6 +406,17 @@ TokenMap cache_tokens(const mla_dims& d, const mla_cache* cache) {
   t.log2_base = std::log2(d.rope_base);
   t.seq_const = -1;
   return t;
+}
+
+// Fills the call's (cos, sin) table for T tokens and points `tk` at it.
+mla_status launch_rope_table(const Ctx& c, TokenMap& tk, int T, void* table) {
+  if (tk.d_R < 2 || T <= 0) return MLA_OK;
+  const long long total = static_cast<long long>(T) * (tk.d_R / 2);
+  const int blocks = static_cast<int>(std::min<long long>(4 * c.num_sms, (total + 255) / 256));
+  const mla_status s = launch(rope_table_kernel, dim3(blocks), dim3(256), 0, c.st, c.pdl, tk, T,
+                              reinterpret_cast<float2*>(table));
+  if (s == MLA_OK) tk.rope = reinterpret_cast<const float2*>(table);
+  return s;
 }
 
 Epi epi_store(void* out, long long ld, int col0, float scale, int out_f32 = 0) {
@@ -512,6 +537,7 @@ mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const 
   if ((s = launch(plan_kernel, dim3(1), dim3(1024), 0, c.st, c.pdl, seqlen, B, tile_tokens, W, tile_start, seg_start,
                   c.status, reinterpret_cast<int*>(ws + c.L.counters), kMaxCounters)) != MLA_OK)
     return s;
+  if ((s = launch_rope_table(c, tk, B, ws + c.L.rope)) != MLA_OK) return s;
 
   // ---- a1 (+a2): down-projections from h, cache append of the new token
   {
@@ -799,6 +825,7 @@ extern "C" mla_status mla_prefill(const mla_dims* dims, const mla_weights* w, co
   tk.pos_base = start_pos;
   tk.seq_const = seq;
   if (cudaMemsetAsync(ws + c.L.counters, 0, kMaxCounters * sizeof(int), c.st) != cudaSuccess) return MLA_ERR_CUDA;
+  if ((s = launch_rope_table(c, tk, T, ws + c.L.p_rope)) != MLA_OK) return s;
   // ---- p1: down-projections and cache rows of the T new tokens
   {
     GemmSpec g;
