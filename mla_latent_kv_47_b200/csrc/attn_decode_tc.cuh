@@ -17,19 +17,21 @@
 //   CTA 1: columns c[256,512)        (4 chunks),     O columns [256,512)
 // Each CTA TMA-loads only its own columns of a tile, so the pair reads every
 // cache byte exactly once.  Each computes a partial score S_r = Q_r C_r^T
-// (tcgen05.mma, M = 128 heads, N = 64 tokens, Q_r held in TMEM) and both CTAs
+// (tcgen05.mma, M = 128 heads, N = 64 tokens, into one of two TMEM buffers;
+// the c^KV part of Q_r in TMEM, CTA 0's k^R part in shared memory) and both CTAs
 // form S = fp16(S_0) + fp16(S_1) from the same rounded halves, so their
 // softmax, P and running max are bit-identical.  O_r += P C_r (N = 256, the
 // same cache tile read as an MN-major operand) accumulates in TMEM.
 //
 // Warp roles (448 threads per CTA); each tile flows through them in order:
 //   warp 0      TMA producer (4-stage ring of tiles)
-//   warp 1      TMEM owner and MMA issuer: S as soon as a tile landed and the
-//               S buffer was read out, PV as soon as P is written
+//   warp 1      TMEM owner and MMA issuer: S(j) as soon as tile j landed and
+//               the S buffer of tile j-2 was read out, PV as soon as P is written
 //   warps 2-5   exchange: read S from TMEM, round it to fp16, push it into the
 //               partner's shared memory with st.async (its bytes complete the
 //               partner's barrier, so the sender neither fences nor waits) and
-//               park this CTA's rounded half in TMEM for the softmax.  The
+//               write this CTA's rounded half back over the S buffer for the
+//               softmax (the S buffer is freed once the softmax read it).  The
 //               partner hands a slot back the same way: a 4-byte st.async per
 //               softmax warp that completes this CTA's slot-free barrier.
 //   warps 6-13  softmax: warp 6+i and warp 10+i share lane quarter i mod 4,
@@ -38,8 +40,7 @@
 //               max is one shuffle.  Online softmax with a lazily refreshed
 //               max (O is rescaled only when a tile's max exceeds the running
 //               one by more than 2^8), P (bf16) into shared memory, and the
-//               per-piece epilogue.  P alternates between two buffers, so P(j+1)
-//               is written while PV(j) still reads P(j).
+//               per-piece epilogue.
 // The exchange warps use thread = head = TMEM lane (warp w owns lanes
 // 32 (w mod 4) ..).
 #pragma once
@@ -59,12 +60,16 @@ constexpr int kChunkBytes = 64 * 128;             // 64 token rows x 64 latent c
 constexpr int kStageBytes = 5 * kChunkBytes;      // up to 5 chunks per CTA
 constexpr int kXBytes = 128 * 128;                // one half of S: 128 heads x 64 tokens, fp16
 constexpr int kPBytes = 128 * 128;                // P: 128 heads x 64 tokens, bf16
+constexpr int kXSlots = 2;                        // exchange slots for the partner's score half
+constexpr int kPBufs = 1;                         // P buffers
+constexpr int kQRBytes = 128 * 128;               // CTA 0's k^R part of Q: 128 heads x 64, bf16 (MMA A operand)
 constexpr int kBarBytes = 512;
-// stages | partner's S half x2 | P x2 | barriers
-constexpr int kSmem = 1024 + kStages * kStageBytes + 2 * kXBytes + 2 * kPBytes + kBarBytes;
-// TMEM columns: O half [0,256), S [256,320), Q half (bf16 pairs) [320,480),
-// this CTA's fp16-rounded S half (pairs) [480,512)
-constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 320, kTmemX = 480, kTmemCols = 512;
+// stages | partner's S half x kXSlots | P x kPBufs | k^R part of Q | barriers
+constexpr int kSmem = 1024 + kStages * kStageBytes + kXSlots * kXBytes + kPBufs * kPBytes + kQRBytes + kBarBytes;
+// TMEM columns: O half [0,256), S buffers [256,320) and [320,384) (after the
+// exchange, their first 32 columns hold this CTA's fp16-rounded half), c^KV
+// part of the Q half (bf16 pairs) [384,512)
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 384, kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kRow = 576;                         // d_c + d_R
 }  // namespace attn
@@ -103,23 +108,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* stages = smem;
-  uint8_t* xpeer = stages + kStages * kStageBytes;  // [2] the partner's half of S (fp16), written by the partner
-  uint8_t* pbuf = xpeer + 2 * kXBytes;              // [2] P (bf16), MMA A operand
-  uint64_t* full = reinterpret_cast<uint64_t*>(pbuf + 2 * kPBytes);
+  uint8_t* xpeer = stages + kStages * kStageBytes;  // [kXSlots] the partner's half of S (fp16), written by the partner
+  uint8_t* pbuf = xpeer + kXSlots * kXBytes;        // [kPBufs] P (bf16), MMA A operand
+  uint8_t* qr = pbuf + kPBufs * kPBytes;            // CTA 0: k^R part of Q (bf16), MMA A operand
+  uint64_t* full = reinterpret_cast<uint64_t*>(qr + kQRBytes);
   uint64_t* empty = full + kStages;
-  uint64_t* s_full = empty + kStages;
-  uint64_t* s_free = s_full + 1;
-  uint64_t* xo_full = s_free + 1;    // own rounded half parked in TMEM (exchange -> softmax)
-  uint64_t* xo_free = xo_full + 1;   // own half read out (softmax -> exchange)
-  uint64_t* x_full = xo_free + 1;    // [2] partner's half landed (st.async bytes)
-  uint64_t* x_free = x_full + 2;     // [2] partner's half consumed (arrivals from the partner's softmax)
-  uint64_t* p_full = x_free + 2;     // [2]
-  uint64_t* p_free = p_full + 2;     // [2]
-  uint64_t* q_full = p_free + 2;
+  uint64_t* s_full = empty + kStages;  // [2] S(j) in buffer j & 1 (MMA -> exchange)
+  uint64_t* s_free = s_full + 2;       // [2] buffer read out by the softmax (softmax -> MMA)
+  uint64_t* xo_full = s_free + 2;      // [2] own rounded half written back (exchange -> softmax)
+  uint64_t* x_full = xo_full + 2;    // [kXSlots] partner's half landed (st.async bytes)
+  uint64_t* x_free = x_full + kXSlots;  // [kXSlots] partner's half consumed (signals from the partner's softmax)
+  uint64_t* p_full = x_free + kXSlots;  // [kPBufs]
+  uint64_t* p_free = p_full + kPBufs;   // [kPBufs]
+  uint64_t* q_full = p_free + kPBufs;
   uint64_t* o_done = q_full + 1;
   uint64_t* drain = o_done + 1;
-  uint32_t* sig = reinterpret_cast<uint32_t*>(drain + 1);  // [2 slots][8] landing words of the partner's slot-free signals
-  uint32_t* tmem_slot = sig + 16;
+  uint32_t* sig = reinterpret_cast<uint32_t*>(drain + 1);  // [kXSlots][8] landing words of the partner's slot-free signals
+  uint32_t* tmem_slot = sig + 8 * kXSlots;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t rank = cluster_ctarank();
@@ -133,15 +138,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
-    mbar_init(xo_full, 4);      // one arrival per exchange warp
-    mbar_init(xo_free, 8);      // one arrival per softmax warp
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 8);   // one arrival per softmax warp
+      mbar_init(&xo_full[i], 4);  // one arrival per exchange warp
+    }
+    for (int i = 0; i < kXSlots; ++i) {
       mbar_init(&x_full[i], 1);   // armed once per phase with the expected bytes
       mbar_init(&x_free[i], 1);   // armed by the exchange before each use; 8 x 4 signal bytes from the partner
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kPBufs; ++i) {
       mbar_init(&p_full[i], 8);   // one arrival per softmax warp
       mbar_init(&p_free[i], 1);
     }
@@ -150,9 +156,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    // phase 0 of both exchange slots expects the partner's 16 KB
-    mbar_arrive_expect_tx(&x_full[0], kXBytes);
-    mbar_arrive_expect_tx(&x_full[1], kXBytes);
+    // phase 0 of every exchange slot expects the partner's 16 KB
+    for (int i = 0; i < kXSlots; ++i) mbar_arrive_expect_tx(&x_full[i], kXBytes);
   }
   if (warp == 0 && lane == 0) prefetch_tmap(&a.map_cache);
   if (warp == 1) {
@@ -206,8 +211,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           if (npv < ns) {
             const int g = it + npv;
             const int s = g % kStages;
-            const int b = g & 1;
-            if (mbar_test_wait(smem_u32(&p_full[b]), (g >> 1) & 1)) {
+            const int b = g % kPBufs;
+            if (mbar_test_wait(smem_u32(&p_full[b]), (g / kPBufs) & 1)) {
               tc_fence_after();
               const uint32_t st = smem_u32(stages + s * kStageBytes);
               const uint32_t pb = smem_u32(pbuf + b * kPBytes);
@@ -226,17 +231,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           if (!issued && ns < nt) {
             const int g = it + ns;
             const int s = g % kStages;
-            if (mbar_test_wait(smem_u32(&full[s]), (g / kStages) & 1) && mbar_test_wait(smem_u32(s_free), (g & 1) ^ 1)) {
+            const int sb = g & 1;
+            if (mbar_test_wait(smem_u32(&full[s]), (g / kStages) & 1) &&
+                mbar_test_wait(smem_u32(&s_free[sb]), ((g >> 1) & 1) ^ 1)) {
               tc_fence_after();
               const uint32_t st = smem_u32(stages + s * kStageBytes);
-              for (int ci = 0; ci < nchunks; ++ci) {
+              const uint32_t dS = tmem + kTmemS + sb * 64;
+              for (int ci = 0; ci < 4; ++ci) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                  mma_ts(tmem + kTmemS, tmem + kTmemQ + ci * 32 + kk * 8,
-                         sdesc_sw128(st + ci * kChunkBytes + kk * 32, 16, 1024), idesc_s, (ci | kk) ? 1u : 0u);
+                  mma_ts(dS, tmem + kTmemQ + ci * 32 + kk * 8, sdesc_sw128(st + ci * kChunkBytes + kk * 32, 16, 1024),
+                         idesc_s, (ci | kk) ? 1u : 0u);
                 }
               }
-              mma_commit(s_full);
+              if (nchunks == 5) {  // CTA 0: the k^R chunk, Q_R from shared memory
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  mma_ss(dS, sdesc_sw128(smem_u32(qr) + kk * 32, 16, 1024),
+                         sdesc_sw128(st + 4 * kChunkBytes + kk * 32, 16, 1024), idesc_s, 1u);
+                }
+              }
+              mma_commit(&s_full[sb]);
               ++ns;
               issued = true;
             }
@@ -269,6 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     const int sw = h & 7;
     const uint32_t peer_row = mapa(smem_u32(xpeer), peer) + h * 128;
     const uint32_t xfull_peer = mapa(smem_u32(x_full), peer);
+    const uint32_t qr_row = smem_u32(qr) + h * 128;
     const bool arm = warp == 2 && lane == 0;
     int it = 0;
     for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
@@ -277,7 +293,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       // previous piece's last S has been read out, so no MMA still reads Q.
       const bool head = h < a.n_h;
       const __nv_bfloat16* qrow = a.qlat + (static_cast<long long>(p.b) * a.n_h + (head ? h : 0)) * kRow;
-      for (int ci = 0; ci < nchunks; ++ci) {
+      for (int ci = 0; ci < 4; ++ci) {
         const uint4* src = reinterpret_cast<const uint4*>(qrow + attn_chunk_col(rank, ci));
         uint32_t r[32];
 #pragma unroll
@@ -287,6 +303,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         }
         tmem_st32(tl + kTmemQ + ci * 32, r);
       }
+      if (nchunks == 5) {  // CTA 0: the k^R part of Q into shared memory, 128-byte swizzled rows
+        const uint4* src = reinterpret_cast<const uint4*>(qrow + attn_chunk_col(rank, 4));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) st_shared_v4(qr_row + ((i ^ sw) << 4), head ? src[i] : make_uint4(0, 0, 0, 0));
+        fence_proxy_async_smem();
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(q_full);
@@ -294,48 +316,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       const int nt = p.t1 - p.t0;
       for (int k = 0; k < nt; ++k) {
         const int g = it + k;
-        const int slot = g & 1;
-        const uint32_t ph = (g >> 1) & 1;
-        if (!mbar_wait(s_full, g & 1, wc)) return;
+        const int slot = g % kXSlots;
+        const uint32_t ph = (g / kXSlots) & 1;
+        const int sb = g & 1;
+        if (!mbar_wait(&s_full[sb], (g >> 1) & 1, wc)) return;
         tc_fence_after();
         uint32_t hx[32];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t sr[32];
-          tmem_ld32(tl + kTmemS + half * 32, sr);
+          tmem_ld32(tl + kTmemS + sb * 64 + half * 32, sr);
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             hx[half * 16 + j] = pack_half2(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1]));
         }
-        tc_fence_before();
-        mbar_arrive(s_free);
         // partner first: its copy has the longer way to go
         if (!mbar_wait<true>(&x_free[slot], ph ^ 1, wc)) return;
         // the partner returns this use of the slot with 8 signals of 4 bytes;
         // armed before this warp's data goes out, so no signal can precede it
         if (arm) mbar_arrive_expect_tx(&x_free[slot], 32);
         const uint32_t dst = peer_row + slot * kXBytes;
-        const uint32_t bar = xfull_peer + slot * 8;
+        const uint32_t bar = xfull_peer + slot * 8;  // x_full[slot] in the partner
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           st_async_v4(dst + ((i ^ sw) << 4), make_uint4(hx[4 * i], hx[4 * i + 1], hx[4 * i + 2], hx[4 * i + 3]), bar);
-        // own half into TMEM once the softmax has read the previous one
-        if (!mbar_wait(xo_free, (g & 1) ^ 1, wc)) return;
-        tc_fence_after();
-        tmem_st32(tl + kTmemX, hx);
+        // own rounded half over the first 32 columns of the S buffer
+        tmem_st32(tl + kTmemS + sb * 64, hx);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(xo_full);
+        if (lane == 0) mbar_arrive(&xo_full[sb]);
       }
       it += nt;
     });
     // The partner's signals for the last use of each slot land in this CTA's
     // shared memory: they must have arrived before the CTA may exit.
     if (arm && !*abort_flag) {
-      for (int s2 = 0; s2 < 2; ++s2) {
-        const int uses = (it + 1 - s2) / 2;
+      for (int s2 = 0; s2 < kXSlots; ++s2) {
+        const int uses = (it + kXSlots - 1 - s2) / kXSlots;  // tiles g < it with g % kXSlots == s2
         if (uses > 0 && !mbar_wait<true>(&x_free[s2], (uses - 1) & 1, wc)) break;
       }
     }
@@ -362,14 +381,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       for (int k = 0; k < nt; ++k) {
         const int g = it + k;
         const int t = p.t0 + k;
-        const int slot = g & 1;
-        const uint32_t ph = (g >> 1) & 1;
-        if (!mbar_wait(xo_full, g & 1, wc)) return;
+        const int slot = g % kXSlots;
+        const uint32_t ph = (g / kXSlots) & 1;
+        const int sb = g & 1;
+        if (!mbar_wait(&xo_full[sb], (g >> 1) & 1, wc)) return;
         if (!mbar_wait<true>(&x_full[slot], ph, wc)) return;
         tc_fence_after();
         // ---- full scores of this thread's 32 tokens (same bits in both CTAs)
         uint32_t own[16];
-        tmem_ld16x2(tl + kTmemX, own);
+        tmem_ld16x2(tl + kTmemS + sb * 64, own);
         uint4 pv[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) pv[i] = ld_shared_v4(peer_row + slot * kXBytes + (((th * 4 + i) ^ sw) << 4));
@@ -377,7 +397,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(xo_free);
+          mbar_arrive(&s_free[sb]);  // S buffer sb may take S(g + 2)
           // the slot's next phase expects the partner's next 16 KB; armed
           // before the slot is released, so no byte can land ahead of it
           if (leader) mbar_arrive_expect_tx(&x_full[slot], kXBytes);
@@ -396,7 +416,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         }
         // every value read from the partner's half is consumed: hand the slot back
         __syncwarp();
-        if (lane == 0) st_async_b32(sig_peer + slot * 32, 0u, xfree_peer + slot * 8);
+        if (lane == 0) st_async_b32(sig_peer + slot * 32, 0u, xfree_peer + slot * 8);  // into sig[slot][warp - 6]
         if (__any_sync(0xffffffffu, valid < 32)) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
@@ -427,12 +447,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         l_run = l_run * alpha + lsum;
         m_run = m_new;
         // ---- P buffer b is free once PV(g-2) retired
-        const int b = g & 1;
-        if (!mbar_wait(&p_free[b], ph ^ 1, wc)) return;
+        const int b = g % kPBufs;
+        if (!mbar_wait(&p_free[b], ((g / kPBufs) & 1) ^ 1, wc)) return;
         tc_fence_after();
         if (__any_sync(0xffffffffu, rescale)) {
           // O must hold PV(g-1) before it is scaled (k >= 1 here, so g >= 1)
-          if (!mbar_wait(&p_free[b ^ 1], ((g - 1) >> 1) & 1, wc)) return;
+          if (kPBufs > 1 && !mbar_wait(&p_free[(g - 1) % kPBufs], ((g - 1) / kPBufs) & 1, wc)) return;
           tc_fence_after();
           for (int c = 0; c < 256; c += 32) {
             uint32_t o[16];
