@@ -522,6 +522,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     }
     __syncwarp();
   }
+  __syncwarp();  // every warp reconverged (elected producer / issuer lanes) before the aligned barriers
   __syncthreads();
   cluster_sync();
   if (warp == 1) {

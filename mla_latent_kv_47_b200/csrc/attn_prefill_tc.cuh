@@ -262,6 +262,7 @@ __global__ void __launch_bounds__(192, 1) attn_prefill_tc_kernel(const __grid_co
     }
     __syncwarp();
   }
+  __syncwarp();  // every warp reconverged (elected lanes) before the aligned barrier
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();

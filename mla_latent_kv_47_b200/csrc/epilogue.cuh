@@ -161,62 +161,34 @@ __device__ __forceinline__ void epi_apply(const Epi& e, const TokenMap& tk, int 
 }
 
 // ---- staged epilogue of the tensor-core GEMM.
-// Phase 1 (thread = output row m of the tile): each output's final value
-// (scale, RoPE) goes into a staging tile in shared memory, column-major
-// ([n][128 rows]), so consecutive rows of one token sit side by side.
-// Phase 2 (all epilogue threads): runs of 16 bytes (8 bf16 or 4 fp32 rows of
-// one token) are copied to their destination with one vector store each.
-// Every kind maps a run of 8 consecutive rows to 8 consecutive destination
-// elements (head blocks are multiples of 8 rows), so one address per run.
+// Phase 1 (thread = output row m of the tile): each output goes into a staging
+// tile in shared memory, column-major ([n][128 rows]), so consecutive rows of
+// one token sit side by side: the final value (scaled, in the output type) for
+// plain kinds, the raw fp32 value for the rotary kinds.
+// Phase 2 (all epilogue threads): runs of 8 rows of one token (16 bytes of
+// bf16 or 32 of fp32) go to their destination with vector stores; a rotary run
+// is 4 interleaved pairs, rotated here with one 32-byte load of their (cos, sin)
+// from the call's table.  Every kind maps a run of 8 consecutive rows to 8
+// consecutive destination elements (head blocks are multiples of 8 rows).
 
-template <int KIND>
-__device__ __forceinline__ float epi_value(const Epi& e, const TokenMap& tk, int m, int n, float y, float yp,
-                                           double inv_freq) {
-  if (KIND == EPI_QLAT_ROPE || KIND == EPI_QP_ROPE) {
-    const int j = m % tk.d_R;
-    float c, s;
-    rope_cs(tk, n, j >> 1, inv_freq, c, s);
-    return rope_apply(j, y, yp, c, s) * e.scale;
-  } else if (KIND == EPI_CACHE_KR) {
-    float c, s;
-    rope_cs(tk, n, m >> 1, inv_freq, c, s);
-    return rope_apply(m, y, yp, c, s);
-  } else if (KIND == EPI_CACHE_CKV) {
-    return y;
-  } else {
-    return y * e.scale;
-  }
+__device__ __forceinline__ bool epi_rotary(int kind) {
+  return kind == EPI_QLAT_ROPE || kind == EPI_CACHE_KR || kind == EPI_QP_ROPE;
 }
 
-// Phase 1 for NV consecutive columns n0.. held by this thread (whole warps
-// call it: the rotary partner row is a lane shuffle away).  Columns at or
-// past n_end are staged as zero and never stored.
-template <int KIND, int NV>
-__device__ __forceinline__ void epi_stage_kind(const Epi& e, const TokenMap& tk, int m, int n0, int n_end,
-                                               const float* v, double inv_freq, uint8_t* stage, int nl0, int ml) {
-#pragma unroll
-  for (int j = 0; j < NV; ++j) {
-    constexpr bool rot = (KIND == EPI_QLAT_ROPE || KIND == EPI_CACHE_KR || KIND == EPI_QP_ROPE);
-    const float yp = rot ? __shfl_xor_sync(0xffffffffu, v[j], 1) : 0.f;
-    const float r = (n0 + j < n_end) ? epi_value<KIND>(e, tk, m, n0 + j, v[j], yp, inv_freq) : 0.f;
-    const int idx = (nl0 + j) * 128 + ml;
-    if (e.out_f32) {
-      reinterpret_cast<float*>(stage)[idx] = r;
-    } else {
-      reinterpret_cast<__nv_bfloat16*>(stage)[idx] = __float2bfloat16_rn(r);
-    }
-  }
-}
-
+// Phase 1 for NV consecutive columns n0.. held by this thread.
 template <int NV>
-__device__ __forceinline__ void epi_stage(const Epi& e, const TokenMap& tk, int m, int n0, int n_end, const float* v,
-                                          double inv_freq, uint8_t* stage, int nl0, int ml) {
-  switch (e.kind) {
-    case EPI_QLAT_ROPE: epi_stage_kind<EPI_QLAT_ROPE, NV>(e, tk, m, n0, n_end, v, inv_freq, stage, nl0, ml); break;
-    case EPI_QP_ROPE: epi_stage_kind<EPI_QP_ROPE, NV>(e, tk, m, n0, n_end, v, inv_freq, stage, nl0, ml); break;
-    case EPI_CACHE_KR: epi_stage_kind<EPI_CACHE_KR, NV>(e, tk, m, n0, n_end, v, inv_freq, stage, nl0, ml); break;
-    case EPI_CACHE_CKV: epi_stage_kind<EPI_CACHE_CKV, NV>(e, tk, m, n0, n_end, v, inv_freq, stage, nl0, ml); break;
-    default: epi_stage_kind<EPI_STORE, NV>(e, tk, m, n0, n_end, v, inv_freq, stage, nl0, ml); break;
+__device__ __forceinline__ void epi_stage(const Epi& e, int n0, int n_end, const float* v, uint8_t* stage, int nl0, int ml) {
+  if (epi_rotary(e.kind) || e.out_f32) {
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const float r = epi_rotary(e.kind) ? v[j] : v[j] * e.scale;
+      reinterpret_cast<float*>(stage)[(nl0 + j) * 128 + ml] = (n0 + j < n_end) ? r : 0.f;
+    }
+  } else {
+    const float sc = e.kind == EPI_CACHE_CKV ? 1.f : e.scale;
+#pragma unroll
+    for (int j = 0; j < NV; ++j)
+      reinterpret_cast<__nv_bfloat16*>(stage)[(nl0 + j) * 128 + ml] = __float2bfloat16_rn((n0 + j < n_end) ? v[j] * sc : 0.f);
   }
 }
 
@@ -241,19 +213,62 @@ __device__ __forceinline__ uint8_t* epi_addr(const Epi& e, const TokenMap& tk, i
   return static_cast<uint8_t*>(e.out) + idx * es;
 }
 
+// Rotated, scaled run of 8 rows (4 interleaved pairs starting at pair i0) of
+// token n from the fp32 staging tile.
+__device__ __forceinline__ void epi_rope_run(const Epi& e, const TokenMap& tk, int n, int i0, const float* x, float* y) {
+  float c[4], s[4];
+  if (tk.rope) {
+    const float4* t = reinterpret_cast<const float4*>(tk.rope + static_cast<long long>(n) * (tk.d_R >> 1) + i0);
+    const float4 a = t[0], b = t[1];
+    c[0] = a.x; s[0] = a.y; c[1] = a.z; s[1] = a.w; c[2] = b.x; s[2] = b.y; c[3] = b.z; s[3] = b.w;
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) rope_cos_sin(tok_pos(tk, n), rope_inv_freq(i0 + q, tk.d_R, tk.log2_base), c[q], s[q]);
+  }
+  const float sc = e.kind == EPI_CACHE_KR ? 1.f : e.scale;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    y[2 * q] = (x[2 * q] * c[q] - x[2 * q + 1] * s[q]) * sc;
+    y[2 * q + 1] = (x[2 * q] * s[q] + x[2 * q + 1] * c[q]) * sc;
+  }
+}
+
 // Phase 2: the staged tile (tokens n_base .. n_base + n_cols - 1, rows m0 ..
-// m0 + 127) to global memory, 16 bytes per store; thread tid of nthr.
+// m0 + 127) to global memory; thread tid of nthr.
 __device__ __forceinline__ void epi_flush(const Epi& e, const TokenMap& tk, int m0, int rows_valid, int n_base, int n_cols,
                                           int n_end, int head, const uint8_t* stage, int tid, int nthr, int* status) {
-  const int vec = e.out_f32 ? 4 : 8;  // rows per 16-byte run
+  const bool rot = epi_rotary(e.kind);
+  const bool f32 = rot || e.out_f32;  // staging type
+  const int vec = (!rot && e.out_f32) ? 4 : 8;  // rows per run
   const int runs = 128 / vec;
-  const int es = e.out_f32 ? 4 : 2;
   for (int id = tid; id < n_cols * runs; id += nthr) {
     const int nl = id / runs, ml = (id % runs) * vec;
     const int n = n_base + nl, m = m0 + ml;
     if (n >= n_end || m >= rows_valid) continue;
     uint8_t* dst = epi_addr(e, tk, m, n, head, status);
-    if (dst) *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(stage + (nl * 128 + ml) * es);
+    if (!dst) continue;
+    if (rot) {
+      const float4* src = reinterpret_cast<const float4*>(stage + (nl * 128 + ml) * 4);
+      const float4 a = src[0], b = src[1];
+      const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      float y[8];
+      const int i0 = (e.kind == EPI_CACHE_KR ? m : m % tk.d_R) >> 1;
+      epi_rope_run(e, tk, n, i0, x, y);
+      if (e.out_f32) {
+        reinterpret_cast<float4*>(dst)[0] = make_float4(y[0], y[1], y[2], y[3]);
+        reinterpret_cast<float4*>(dst)[1] = make_float4(y[4], y[5], y[6], y[7]);
+      } else {
+        uint4 o;
+        __nv_bfloat162 t;
+        t = __floats2bfloat162_rn(y[0], y[1]); o.x = *reinterpret_cast<uint32_t*>(&t);
+        t = __floats2bfloat162_rn(y[2], y[3]); o.y = *reinterpret_cast<uint32_t*>(&t);
+        t = __floats2bfloat162_rn(y[4], y[5]); o.z = *reinterpret_cast<uint32_t*>(&t);
+        t = __floats2bfloat162_rn(y[6], y[7]); o.w = *reinterpret_cast<uint32_t*>(&t);
+        *reinterpret_cast<uint4*>(dst) = o;
+      }
+    } else {
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(stage + (nl * 128 + ml) * (f32 ? 4 : 2));
+    }
   }
 }
 

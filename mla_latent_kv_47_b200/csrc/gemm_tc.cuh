@@ -226,14 +226,12 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         uint8_t* stage = sA;
 #pragma unroll 1
         for (int t = 0; t < MT; ++t) {
-          const int mr = m + t * 128;
-          const double inv_freq = epi_inv_freq(e, args.tok, mr);
 #pragma unroll 1
           for (int c = 0; c < BN; c += 16) {
             float v[16];
             tmem_ld16(trow + t * BN + c, v);
             tmem_wait_ld();
-            epi_stage<16>(e, args.tok, mr, nt * BN + c, args.N, v, inv_freq, stage, c, row);
+            epi_stage<16>(e, nt * BN + c, args.N, v, stage, c, row);
           }
           named_bar_sync(1, 128);
           epi_flush(e, args.tok, m0 + t * 128, args.seg_rows[seg], nt * BN, BN, args.N, head, stage, threadIdx.x - 64, 128,
@@ -243,6 +241,11 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       }
     }
   }
+  // The producer and MMA warps arrive here with their elected lane last: the
+  // warp must be reconverged before the CTA barrier (bar.sync is warp-aligned;
+  // a warp that arrives split can release the barrier before the epilogue
+  // warps arrive, and TMEM would be freed under their loads).
+  __syncwarp();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -282,9 +285,8 @@ __global__ void __launch_bounds__(128) gemm_splitk_epilogue_kernel(const __grid_
   }
   __shared__ __align__(16) uint8_t stage[4 * 128 * 4];
   const Epi& e = args.epi[seg];
-  const int m = m0 + row;
   const float v[4] = {acc.x, acc.y, acc.z, acc.w};
-  epi_stage<4>(e, args.tok, m, cg * 4, args.N, v, epi_inv_freq(e, args.tok, m), stage, 0, row);
+  epi_stage<4>(e, cg * 4, args.N, v, stage, 0, row);
   __syncthreads();
   epi_flush(e, args.tok, m0, args.seg_rows[seg], cg * 4, 4, args.N, head, stage, threadIdx.x, 128, args.status);
 }

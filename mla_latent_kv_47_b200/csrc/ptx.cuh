@@ -371,7 +371,10 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
                : "memory");
   return v;
 }
+// bar.sync is warp-aligned: every lane of each participating warp must reach
+// it together, so the warp is reconverged first.
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  __syncwarp();
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 __device__ __forceinline__ float ld_cg_f32(const float* p) { return __ldcg(p); }
