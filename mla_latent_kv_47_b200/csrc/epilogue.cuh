@@ -234,10 +234,34 @@ __device__ __forceinline__ void epi_rope_run(const Epi& e, const TokenMap& tk, i
 }
 
 // Phase 2: the staged tile (tokens n_base .. n_base + n_cols - 1, rows m0 ..
-// m0 + 127) to global memory; thread tid of nthr.
+// m0 + 127) to global memory; thread tid of nthr.  Plain kinds take a direct
+// path (destination of a token computed once, loop unrolled so the
+// shared-memory loads and global stores overlap); cache and rotary kinds take
+// the general one.
 __device__ __forceinline__ void epi_flush(const Epi& e, const TokenMap& tk, int m0, int rows_valid, int n_base, int n_cols,
                                           int n_end, int head, const uint8_t* stage, int tid, int nthr, int* status) {
-  const bool rot = epi_rotary(e.kind);
+  const int kind = e.kind;
+  const bool rot = epi_rotary(kind);
+  if (!rot && kind != EPI_CACHE_CKV) {
+    // runs of 16 bytes: 8 bf16 or 4 fp32 rows; log2 of runs per token
+    const int lg = e.out_f32 ? 5 : 4;
+    const int es = e.out_f32 ? 4 : 2;
+    uint8_t* const out = static_cast<uint8_t*>(e.out);
+    const long long ld = e.ld;
+    const long long off0 = kind == EPI_PER_HEAD ? static_cast<long long>(head) * e.hs : e.col0;
+    const int total = n_cols << lg;
+#pragma unroll 4
+    for (int id = tid; id < total; id += nthr) {
+      const int nl = id >> lg, ml = (id & ((1 << lg) - 1)) * (16 / es);
+      const int n = n_base + nl, m = m0 + ml;
+      if (n >= n_end || m >= rows_valid) continue;
+      long long idx;
+      if (kind == EPI_HEADS) idx = static_cast<long long>(n) * ld + (m / e.dh) * e.hs + e.col0 + m % e.dh;
+      else idx = static_cast<long long>(n) * ld + off0 + m;
+      *reinterpret_cast<uint4*>(out + idx * es) = *reinterpret_cast<const uint4*>(stage + (nl * 128 + ml) * es);
+    }
+    return;
+  }
   const bool f32 = rot || e.out_f32;  // staging type
   const int vec = (!rot && e.out_f32) ? 4 : 8;  // rows per run
   const int runs = 128 / vec;
@@ -252,7 +276,7 @@ __device__ __forceinline__ void epi_flush(const Epi& e, const TokenMap& tk, int 
       const float4 a = src[0], b = src[1];
       const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
       float y[8];
-      const int i0 = (e.kind == EPI_CACHE_KR ? m : m % tk.d_R) >> 1;
+      const int i0 = (kind == EPI_CACHE_KR ? m : m % tk.d_R) >> 1;
       epi_rope_run(e, tk, n, i0, x, y);
       if (e.out_f32) {
         reinterpret_cast<float4*>(dst)[0] = make_float4(y[0], y[1], y[2], y[3]);
