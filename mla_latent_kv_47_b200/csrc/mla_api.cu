@@ -630,7 +630,7 @@ mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const 
   }
   attn_event(g_attn_end, c.st);
   {
-    dim3 grid(B, d.n_h);
+    dim3 grid(B, (d.n_h + 3) / 4);  // one warp per (sequence, head)
     if (d.dtype == MLA_FP32)
       s = launch(combine_kernel<float>, grid, dim3(128), 0, c.st, c.pdl, opart, ml, seg_start, d.n_h, d.d_c,
                  static_cast<float*>(olat));

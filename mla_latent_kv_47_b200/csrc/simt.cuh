@@ -238,11 +238,26 @@ __global__ void __launch_bounds__(128) simt_decode_attn_kernel(
 // O_lat[b][h][c] = sum_s 2^(m_s - M) O_s[c] / sum_s 2^(m_s - M) l_s over the
 // pieces s of sequence b (the log-sum-exp merge of softmax partials).
 template <typename T>
+__device__ __forceinline__ void store4(T* dst, float4 v);
+template <>
+__device__ __forceinline__ void store4<float>(float* dst, float4 v) {
+  *reinterpret_cast<float4*>(dst) = v;
+}
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* dst, float4 v) {
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+  *reinterpret_cast<uint2*>(dst) = make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+}
+
+// One warp per (sequence, head): lane l owns columns 4l + 128k.  The pieces
+// are merged in order, weights 2^(m_s - M), then normalised by the merged l.
+template <typename T>
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ o_part, const float* __restrict__ ml_part,
                                                      const int* seg_start, int n_h, int d_c, T* __restrict__ olat) {
   griddep_wait();
   if (threadIdx.x == 0) griddep_launch_dependents();
-  const int b = blockIdx.x, h = blockIdx.y;
+  const int b = blockIdx.x, h = blockIdx.y * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (h >= n_h) return;
   const int s0 = seg_start[b], s1 = seg_start[b + 1];
   float M = -INFINITY;
   for (int s = s0; s < s1; ++s) M = fmaxf(M, ml_part[(static_cast<long long>(s) * n_h + h) * 2]);
@@ -252,18 +267,15 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
     Ls += exp2f(ml_part[i] - M) * ml_part[i + 1];
   }
   const float inv = 1.f / Ls;
-  for (int c = threadIdx.x * 4; c < d_c; c += 128 * 4) {
+  for (int c = lane * 4; c < d_c; c += 128) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s = s0; s < s1; ++s) {
       const float wgt = exp2f(ml_part[(static_cast<long long>(s) * n_h + h) * 2] - M);
       const float4 v = *reinterpret_cast<const float4*>(o_part + (static_cast<long long>(s) * n_h + h) * d_c + c);
       acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
     }
-    T* dst = olat + (static_cast<long long>(b) * n_h + h) * d_c + c;
-    dst[0] = static_cast<T>(acc.x * inv);
-    dst[1] = static_cast<T>(acc.y * inv);
-    dst[2] = static_cast<T>(acc.z * inv);
-    dst[3] = static_cast<T>(acc.w * inv);
+    store4<T>(olat + (static_cast<long long>(b) * n_h + h) * d_c + c,
+              make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv));
   }
 }
 
