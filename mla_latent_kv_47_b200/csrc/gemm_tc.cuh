@@ -205,7 +205,6 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     named_bar_sync(1, 128);            // every epilogue thread sees the same abort decision
     if (!*abort_flag) {
       const Epi& e = args.epi[seg];
-      const int m = m0 + row;
       const int tile_id = mt + gridDim.x * nt;
       if (args.splits > 1) {
         // split-K: store this split's partial tile ([BN/4 column groups][128 rows][4],

@@ -19,7 +19,6 @@ using namespace mla;
 namespace {
 
 constexpr int kMaxWorkers = 296;        // attention workers (partial slots beyond B)
-constexpr int kMaxCounters = 4096;      // split-K tickets
 constexpr int kMaxGemmCtas = 296;       // split-K target: two CTAs per SM on 148 SMs
 constexpr size_t kAlign = 256;
 
@@ -29,7 +28,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // the decode region (sized by the batch) or the prefill region (sized by the
 // number of key tokens); a call uses only its own region.
 struct Layout {
-  size_t status, counters, gpart, base_end;
+  size_t status, gpart, base_end;
   size_t tile_start, seg_start, rope, cq, qc, qlat, olat, o, opart, ml, decode_end;
   size_t p_rope, p_cq, p_qp, p_rows, p_kc, p_v, p_out, prefill_end;
 };
@@ -50,7 +49,6 @@ Layout make_layout_sized(const mla_dims& d, int max_batch, int max_tokens, int g
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, kAlign); return o; };
   L.status = take(256);
-  L.counters = take(kMaxCounters * sizeof(int));
   L.gpart = take(static_cast<size_t>(kMaxGemmCtas) * gpart_bn * 128 * sizeof(float));
   L.base_end = off;
   L.tile_start = take((B + 1) * sizeof(int));
@@ -252,7 +250,11 @@ mla_status run_gemm_tc(const Ctx& c, const GemmSpec& g, const GemmConfig& cfg) {
   const int tiles = m_tiles * n_tiles;
   const int target = std::min(cfg.target_ctas, kMaxGemmCtas);
   int splits = 1;
-  if (mt_per_cta == 1 && n_tiles == 1 && tiles < target && tiles <= kMaxCounters) {
+  // per-head GEMMs (W_UV at n_h = 128) that already cover half the SMs run
+  // without split-K: the partial round trip and second kernel cost more than
+  // the extra parallelism gains
+  const bool split_ok = g.mode == GEMM_DENSE || 2 * tiles <= c.num_sms;
+  if (split_ok && mt_per_cta == 1 && n_tiles == 1 && tiles < target) {
     splits = std::max(1, std::min(a.kb_total / (2 * cfg.kbb), target / tiles));
   }
   int kbps = (a.kb_total + splits - 1) / splits;
@@ -529,15 +531,16 @@ mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const 
   tk.pos = seqlen;  // the new token of sequence b sits at position L_b
   (void)es;
 
-  // ---- attention plan (device side: reads seqlen, no host sync); also zeroes the split-K tickets
+  // ---- attention plan (device side: reads seqlen, no host sync) and the RoPE table of the new tokens
   const bool tc_attn = attn_tc_ok(d);
   const int tile_tokens = tc_attn ? kAttnTileTokens : 64;
   const int W = decode_workers(d, c.num_sms);
   c.pdl = tc_gemm_ok(d);
+  float2* rope = d.d_R >= 2 ? reinterpret_cast<float2*>(ws + c.L.rope) : nullptr;
   if ((s = launch(plan_kernel, dim3(1), dim3(1024), 0, c.st, c.pdl, seqlen, B, tile_tokens, W, tile_start, seg_start,
-                  c.status, reinterpret_cast<int*>(ws + c.L.counters), kMaxCounters)) != MLA_OK)
+                  c.status, tk, rope)) != MLA_OK)
     return s;
-  if ((s = launch_rope_table(c, tk, B, ws + c.L.rope)) != MLA_OK) return s;
+  tk.rope = rope;
 
   // ---- a1 (+a2): down-projections from h, cache append of the new token
   {
@@ -764,7 +767,6 @@ mla_status mla_cache_append(const mla_dims* dims, const mla_weights* w, const vo
   g.tok.pos = pos;
   g.tok.seq = seq_idx;
   add_cache_segments(g, d, w);
-  if (cudaMemsetAsync(c.ws + c.L.counters, 0, kMaxCounters * sizeof(int), c.st) != cudaSuccess) return MLA_ERR_CUDA;
   return run_gemm(c, g);
 }
 
@@ -824,7 +826,6 @@ extern "C" mla_status mla_prefill(const mla_dims* dims, const mla_weights* w, co
   TokenMap tk = cache_tokens(d, cache);
   tk.pos_base = start_pos;
   tk.seq_const = seq;
-  if (cudaMemsetAsync(ws + c.L.counters, 0, kMaxCounters * sizeof(int), c.st) != cudaSuccess) return MLA_ERR_CUDA;
   if ((s = launch_rope_table(c, tk, T, ws + c.L.p_rope)) != MLA_OK) return s;
   // ---- p1: down-projections and cache rows of the T new tokens
   {

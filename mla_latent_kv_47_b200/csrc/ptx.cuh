@@ -199,18 +199,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-      "r"(__float_as_uint(v[15]))
-      : "memory");
-}
 
 // Shared-memory matrix descriptor, 128-byte swizzle (sm100 format: version 1
 // at bit 46, layout type 2 at bits 61-63).  Addresses and offsets in bytes.
@@ -256,11 +244,6 @@ __device__ __forceinline__ void cluster_sync() {
   cluster_arrive_release();
   cluster_wait_acquire();
 }
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint4 v) {
-  asm volatile("st.shared::cluster.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
-               "r"(v.w)
-               : "memory");
-}
 // 16-byte store into another CTA's shared memory that completes 16 transaction
 // bytes on that CTA's mbarrier (both addresses from mapa).  Nothing on the
 // sending side waits for it; the receiver's barrier phase completes once all
@@ -275,9 +258,6 @@ __device__ __forceinline__ void st_async_b32(uint32_t cluster_addr, uint32_t v, 
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(cluster_addr), "r"(v),
                "r"(cluster_bar)
                : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // D(tmem) (+)= A(tmem) * B(smem desc)^T: A is read from tensor memory (128 lanes
@@ -377,6 +357,5 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   __syncwarp();
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
-__device__ __forceinline__ float ld_cg_f32(const float* p) { return __ldcg(p); }
 
 }  // namespace mla

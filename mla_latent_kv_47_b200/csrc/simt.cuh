@@ -67,14 +67,23 @@ __host__ __device__ __forceinline__ long long worker_begin(int w, long long T, i
   return (static_cast<long long>(w) * T) / W;
 }
 
+// Also fills the call's RoPE (cos, sin) table for the B new tokens (at
+// positions seqlen[b]) when `rope` is not null, one launch fewer per step.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seqlen, int B, int tile_tokens, int W,
-                                                    int* tile_start, int* seg_start, int* status, int* counters,
-                                                    int n_counters) {
+                                                    int* tile_start, int* seg_start, int* status, const TokenMap tk,
+                                                    float2* rope) {
   __shared__ long long s_scan[1024];
   __shared__ long long s_base;
   griddep_wait();
   if (threadIdx.x == 0) griddep_launch_dependents();
-  for (int i = threadIdx.x; i < n_counters; i += 1024) counters[i] = 0;  // split-K tickets of this call
+  if (rope) {
+    const int half = tk.d_R >> 1;
+    for (int idx = threadIdx.x; idx < B * half; idx += 1024) {
+      float c, s;
+      rope_cos_sin(tok_pos(tk, idx / half), rope_inv_freq(idx % half, tk.d_R, tk.log2_base), c, s);
+      rope[idx] = make_float2(c, s);
+    }
+  }
   // pass 1: cumulative tiles
   if (threadIdx.x == 0) s_base = 0;
   __syncthreads();
