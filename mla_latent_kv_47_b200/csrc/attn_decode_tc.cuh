@@ -10,39 +10,32 @@
 // leave the spare MMA rows zero).
 //
 // Layout on the GPU.  All 128 heads of a sequence share each cache tile, so a
-// tile is read from HBM once per sequence, not once per head.  The fp32 latent
-// accumulator O (128 heads x 512) fills a whole SM's tensor memory, so each
-// worker is a cluster of two CTAs that split the 576 latent columns:
-//   CTA 0: columns c[0,256) and k^R (5 chunks of 64), O columns [0,256)
-//   CTA 1: columns c[256,512)        (4 chunks),     O columns [256,512)
-// Each CTA TMA-loads only its own columns of a tile, so the pair reads every
-// cache byte exactly once.  Each computes a partial score S_r = Q_r C_r^T
-// (tcgen05.mma, M = 128 heads, N = 64 tokens, into one of two TMEM buffers;
-// the c^KV part of Q_r in TMEM, CTA 0's k^R part in shared memory) and both CTAs
-// form S = fp16(S_0) + fp16(S_1) from the same rounded halves, so their
-// softmax, P and running max are bit-identical.  O_r += P C_r (N = 256, the
-// same cache tile read as an MN-major operand) accumulates in TMEM.
+// tile feeds M = 128 MMAs instead of being read once per head.  The fp32
+// latent accumulator O (128 heads x 512) fills a whole SM's tensor memory, so
+// each worker is a cluster of two CTAs, and CTA r accumulates the columns
+// O[:, 256r, 256r + 256).  The pair splits every 64-token tile by tokens for
+// the scores: CTA r computes S for the tile's rows [32r, 32r + 32) over all
+// 576 columns (tcgen05.mma, M = 128 heads, N = 32, K = 576), the two CTAs
+// swap their per-head tile maxima (512 bytes) so both take the same max, and
+// each sends the bf16 P of its 32 rows (8 KB) into the partner's P buffer.
+// Both then run O_r += P C_r over all 64 rows (N = 256): CTA r TMA-loads its
+// own 32 rows whole and the partner's 32 rows in its own 256 columns, so the
+// pair reads the partner-row columns twice, the second time from L2.  A PV
+// retirement is committed to both CTAs' barriers (multicast commit), which
+// tells each side that both P buffers may take the next tile.
 //
-// Warp roles (448 threads per CTA); each tile flows through them in order:
-//   warp 0      TMA producer (4-stage ring of tiles)
-//   warp 1      TMEM owner and MMA issuer: S(j) as soon as tile j landed and
-//               the S buffer of tile j-2 was read out, PV as soon as P is written
-//   warps 2-5   exchange: read S from TMEM, round it to fp16, push it into the
-//               partner's shared memory with st.async (its bytes complete the
-//               partner's barrier, so the sender neither fences nor waits) and
-//               write this CTA's rounded half back over the S buffer for the
-//               softmax (the S buffer is freed once the softmax read it).  The
-//               partner hands a slot back the same way: a 4-byte st.async per
-//               softmax warp that completes this CTA's slot-free barrier.
+// Warp roles (448 threads per CTA):
+//   warp 0      TMA producer (3-stage ring)
+//   warp 1      TMEM owner and MMA issuer: S(j) once tile j landed and the S
+//               buffer was read out, PV(j) once both halves of P(j) are in place
+//   warps 2-5   Q_lat of each piece: chunks 0-6 (bf16 pairs) into TMEM, chunks
+//               7-8 into shared memory, both MMA A operands
 //   warps 6-13  softmax: warp 6+i and warp 10+i share lane quarter i mod 4,
-//               16 heads each; two threads per head (tokens 0-31 and 32-63 of
-//               the tile, via the 16-lane TMEM access shape), so a head's tile
-//               max is one shuffle.  Online softmax with a lazily refreshed
-//               max (O is rescaled only when a tile's max exceeds the running
-//               one by more than 2^8), P (bf16) into shared memory, and the
-//               per-piece epilogue.
-// The exchange warps use thread = head = TMEM lane (warp w owns lanes
-// 32 (w mod 4) ..).
+//               16 heads each; two threads per head (rows 0-15 and 16-31 of
+//               this CTA's half, via the 16-lane TMEM access shape).  Online
+//               softmax with a lazily refreshed max (O is rescaled only when a
+//               tile's max exceeds the running one by more than 2^8), and the
+//               per-piece epilogue; CTA 1 sends its share of l to CTA 0.
 #pragma once
 #include "mla.h"
 #include "ptx.cuh"
@@ -54,28 +47,31 @@ constexpr int kAttnTileTokens = 64;
 constexpr bool kAttnTcReady = true;
 
 namespace attn {
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kThreads = 448;
-constexpr int kChunkBytes = 64 * 128;             // 64 token rows x 64 latent columns, bf16
-constexpr int kStageBytes = 5 * kChunkBytes;      // up to 5 chunks per CTA
-constexpr int kXBytes = 128 * 128;                // one half of S: 128 heads x 64 tokens, fp16
-constexpr int kPBytes = 128 * 128;                // P: 128 heads x 64 tokens, bf16
-constexpr int kXSlots = 2;                        // exchange slots for the partner's score half
-constexpr int kPBufs = 1;                         // P buffers
-constexpr int kQRBytes = 128 * 128;               // CTA 0's k^R part of Q: 128 heads x 64, bf16 (MMA A operand)
-constexpr int kBarBytes = 512;
-// stages | partner's S half x kXSlots | P x kPBufs | k^R part of Q | barriers
-constexpr int kSmem = 1024 + kStages * kStageBytes + kXSlots * kXBytes + kPBufs * kPBytes + kQRBytes + kBarBytes;
-// TMEM columns: O half [0,256), S buffers [256,320) and [320,384) (after the
-// exchange, their first 32 columns hold this CTA's fp16-rounded half), c^KV
-// part of the Q half (bf16 pairs) [384,512)
-constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 384, kTmemCols = 512;
+constexpr int kHalf = 32;                              // rows of a tile whose scores one CTA computes
+constexpr int kChunkBytes = kHalf * 128;               // 32 token rows x 64 latent columns, bf16, 128B swizzle
+constexpr int kOwnChunks = 9;                          // own rows: all 576 columns
+constexpr int kPeerChunks = 4;                         // partner's rows: this CTA's 256 c^KV columns
+constexpr int kStageBytes = (kOwnChunks + kPeerChunks) * kChunkBytes;
+constexpr int kQTmemChunks = 7;                        // Q chunks held in TMEM; the rest in shared memory
+constexpr int kQSmemChunks = 9 - kQTmemChunks;
+constexpr int kQChunkBytes = 128 * 128;                // 128 heads x 64 columns, bf16
+constexpr int kPBytes = 128 * 128;                     // P: 128 heads x 64 rows, bf16 (CTA 0's rows first)
+constexpr int kPBufs = 2;
+constexpr int kAuxBytes = 2048;                        // partner maxima, CTA 1's l, barriers
+// stages | Q chunks 7-8 | P x 2 | aux
+constexpr int kSmem = 1024 + kStages * kStageBytes + kQSmemChunks * kQChunkBytes + kPBufs * kPBytes + kAuxBytes;
+// TMEM columns: O half [0,256), S [256,288), Q chunks 0-6 (bf16 pairs) [288,512)
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 288, kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;
-constexpr int kRow = 576;                         // d_c + d_R
+constexpr int kRow = 576;                              // d_c + d_R
+static_assert(kTmemQ + kQTmemChunks * 32 == kTmemCols, "TMEM budget");
+static_assert(kSmem <= 232448, "shared memory budget");
 }  // namespace attn
 
 struct AttnArgs {
-  CUtensorMap map_cache;       // cache rows [n_rows x 576] bf16, box {64 columns, 64 rows}, 128B swizzle
+  CUtensorMap map_cache;       // cache rows [n_rows x 576] bf16, box {64 columns, 32 rows}, 128B swizzle
   const __nv_bfloat16* qlat;   // [B][n_h][576]
   const int64_t* seq_start;
   const int32_t* seqlen;
@@ -87,77 +83,63 @@ struct AttnArgs {
   int* status;
 };
 
-__device__ __forceinline__ int attn_chunk_col(uint32_t rank, int ci) {
-  return rank == 0 ? (ci < 4 ? ci * 64 : 512) : 256 + ci * 64;
-}
-
-// fp16 pair (lo in the low half), rounded to nearest and saturated to the
-// largest finite fp16 so an extreme partial score cannot become inf.
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-__device__ __forceinline__ float2 unpack_half2(uint32_t v) {
-  return __half22float2(*reinterpret_cast<const __half2*>(&v));
-}
-
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     attn_decode_tc_kernel(const __grid_constant__ AttnArgs a) {
   using namespace attn;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* stages = smem;
-  uint8_t* xpeer = stages + kStages * kStageBytes;  // [kXSlots] the partner's half of S (fp16), written by the partner
-  uint8_t* pbuf = xpeer + kXSlots * kXBytes;        // [kPBufs] P (bf16), MMA A operand
-  uint8_t* qr = pbuf + kPBufs * kPBytes;            // CTA 0: k^R part of Q (bf16), MMA A operand
-  uint64_t* full = reinterpret_cast<uint64_t*>(qr + kQRBytes);
+  uint8_t* qs = stages + kStages * kStageBytes;       // Q chunks 7-8, MMA A operand
+  uint8_t* pbuf = qs + kQSmemChunks * kQChunkBytes;   // [2] P (bf16), MMA A operand
+  uint8_t* aux = pbuf + kPBufs * kPBytes;
+  float* mx = reinterpret_cast<float*>(aux);          // [2][128] the partner's tile maxima (st.async)
+  float* lsh = mx + 256;                              // [128] CTA 1's share of l, in CTA 0 (st.async)
+  uint64_t* full = reinterpret_cast<uint64_t*>(aux + 1536);
   uint64_t* empty = full + kStages;
-  uint64_t* s_full = empty + kStages;  // [2] S(j) in buffer j & 1 (MMA -> exchange)
-  uint64_t* s_free = s_full + 2;       // [2] buffer read out by the softmax (softmax -> MMA)
-  uint64_t* xo_full = s_free + 2;      // [2] own rounded half written back (exchange -> softmax)
-  uint64_t* x_full = xo_full + 2;    // [kXSlots] partner's half landed (st.async bytes)
-  uint64_t* x_free = x_full + kXSlots;  // [kXSlots] partner's half consumed (signals from the partner's softmax)
-  uint64_t* p_full = x_free + kXSlots;  // [kPBufs]
-  uint64_t* p_free = p_full + kPBufs;   // [kPBufs]
-  uint64_t* q_full = p_free + kPBufs;
-  uint64_t* o_done = q_full + 1;
-  uint64_t* drain = o_done + 1;
-  uint32_t* sig = reinterpret_cast<uint32_t*>(drain + 1);  // [kXSlots][8] landing words of the partner's slot-free signals
-  uint32_t* tmem_slot = sig + 8 * kXSlots;
+  uint64_t* s_full = empty + kStages;  // S(j) in TMEM (MMA -> softmax)
+  uint64_t* s_free = s_full + 1;       // S read out (softmax -> MMA)
+  uint64_t* mx_full = s_free + 1;      // [2] the partner's maxima of tile j landed (index j & 1)
+  uint64_t* p_full = mx_full + 2;      // [2] this CTA's half of P(j) written
+  uint64_t* px_full = p_full + 2;      // [2] the partner's half of P(j) landed
+  uint64_t* pv_done = px_full + 2;     // [2] PV(j) retired in both CTAs (one commit from each)
+  uint64_t* q_full = pv_done + 2;
+  uint64_t* q_free = q_full + 1;       // last S of the piece retired (MMA -> Q warps)
+  uint64_t* o_done = q_free + 1;
+  uint64_t* l_full = o_done + 1;       // CTA 0: CTA 1's l of the piece landed
+  uint64_t* drain = l_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
   const int w = blockIdx.x >> 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nchunks = rank == 0 ? 5 : 4;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 8);        // one arrival per softmax warp
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 8);   // one arrival per softmax warp
-      mbar_init(&xo_full[i], 4);  // one arrival per exchange warp
-    }
-    for (int i = 0; i < kXSlots; ++i) {
-      mbar_init(&x_full[i], 1);   // armed once per phase with the expected bytes
-      mbar_init(&x_free[i], 1);   // armed by the exchange before each use; 8 x 4 signal bytes from the partner
-    }
-    for (int i = 0; i < kPBufs; ++i) {
+      mbar_init(&mx_full[i], 1);  // armed per phase with the partner's 512 bytes
       mbar_init(&p_full[i], 8);   // one arrival per softmax warp
-      mbar_init(&p_free[i], 1);
+      mbar_init(&px_full[i], 1);  // armed per phase with the partner's 8 KB
+      mbar_init(&pv_done[i], 2);  // this CTA's and the partner's PV commit
     }
     mbar_init(q_full, 128);
+    mbar_init(q_free, 1);
     mbar_init(o_done, 1);
+    mbar_init(l_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    // phase 0 of every exchange slot expects the partner's 16 KB
-    for (int i = 0; i < kXSlots; ++i) mbar_arrive_expect_tx(&x_full[i], kXBytes);
+    for (int i = 0; i < 2; ++i) {
+      mbar_arrive_expect_tx(&mx_full[i], 128 * 4);
+      mbar_arrive_expect_tx(&px_full[i], kPBytes / 2);
+    }
+    if (rank == 0) mbar_arrive_expect_tx(l_full, 128 * 4);
   }
   if (warp == 0 && lane == 0) prefetch_tmap(&a.map_cache);
   if (warp == 1) {
@@ -174,7 +156,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (elect_one()) {
-      const uint64_t pol = policy_evict_first();
+      // Bytes the partner also loads keep the normal L2 priority, so that the
+      // second read is an L2 hit; the rest is streamed with evict-first.
+      const uint64_t pol_once = policy_evict_first();
+      const uint64_t pol_twice = policy_evict_normal();
       int it = 0;
       for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
         if (*abort_flag) return;
@@ -182,18 +167,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         for (int t = p.t0; t < p.t1; ++t, ++it) {
           const int s = it % kStages;
           if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, wc)) return;
-          mbar_arrive_expect_tx(&full[s], nchunks * kChunkBytes);
+          mbar_arrive_expect_tx(&full[s], kStageBytes);
           uint8_t* dst = stages + s * kStageBytes;
-          const int y = static_cast<int>(row0 + static_cast<long long>(t) * 64);
-          for (int ci = 0; ci < nchunks; ++ci)
-            tma_load_2d(dst + ci * kChunkBytes, &a.map_cache, &full[s], attn_chunk_col(rank, ci), y, pol);
+          const long long y0 = row0 + static_cast<long long>(t) * kAttnTileTokens;
+          const int y_own = static_cast<int>(y0 + kHalf * rank), y_peer = static_cast<int>(y0 + kHalf * peer);
+          for (int ci = 0; ci < kOwnChunks; ++ci) {
+            const bool shared = ci >= 4 * static_cast<int>(peer) && ci < 4 * static_cast<int>(peer) + 4;
+            tma_load_2d(dst + ci * kChunkBytes, &a.map_cache, &full[s], ci * 64, y_own, shared ? pol_twice : pol_once);
+          }
+          for (int cj = 0; cj < kPeerChunks; ++cj)
+            tma_load_2d(dst + (kOwnChunks + cj) * kChunkBytes, &a.map_cache, &full[s],
+                        (4 * static_cast<int>(rank) + cj) * 64, y_peer, pol_twice);
         }
       });
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
-      constexpr uint32_t idesc_s = idesc_bf16(128, 64, false, false);
+      constexpr uint32_t idesc_s = idesc_bf16(128, kHalf, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(128, 256, false, true);
       int it = 0, piece = 0;
       for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
@@ -201,8 +192,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         if (!mbar_wait(q_full, piece & 1, wc)) return;
         tc_fence_after();
         const int nt = p.t1 - p.t0;
-        // PV first: it gates the softmax of the next tile, while S only has
-        // to be ready by the time the exchange warps come back for it.
         int ns = 0, npv = 0;
         uint32_t spins = 0;
         uint64_t t_idle = 0;
@@ -211,17 +200,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           if (npv < ns) {
             const int g = it + npv;
             const int s = g % kStages;
-            const int b = g % kPBufs;
-            if (mbar_test_wait(smem_u32(&p_full[b]), (g / kPBufs) & 1)) {
+            const int b = g & 1;
+            const uint32_t ph = (g >> 1) & 1;
+            if (mbar_test_wait(smem_u32(&p_full[b]), ph) && mbar_test_wait_cluster(smem_u32(&px_full[b]), ph)) {
               tc_fence_after();
+              fence_proxy_async_smem();  // the partner's half came in through st.async
+              // next phase: the partner's half of P(g + 2), which it sends only
+              // after this PV retired
+              mbar_arrive_expect_tx(&px_full[b], kPBytes / 2);
               const uint32_t st = smem_u32(stages + s * kStageBytes);
+              const uint32_t own_rows = st + 4 * rank * kChunkBytes;      // own rows, this CTA's c^KV columns
+              const uint32_t peer_rows = st + kOwnChunks * kChunkBytes;   // partner rows, the same columns
               const uint32_t pb = smem_u32(pbuf + b * kPBytes);
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                mma_ss(tmem + kTmemO, sdesc_sw128(pb + kk * 32, 16, 1024), sdesc_sw128(st + kk * 2048, 8192, 1024),
-                       idesc_pv, (npv > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk) {  // rows [16 kk, 16 kk + 16) of the tile; CTA 0's rows first
+                const uint32_t rows = (kk >> 1) == static_cast<int>(rank) ? own_rows : peer_rows;
+                mma_ss(tmem + kTmemO, sdesc_sw128(pb + kk * 32, 16, 1024),
+                       sdesc_sw128(rows + (kk & 1) * 2048, kChunkBytes, 1024), idesc_pv, (npv > 0 || kk > 0) ? 1u : 0u);
               }
-              mma_commit(&p_free[b]);
+              mma_commit_multicast(&pv_done[b], 0x3);  // P buffer b is free in both CTAs once both commits land
               mma_commit(&empty[s]);
               if (npv == nt - 1) mma_commit(o_done);
               ++npv;
@@ -231,27 +228,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           if (!issued && ns < nt) {
             const int g = it + ns;
             const int s = g % kStages;
-            const int sb = g & 1;
             if (mbar_test_wait(smem_u32(&full[s]), (g / kStages) & 1) &&
-                mbar_test_wait(smem_u32(&s_free[sb]), ((g >> 1) & 1) ^ 1)) {
+                mbar_test_wait(smem_u32(s_free), (g & 1) ^ 1)) {
               tc_fence_after();
               const uint32_t st = smem_u32(stages + s * kStageBytes);
-              const uint32_t dS = tmem + kTmemS + sb * 64;
-              for (int ci = 0; ci < 4; ++ci) {
+              const uint32_t dS = tmem + kTmemS;
+              for (int ci = 0; ci < kQTmemChunks; ++ci) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                   mma_ts(dS, tmem + kTmemQ + ci * 32 + kk * 8, sdesc_sw128(st + ci * kChunkBytes + kk * 32, 16, 1024),
                          idesc_s, (ci | kk) ? 1u : 0u);
                 }
               }
-              if (nchunks == 5) {  // CTA 0: the k^R chunk, Q_R from shared memory
+              for (int ci = 0; ci < kQSmemChunks; ++ci) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                  mma_ss(dS, sdesc_sw128(smem_u32(qr) + kk * 32, 16, 1024),
-                         sdesc_sw128(st + 4 * kChunkBytes + kk * 32, 16, 1024), idesc_s, 1u);
+                  mma_ss(dS, sdesc_sw128(smem_u32(qs) + ci * kQChunkBytes + kk * 32, 16, 1024),
+                         sdesc_sw128(st + (kQTmemChunks + ci) * kChunkBytes + kk * 32, 16, 1024), idesc_s, 1u);
                 }
               }
-              mma_commit(&s_full[sb]);
+              mma_commit(s_full);
+              if (ns == nt - 1) mma_commit(q_free);  // no MMA of this piece reads Q any more
               ++ns;
               issued = true;
             }
@@ -277,24 +274,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       mma_commit(drain);
     }
   } else if (warp < 6) {
-    // ------------------------------------------------------------ exchange
+    // ------------------------------------------------------------ Q_lat of each piece
     const int q4 = warp & 3;
     const int h = q4 * 32 + lane;  // head = TMEM lane
     const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int sw = h & 7;
-    const uint32_t peer_row = mapa(smem_u32(xpeer), peer) + h * 128;
-    const uint32_t xfull_peer = mapa(smem_u32(x_full), peer);
-    const uint32_t qr_row = smem_u32(qr) + h * 128;
-    const bool arm = warp == 2 && lane == 0;
-    int it = 0;
+    const uint32_t q_row = smem_u32(qs) + h * 128;
+    int piece = 0;
     for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
       if (*abort_flag) return;
-      // ---- this CTA's half of Q_lat[b, h] into TMEM (MMA A operand).  The
-      // previous piece's last S has been read out, so no MMA still reads Q.
+      // the previous piece's S products have retired: nothing reads Q now
+      if (piece > 0 && !mbar_wait(q_free, (piece - 1) & 1, wc)) return;
+      tc_fence_after();
       const bool head = h < a.n_h;
       const __nv_bfloat16* qrow = a.qlat + (static_cast<long long>(p.b) * a.n_h + (head ? h : 0)) * kRow;
-      for (int ci = 0; ci < 4; ++ci) {
-        const uint4* src = reinterpret_cast<const uint4*>(qrow + attn_chunk_col(rank, ci));
+      for (int ci = 0; ci < kQTmemChunks; ++ci) {
+        const uint4* src = reinterpret_cast<const uint4*>(qrow + ci * 64);
         uint32_t r[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -303,156 +298,107 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         }
         tmem_st32(tl + kTmemQ + ci * 32, r);
       }
-      if (nchunks == 5) {  // CTA 0: the k^R part of Q into shared memory, 128-byte swizzled rows
-        const uint4* src = reinterpret_cast<const uint4*>(qrow + attn_chunk_col(rank, 4));
+      for (int ci = 0; ci < kQSmemChunks; ++ci) {  // 128-byte swizzled rows
+        const uint4* src = reinterpret_cast<const uint4*>(qrow + (kQTmemChunks + ci) * 64);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) st_shared_v4(qr_row + ((i ^ sw) << 4), head ? src[i] : make_uint4(0, 0, 0, 0));
-        fence_proxy_async_smem();
+        for (int i = 0; i < 8; ++i)
+          st_shared_v4(q_row + ci * kQChunkBytes + ((i ^ sw) << 4), head ? src[i] : make_uint4(0, 0, 0, 0));
       }
+      fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(q_full);
-
-      const int nt = p.t1 - p.t0;
-      for (int k = 0; k < nt; ++k) {
-        const int g = it + k;
-        const int slot = g % kXSlots;
-        const uint32_t ph = (g / kXSlots) & 1;
-        const int sb = g & 1;
-        if (!mbar_wait(&s_full[sb], (g >> 1) & 1, wc)) return;
-        tc_fence_after();
-        uint32_t hx[32];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t sr[32];
-          tmem_ld32(tl + kTmemS + sb * 64 + half * 32, sr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            hx[half * 16 + j] = pack_half2(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1]));
-        }
-        // partner first: its copy has the longer way to go
-        if (!mbar_wait<true>(&x_free[slot], ph ^ 1, wc)) return;
-        // the partner returns this use of the slot with 8 signals of 4 bytes;
-        // armed before this warp's data goes out, so no signal can precede it
-        if (arm) mbar_arrive_expect_tx(&x_free[slot], 32);
-        const uint32_t dst = peer_row + slot * kXBytes;
-        const uint32_t bar = xfull_peer + slot * 8;  // x_full[slot] in the partner
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          st_async_v4(dst + ((i ^ sw) << 4), make_uint4(hx[4 * i], hx[4 * i + 1], hx[4 * i + 2], hx[4 * i + 3]), bar);
-        // own rounded half over the first 32 columns of the S buffer
-        tmem_st32(tl + kTmemS + sb * 64, hx);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&xo_full[sb]);
-      }
-      it += nt;
+      ++piece;
     });
-    // The partner's signals for the last use of each slot land in this CTA's
-    // shared memory: they must have arrived before the CTA may exit.
-    if (arm && !*abort_flag) {
-      for (int s2 = 0; s2 < kXSlots; ++s2) {
-        const int uses = (it + kXSlots - 1 - s2) / kXSlots;  // tiles g < it with g % kXSlots == s2
-        if (uses > 0 && !mbar_wait<true>(&x_free[s2], (uses - 1) & 1, wc)) break;
-      }
-    }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int q4 = warp & 3;
     const int hs = (warp - 6) >> 2;  // which 16 heads of the lane quarter
-    const int th = lane >> 4;        // token half of the tile: [32 th, 32 th + 32)
+    const int th = lane >> 4;        // rows [16 th, 16 th + 16) of this CTA's half
     const int h = q4 * 32 + hs * 16 + (lane & 15);
     const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32 + hs * 16) << 16);
     const int sw = h & 7;
-    const bool leader = warp == 6;   // re-arms the exchange barriers
-    const uint32_t peer_row = smem_u32(xpeer) + h * 128;
+    const bool lead = warp == 6 && lane == 0;  // re-arms the barriers the partner completes
     const uint32_t p_row = smem_u32(pbuf) + h * 128;
-    const uint32_t xfree_peer = mapa(smem_u32(x_free), peer);
-    const uint32_t sig_peer = mapa(smem_u32(sig), peer) + (warp - 6) * 4;
+    const uint32_t p_row_peer = mapa(p_row, peer);
+    const uint32_t pxfull_peer = mapa(smem_u32(px_full), peer);
+    const uint32_t mx_peer = mapa(smem_u32(mx), peer) + h * 4;
+    const uint32_t mxfull_peer = mapa(smem_u32(mx_full), peer);
     int it = 0, piece = 0;
     for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
       if (*abort_flag) return;
       const bool head = h < a.n_h;
       const int L1 = a.seqlen[p.b] + 1;
-      float m_run = -INFINITY, l_run = 0.f;  // l_run: this thread's token half only
+      float m_run = -INFINITY, l_run = 0.f;  // l_run: this thread's 16 rows only
       const int nt = p.t1 - p.t0;
       for (int k = 0; k < nt; ++k) {
         const int g = it + k;
-        const int t = p.t0 + k;
-        const int slot = g % kXSlots;
-        const uint32_t ph = (g / kXSlots) & 1;
-        const int sb = g & 1;
-        if (!mbar_wait(&xo_full[sb], (g >> 1) & 1, wc)) return;
-        if (!mbar_wait<true>(&x_full[slot], ph, wc)) return;
+        const int b = g & 1;
+        const uint32_t ph = (g >> 1) & 1;
+        if (!mbar_wait(s_full, g & 1, wc)) return;
         tc_fence_after();
-        // ---- full scores of this thread's 32 tokens (same bits in both CTAs)
-        uint32_t own[16];
-        tmem_ld16x2(tl + kTmemS + sb * 64, own);
-        uint4 pv[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) pv[i] = ld_shared_v4(peer_row + slot * kXBytes + (((th * 4 + i) ^ sw) << 4));
+        uint32_t sr[16];
+        tmem_ld16x2(tl + kTmemS, sr);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&s_free[sb]);  // S buffer sb may take S(g + 2)
-          // the slot's next phase expects the partner's next 16 KB; armed
-          // before the slot is released, so no byte can land ahead of it
-          if (leader) mbar_arrive_expect_tx(&x_full[slot], kXBytes);
-        }
-        const int valid = min(64, L1 - t * 64) - th * 32;  // valid tokens of this half (may be <= 0)
-        float sc[32];
+        if (lane == 0) mbar_arrive(s_free);
+        const int tile0 = (p.t0 + k) * kAttnTileTokens;
+        const int valid = min(16, L1 - (tile0 + kHalf * static_cast<int>(rank) + 16 * th));  // may be <= 0
+        float sc[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t vv[4] = {pv[i].x, pv[i].y, pv[i].z, pv[i].w};
+        for (int j = 0; j < 16; ++j) sc[j] = __uint_as_float(sr[j]);
+        if (__any_sync(0xffffffffu, valid < 16)) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 x = unpack_half2(own[4 * i + e]), y = unpack_half2(vv[e]);
-            sc[8 * i + 2 * e] = x.x + y.x;
-            sc[8 * i + 2 * e + 1] = x.y + y.y;
-          }
-        }
-        // every value read from the partner's half is consumed: hand the slot back
-        __syncwarp();
-        if (lane == 0) st_async_b32(sig_peer + slot * 32, 0u, xfree_peer + slot * 8);  // into sig[slot][warp - 6]
-        if (__any_sync(0xffffffffu, valid < 32)) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
+          for (int j = 0; j < 16; ++j)
             if (j >= valid) sc[j] = -INFINITY;
         }
-        float mh = sc[0];
+        float mo = sc[0];
 #pragma unroll
-        for (int j = 1; j < 32; ++j) mh = fmaxf(mh, sc[j]);
-        const float mt = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));  // the head's other token half
+        for (int j = 1; j < 16; ++j) mo = fmaxf(mo, sc[j]);
+        mo = fmaxf(mo, __shfl_xor_sync(0xffffffffu, mo, 16));  // this CTA's 32 rows
+        if (th == 0) st_async_b32(mx_peer + b * 512, __float_as_uint(mo), mxfull_peer + b * 8);
+        // P of this thread's rows against max m; returns their sum
+        uint32_t pk[8];
+        auto exp_rows = [&](float m) {
+          float sum = 0.f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float p0 = ex2_approx(sc[2 * j] - m), p1 = ex2_approx(sc[2 * j + 1] - m);
+            sum += p0 + p1;
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+            pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          return sum;
+        };
+        // Past a piece's first tile the max almost always stays, so P is formed
+        // against it while the partner's maxima are on their way, and formed
+        // again only if the tile's max does move it.
+        float lsum = k > 0 ? exp_rows(m_run) : 0.f;
+        if (!mbar_wait<true>(&mx_full[b], ph, wc)) return;
+        const float mt = fmaxf(mo, mx[b * 128 + h]);  // the tile's max, the same in both CTAs
+        // next phase: the partner's maxima of tile g + 2, which it sends only
+        // after this CTA's maxima of tile g + 1 (sent after this point) landed
+        if (lead) mbar_arrive_expect_tx(&mx_full[b], 128 * 4);
         float m_new = m_run, alpha = 1.f;
         bool rescale = false;
         if (k == 0) {
           m_new = mt;
+          lsum = exp_rows(m_new);
         } else if (mt > m_run + kRescaleLog2) {
           m_new = mt;
           alpha = ex2_approx(m_run - m_new);
           rescale = true;
-        }
-        uint32_t pk[16];
-        float lsum = 0.f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float p0 = ex2_approx(sc[2 * j] - m_new), p1 = ex2_approx(sc[2 * j + 1] - m_new);
-          lsum += p0 + p1;
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-          pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
+          lsum = exp_rows(m_new);
         }
         l_run = l_run * alpha + lsum;
         m_run = m_new;
-        // ---- P buffer b is free once PV(g-2) retired
-        const int b = g % kPBufs;
-        if (!mbar_wait(&p_free[b], ((g / kPBufs) & 1) ^ 1, wc)) return;
+        // ---- P buffer b is free in both CTAs once PV(g-2) retired in both
+        if (!mbar_wait_inline(&pv_done[b], ph ^ 1, wc)) return;
         tc_fence_after();
         if (__any_sync(0xffffffffu, rescale)) {
           // O must hold PV(g-1) before it is scaled (k >= 1 here, so g >= 1)
-          if (kPBufs > 1 && !mbar_wait(&p_free[(g - 1) % kPBufs], ((g - 1) / kPBufs) & 1, wc)) return;
+          if (!mbar_wait_inline(&pv_done[b ^ 1], ((g - 1) >> 1) & 1, wc)) return;
           tc_fence_after();
           for (int c = 0; c < 256; c += 32) {
             uint32_t o[16];
@@ -464,27 +410,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           }
           tmem_wait_st();
         }
-        const int v64 = valid + th * 32;
-        if (v64 < 64) {
+        const int v64 = min(kAttnTileTokens, L1 - tile0);  // valid rows of the tile
+        if (v64 < kAttnTileTokens) {
           // rows past the sequence may hold anything (even NaN); 0 * NaN would
           // poison O, so the rows this CTA multiplies into O are zeroed
           uint8_t* st = stages + (g % kStages) * kStageBytes;
-          const int n16 = (64 - v64) * 32;
+          const int n16 = (kAttnTileTokens - v64) * 32;  // 16-byte pieces: 4 chunks x 8 per row
           for (int idx = (warp - 6) * 32 + lane; idx < n16; idx += 256) {
             const int row = v64 + (idx >> 5), c16 = idx & 31;
-            *reinterpret_cast<uint4*>(st + (c16 >> 3) * kChunkBytes + row * 128 + (c16 & 7) * 16) = make_uint4(0, 0, 0, 0);
+            const bool own = (row >> 5) == static_cast<int>(rank);
+            const int chunk = (own ? 4 * static_cast<int>(rank) : kOwnChunks) + (c16 >> 3);
+            *reinterpret_cast<uint4*>(st + chunk * kChunkBytes + (row & 31) * 128 + (c16 & 7) * 16) = make_uint4(0, 0, 0, 0);
           }
         }
+        // ---- this CTA's half of P(g): rows [32 rank + 16 th, +16) of the tile,
+        // into the local buffer and the partner's
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          st_shared_v4(p_row + b * kPBytes + (((th * 4 + i) ^ sw) << 4),
-                       make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
+        for (int i = 0; i < 2; ++i) {
+          const uint32_t off = b * kPBytes + (((4 * rank + 2 * th + i) ^ sw) << 4);
+          const uint4 v = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          st_async_v4(p_row_peer + off, v, pxfull_peer + b * 8);
+          st_shared_v4(p_row + off, v);
+        }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[b]);
       }
-      // ---- epilogue of the piece: unnormalised O_r, m, l
+      // ---- epilogue of the piece: unnormalised O_r; CTA 0 writes m and l
       if (!mbar_wait(o_done, piece & 1, wc)) return;
       tc_fence_after();
       float* dst = a.o_part + (static_cast<long long>(p.slot) * a.n_h + h) * 512 + rank * 256 + th * 16;
@@ -499,15 +452,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
                                                                 __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
         }
       }
-      const float l_head = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
-      if (rank == 0 && th == 0 && head) {
-        a.ml_part[(static_cast<long long>(p.slot) * a.n_h + h) * 2] = m_run;
-        a.ml_part[(static_cast<long long>(p.slot) * a.n_h + h) * 2 + 1] = l_head;
+      const float l_head = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);  // this CTA's 32 rows of each tile
+      if (rank == 1) {
+        if (th == 0) st_async_b32(mapa(smem_u32(lsh), peer) + h * 4, __float_as_uint(l_head), mapa(smem_u32(l_full), peer));
+      } else {
+        if (!mbar_wait<true>(l_full, piece & 1, wc)) return;
+        if (th == 0 && head) {
+          a.ml_part[(static_cast<long long>(p.slot) * a.n_h + h) * 2] = m_run;
+          a.ml_part[(static_cast<long long>(p.slot) * a.n_h + h) * 2 + 1] = l_head + lsh[h];
+        }
+        // next phase: CTA 1's l of the next piece, which needs this CTA's P of
+        // that piece first
+        if (lead) mbar_arrive_expect_tx(l_full, 128 * 4);
       }
       tc_fence_before();
       it += nt;
       ++piece;
     });
+    // The partner's PV commits for the last uses of both P buffers land in
+    // this CTA's shared memory: they must have arrived before the CTA may exit.
+    if (lead && !*abort_flag) {
+      for (int b = 0; b < 2; ++b) {
+        const int uses = (it + 1 - b) / 2;  // tiles g < it with g & 1 == b
+        if (uses > 0 && !mbar_wait<true>(&pv_done[b], (uses - 1) & 1, wc)) break;
+      }
+    }
   }
   // ---- teardown: every MMA retired, the partner no longer writes into this CTA.
   // The next kernel is released only now: its CTAs would otherwise sit on

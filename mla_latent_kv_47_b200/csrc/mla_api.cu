@@ -472,7 +472,7 @@ mla_status launch_attn_decode_tc(const __nv_bfloat16* qlat, const mla_cache* cac
   AttnArgs a;
   memset(&a, 0, sizeof(a));
   if (cache->n_rows > (1ll << 31) - 128) return MLA_ERR_UNSUPPORTED;  // tile rows are int32 TMA coordinates
-  if (!make_map_2d(&a.map_cache, cache->base, attn::kRow, cache->n_rows, attn::kRow, 64)) return MLA_ERR_CUDA;
+  if (!make_map_2d(&a.map_cache, cache->base, attn::kRow, cache->n_rows, attn::kRow, attn::kHalf)) return MLA_ERR_CUDA;
   a.qlat = qlat;
   a.seq_start = cache->seq_start;
   a.seqlen = seqlen;
