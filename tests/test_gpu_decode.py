@@ -26,7 +26,7 @@ def m():
     return mod
 
 
-def run_decode(m, preset, checked, lengths=None, pad=2, oracle="unabsorbed", dirty_workspace=False):
+def run_decode(m, preset, checked, lengths=None, pad=2, oracle="unabsorbed", dirty_workspace=False, h_scale=None):
     from mla_latent_kv_47_b200.cache import LatentCache
     p = synth.preset(preset)
     d = p.dims
@@ -40,6 +40,8 @@ def run_decode(m, preset, checked, lengths=None, pad=2, oracle="unabsorbed", dir
         ws.fill_(0xFF)      # NaN floats, -1 counters: nothing may be read before it is written
         ws[:256].zero_()    # except the status word, zeroed once by contract
     seqs_h = {b: synth.hidden(p, b, L[b] + 1) for b in checked}
+    if h_scale is not None:   # per-token scale of the checked sequences (powers of two keep bf16 values exact)
+        seqs_h = {b: h * h_scale(np.arange(h.shape[0]))[:, None].astype(h.dtype) for b, h in seqs_h.items()}
     gu.fill_cache(m, dims, Wd, cache, ws, seqs_h, L, p)
     tdt = torch.float32 if d.dtype == "fp32" else torch.bfloat16
     g = torch.Generator(device="cuda")
@@ -138,6 +140,29 @@ def test_decode_with_dirty_workspace(m, preset, L):
             gu.assert_gate(s, 1e-4, 1e-4)
         else:
             gu.assert_gate(s)
+
+
+def test_lazy_rescale_of_o(m):
+    """Cached tokens scaled by 1 and 4 in alternate 64-token tiles (the query
+    row unscaled) put the max score of a scaled tile ~11.5 log2 units above an
+    unscaled tile's (~15 against ~3.5), past the kernel's 2^8 rescale
+    threshold, so the lazy rescale of O and l runs inside most pieces;
+    unscaled inputs never reach it.  The lengths give ~2.8 tiles per worker,
+    so pieces span several tiles.  With scores this large the bf16 operands
+    alone (Q_lat, cache rows, P) cost up to 0.72% max / 0.15% mean of max|u|
+    (fp64 emulation of those roundings), inside the gate; larger scales push
+    that bound past it."""
+    L = [8192, 4000, 777]
+
+    def scale(pos):
+        s = np.array([1.0, 4.0])[(pos // 64) % 2]
+        s[-1] = 1.0   # the new token, whose query scores the rest
+        return s
+
+    st = run_decode(m, "v2", checked=[0, 1, 2], lengths=L, h_scale=scale)
+    for s in st.values():
+        gu.assert_gate(s)
+    print("rescale gate", st)
 
 
 def test_single_token_closed_form(m):
