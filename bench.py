@@ -69,6 +69,17 @@ def workload_lengths(name, ctx=0, batch=0):
     return p, L
 
 
+def workload_config(args, world):
+    """The `config` object of the JSON line; both arms report the same one."""
+    p, L = workload_lengths(args.workload, args.ctx, args.batch)
+    cache_bytes = decode_flops_bytes(p.dims, L)[2]
+    return {"workload": f"{args.workload} decode: DeepSeek-V2 MLA dims" if args.workload != "lite"
+            else "lite decode: DeepSeek-V2-Lite MLA dims",
+            "global_batch": world * len(L), "seq_len": max(L) + 1, "cached_tokens": sum(L),
+            "parallelism": f"dp-by-sequence replicas x{world}",
+            "l2": f"inputs larger than L2 (cache {cache_bytes / 1e6:.0f} MB + weights)"}
+
+
 def decode_flops_bytes(d, L):
     """Algorithmic FLOPs and HBM bytes of one decode step (bf16 storage)."""
     B = len(L)
@@ -217,14 +228,14 @@ def run_reference(args):
     import numpy as np
     import synth
     from oracle import mla as om
-    p = synth.preset(args.workload)
+    p, L = workload_lengths(args.workload, args.ctx, args.batch)
     Wh = synth.weights(p)
     hs = {}
 
     def step(i):
-        b = i % p.batch
+        b = i % len(L)
         if b not in hs:
-            hs[b] = synth.hidden(p, b, p.seqlen[b] + 1)
+            hs[b] = synth.hidden(p, b, L[b] + 1)
         u = om.decode_unabsorbed(Wh, hs[b], p.dims)
         assert np.all(np.isfinite(u))
 
@@ -236,13 +247,12 @@ def run_reference(args):
     dt = (time.perf_counter() - t0) / args.steps
     value = 1.0 / dt  # one new token per step (one sequence of the batch)
     cores = blas_threads()
-    sample = f"{args.steps} steps, each the fp64 un-absorbed oracle on one whole sequence of the {args.workload} workload ({p.seqlen[0] + 1} tokens)"
+    sample = f"{args.steps} steps, each the fp64 un-absorbed oracle on one whole sequence of the {args.workload} workload ({L[0] + 1} tokens)"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{args.workload} decode", "global_batch": p.batch, "seq_len": p.seqlen[0] + 1,
-                   "parallelism": "host cores"},
+        "config": workload_config(args, args.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -431,11 +441,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,0.02) weights, N(0,1) hidden states)",
-        "config": {"workload": f"{args.workload} decode: DeepSeek-V2 MLA dims" if args.workload != "lite"
-                   else "lite decode: DeepSeek-V2-Lite MLA dims",
-                   "global_batch": world * B, "seq_len": max(L) + 1, "cached_tokens": sum(L),
-                   "parallelism": f"dp-by-sequence replicas x{world}",
-                   "l2": f"inputs larger than L2 (cache {cache_bytes / 1e6:.0f} MB + weights)"},
+        "config": workload_config(args, world),
         "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": hbm_gbs, "unit": "GB/s",
                      "frac": attn_gbs / hbm_gbs, "traffic": traffic,
                      "kernel": "decode attention (latent-cache stream)",
