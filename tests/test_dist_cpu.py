@@ -56,3 +56,23 @@ def test_single_rank_reduce_is_identity():
     import bench
     assert bench.reduce_max(3.25, 1, None) == 3.25
     assert bench.job_throughput(1, 64, 0.5) == pytest.approx(128000.0)
+
+
+def test_reference_arm_line_keeps_the_contract(capsys, monkeypatch):
+    """The reference arm's JSON line carries the contract's keys and the same
+    config object as the CUDA arm (both come from bench.workload_config)."""
+    import json
+    import bench
+    monkeypatch.setenv("RANK", "0")
+
+    class A:
+        workload = "tiny"; steps = 1; warmup = 0; gpus = 1; ctx = 0; batch = 0
+    assert bench.run_reference(A()) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in line, k
+    assert line["impl"] == "reference" and line["higher_is_better"] is True
+    assert line["config"] == bench.workload_config(A(), 1)
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
