@@ -29,8 +29,12 @@ design notes of this repository):
     cache row is [c^KV | k^R].
   * Without query compression (V2-Lite, App. B.1) W^{UQ} and W^{QR} act on
     h_t directly.
-  * RMSNorm on the latents and YaRN scaling (§3.1.2, §3.1.4) are not part of
-    App. C and are not applied.
+  * RMSNorm on the latents (§3.1.2) is not part of App. C.  It is applied
+    only when the weights carry its gains: "g_kv" [d_c] normalises c^KV
+    before it is cached, and "g_q" [d_cq] normalises c^Q before the
+    up-projections (RMS over the latent's own width, eps = RMS_EPS; the pages
+    give neither the placement nor eps).  YaRN scaling (§3.1.4) is not
+    applied.
 
 Weights use the pages' shapes W in R^{out x in} with y = W x.  Head i owns rows
 [i d_h, (i+1) d_h) of W^{UQ}, W^{UK}, W^{UV}, rows [i d_R, (i+1) d_R) of W^{QR}
@@ -41,7 +45,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "rope", "latent_rows", "queries", "keys_values", "softmax", "attend",
+    "rope", "rmsnorm", "RMS_EPS", "latent_rows", "queries", "keys_values", "softmax", "attend",
     "decode_unabsorbed", "decode_absorbed", "prefill_unabsorbed",
     "round_bf16_f64", "cache_row_elems",
 ]
@@ -76,22 +80,38 @@ def rope(x, pos, base: float):
     return out
 
 
+RMS_EPS = 1e-6
+
+
+def rmsnorm(x, g, eps=None):
+    """x / sqrt(mean(x^2) + eps) * g over the last axis."""
+    x = _f64(x)
+    eps = RMS_EPS if eps is None else eps
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * _f64(g)
+
+
 def latent_rows(W: dict, h, pos, dims):
     """The cached vectors of tokens h [T, d] at positions pos [T].
 
-    Returns (c_kv [T, d_c], k_r [T, d_R]): c^KV = W^{DKV} h, k^R = RoPE(W^{KR} h).
+    Returns (c_kv [T, d_c], k_r [T, d_R]): c^KV = W^{DKV} h (RMS-normalised
+    with gains W["g_kv"] when present), k^R = RoPE(W^{KR} h).
     """
     h = _f64(h)
     c_kv = h @ _f64(W["W_DKV"]).T
+    if "g_kv" in W:
+        c_kv = rmsnorm(c_kv, W["g_kv"])
     k_r = rope(h @ _f64(W["W_KR"]).T, pos, dims.rope_base)
     return c_kv, k_r
 
 
 def queries(W: dict, h, pos, dims):
-    """Per-head query parts: q^C [T, n_h, d_h] and q^R [T, n_h, d_R]."""
+    """Per-head query parts: q^C [T, n_h, d_h] and q^R [T, n_h, d_R] (c^Q
+    RMS-normalised with gains W["g_q"] when present)."""
     h = _f64(h)
     T = h.shape[0]
     c_q = h @ _f64(W["W_DQ"]).T if dims.d_cq else h
+    if dims.d_cq and "g_q" in W:
+        c_q = rmsnorm(c_q, W["g_q"])
     q_c = (c_q @ _f64(W["W_UQ"]).T).reshape(T, dims.n_h, dims.d_h)
     q_r = rope((c_q @ _f64(W["W_QR"]).T).reshape(T, dims.n_h, dims.d_R),
                _f64(pos)[:, None], dims.rope_base)
