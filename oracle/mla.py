@@ -33,8 +33,13 @@ design notes of this repository):
     only when the weights carry its gains: "g_kv" [d_c] normalises c^KV
     before it is cached, and "g_q" [d_cq] normalises c^Q before the
     up-projections (RMS over the latent's own width, eps = RMS_EPS; the pages
-    give neither the placement nor eps).  YaRN scaling (§3.1.4) is not
-    applied.
+    give neither the placement nor eps).
+  * YaRN (§3.1.4) is not part of App. C either.  It is applied only when
+    dims carries `yarn` = (s, alpha, beta, L0): the rotary frequencies of q^R
+    and k^R ramp from theta/s to theta as L0 holds between alpha and beta of
+    their wavelengths (the published YaRN rule; the pages give s = 40,
+    alpha = 1, beta = 32 and the 4K pre-training length), and every score is
+    multiplied by t with sqrt(t) = 0.0707 ln s + 1.
 
 Weights use the pages' shapes W in R^{out x in} with y = W x.  Head i owns rows
 [i d_h, (i+1) d_h) of W^{UQ}, W^{UK}, W^{UV}, rows [i d_R, (i+1) d_R) of W^{QR}
@@ -45,7 +50,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "rope", "rmsnorm", "RMS_EPS", "latent_rows", "queries", "keys_values", "softmax", "attend",
+    "rope", "yarn_theta", "yarn_score_factor", "score_scale", "rmsnorm", "RMS_EPS", "latent_rows", "queries", "keys_values", "softmax", "attend",
     "decode_unabsorbed", "decode_absorbed", "prefill_unabsorbed",
     "round_bf16_f64", "cache_row_elems",
 ]
@@ -60,17 +65,20 @@ def cache_row_elems(d_c: int, d_R: int) -> int:
     return d_c + d_R
 
 
-def rope(x, pos, base: float):
+def rope(x, pos, base: float, theta=None):
     """Rotary position embedding on the last axis (width d_R, even).
 
-    Pair m = (x[2m], x[2m+1]) is rotated by phi = pos * base^(-2m/d_R):
+    Pair m = (x[2m], x[2m+1]) is rotated by phi = pos * theta_m with
+    theta_m = base^(-2m/d_R) unless `theta` gives the frequencies:
     (a, b) -> (a cos phi - b sin phi, a sin phi + b cos phi).
     `pos` broadcasts against x's leading axes.
     """
     x = _f64(x)
     d_R = x.shape[-1]
-    m = np.arange(d_R // 2, dtype=np.float64)
-    theta = np.power(float(base), -2.0 * m / d_R)
+    if theta is None:
+        m = np.arange(d_R // 2, dtype=np.float64)
+        theta = np.power(float(base), -2.0 * m / d_R)
+    theta = _f64(theta)
     phi = _f64(pos)[..., None] * theta
     c, s = np.cos(phi), np.sin(phi)
     a, b = x[..., 0::2], x[..., 1::2]
@@ -78,6 +86,38 @@ def rope(x, pos, base: float):
     out[..., 0::2] = a * c - b * s
     out[..., 1::2] = a * s + b * c
     return out
+
+
+def yarn_theta(d_R: int, base: float, yarn):
+    """YaRN rotary frequencies for yarn = (s, alpha, beta, L0).
+
+    Pair m keeps theta_m = base^(-2m/d_R) when the pre-training length L0
+    spans more than beta of its wavelengths 2 pi / theta_m, takes theta_m / s
+    (position interpolation) below alpha of them, and ramps linearly in
+    between.
+    """
+    s, alpha, beta, L0 = yarn
+    m = np.arange(d_R // 2, dtype=np.float64)
+    theta = np.power(float(base), -2.0 * m / d_R)
+    r = L0 * theta / (2.0 * np.pi)            # wavelengths inside L0
+    ramp = np.clip((r - alpha) / (beta - alpha), 0.0, 1.0)
+    return (1.0 - ramp) * theta / s + ramp * theta
+
+
+def yarn_score_factor(s: float) -> float:
+    """t with sqrt(t) = 0.0707 ln s + 1, the factor on every attention score."""
+    return (0.0707 * np.log(s) + 1.0) ** 2
+
+
+def _theta(dims):
+    y = getattr(dims, "yarn", None)
+    return None if y is None else yarn_theta(dims.d_R, dims.rope_base, y)
+
+
+def score_scale(dims) -> float:
+    """Softmax scale: 1/sqrt(d_h + d_R), times YaRN's t when dims carries yarn."""
+    y = getattr(dims, "yarn", None)
+    return (1.0 if y is None else yarn_score_factor(y[0])) / np.sqrt(dims.d_h + dims.d_R)
 
 
 RMS_EPS = 1e-6
@@ -100,7 +140,7 @@ def latent_rows(W: dict, h, pos, dims):
     c_kv = h @ _f64(W["W_DKV"]).T
     if "g_kv" in W:
         c_kv = rmsnorm(c_kv, W["g_kv"])
-    k_r = rope(h @ _f64(W["W_KR"]).T, pos, dims.rope_base)
+    k_r = rope(h @ _f64(W["W_KR"]).T, pos, dims.rope_base, _theta(dims))
     return c_kv, k_r
 
 
@@ -114,7 +154,7 @@ def queries(W: dict, h, pos, dims):
         c_q = rmsnorm(c_q, W["g_q"])
     q_c = (c_q @ _f64(W["W_UQ"]).T).reshape(T, dims.n_h, dims.d_h)
     q_r = rope((c_q @ _f64(W["W_QR"]).T).reshape(T, dims.n_h, dims.d_R),
-               _f64(pos)[:, None], dims.rope_base)
+               _f64(pos)[:, None], dims.rope_base, _theta(dims))
     return q_c, q_r
 
 
@@ -169,7 +209,7 @@ def decode_unabsorbed(W: dict, h_seq, dims, cache_rows=None):
     k, v = keys_values(W, c_kv, k_r, dims)
     q_c, q_r = queries(W, h_seq[-1:], pos[-1:], dims)
     q = np.concatenate([q_c[0], q_r[0]], axis=-1)
-    o, _ = attend(q, k, v, 1.0 / np.sqrt(dims.d_h + dims.d_R))
+    o, _ = attend(q, k, v, score_scale(dims))
     return _output(W, o, dims)
 
 
@@ -191,7 +231,7 @@ def decode_absorbed(W: dict, h_seq, dims, return_parts=False):
     q_abs = np.einsum("hdc,hd->hc", W_UK, q_c[0])                      # [n_h, d_c]
     q_lat = np.concatenate([q_abs, q_r[0]], axis=-1)                   # [n_h, d_c + d_R]
     rows = np.concatenate([c_kv, k_r], axis=-1)                        # [L+1, d_c + d_R]
-    s = (q_lat @ rows.T) / np.sqrt(dims.d_h + dims.d_R)                # [n_h, L+1]
+    s = (q_lat @ rows.T) * score_scale(dims)                          # [n_h, L+1]
     p = softmax(s, axis=-1)
     o_lat = p @ c_kv                                                   # [n_h, d_c]
     o = np.einsum("hdc,hc->hd", W_UV, o_lat)                           # [n_h, d_h]
@@ -219,7 +259,7 @@ def prefill_unabsorbed(W: dict, h, dims, start_pos: int = 0, h_prefix=None, rows
     rows = list(range(T)) if rows is None else [int(r) for r in rows]
     q_c, q_r = queries(W, h[rows], pos_all[start_pos:][rows], dims)
     q = np.concatenate([q_c, q_r], axis=-1)                            # [len(rows), n_h, dq]
-    scale = 1.0 / np.sqrt(dims.d_h + dims.d_R)
+    scale = score_scale(dims)
     u = np.empty((len(rows), dims.d_model), dtype=np.float64)
     for i, t in enumerate(rows):
         n = start_pos + t + 1

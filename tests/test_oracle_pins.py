@@ -252,7 +252,7 @@ def test_hidden_subset_regenerates():
 _ORIG_ROPE = om.rope
 
 
-def _rope_half_split(x, pos, base):
+def _rope_half_split(x, pos, base, theta=None):
     x = np.asarray(x, dtype=np.float64)
     d = x.shape[-1]
     perm = np.concatenate([np.arange(0, d, 2), np.arange(1, d, 2)])
@@ -260,7 +260,7 @@ def _rope_half_split(x, pos, base):
     xi = np.empty_like(x)
     xi[..., 0::2] = x[..., : d // 2]
     xi[..., 1::2] = x[..., d // 2:]
-    y = _ORIG_ROPE(xi, pos, base)
+    y = _ORIG_ROPE(xi, pos, base, theta)
     out = np.empty_like(y)
     out[..., : d // 2] = y[..., 0::2]
     out[..., d // 2:] = y[..., 1::2]
@@ -268,9 +268,9 @@ def _rope_half_split(x, pos, base):
 
 
 MUTANTS = {
-    "rope_direction": ("rope", lambda x, pos, base: _ORIG_ROPE(x, -np.asarray(pos, dtype=np.float64), base)),
+    "rope_direction": ("rope", lambda x, pos, base, theta=None: _ORIG_ROPE(x, -np.asarray(pos, dtype=np.float64), base, theta)),
     "rope_half_split": ("rope", _rope_half_split),
-    "rope_frequency": ("rope", lambda x, pos, base: _ORIG_ROPE(x, pos, base * 2)),
+    "rope_frequency": ("rope", lambda x, pos, base, theta=None: _ORIG_ROPE(x, pos, base * 2, theta)),
     "scale_dh_only": ("attend", lambda q, k, v, scale: _ORIG_ATTEND(q, k, v, scale * math.sqrt((4 + 4) / 4))),
     "no_rope_key": ("keys_values", lambda W, c, kr, dims: _ORIG_KV(W, c, kr * 0, dims)),
     "uk_row_order": ("keys_values", lambda W, c, kr, dims: _ORIG_KV(
