@@ -6,7 +6,9 @@ d_R=64, d_c=512, d_c'=1536), batch 64, 8192 cached tokens per sequence plus
 one new token each, bf16 storage.  One step = one mla_decode call: the new
 tokens' down-projections and cache append, the query up-projection, W_UK
 absorption, attention over the latent cache, split combine, W_UV and W_O.
-Also reported: the causal prefill of 16384 tokens at the same dims.
+Also reported in the same line: the causal prefill of 16384 tokens at the same
+dims, and the V2-Lite (batch 32, 4096 cached tokens) and ragged long-context
+(batch 128, seeded log-uniform lengths) decode workloads.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -44,6 +46,7 @@ def parse():
     ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling cases)")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the V2-Lite and ragged decode objects")
     ap.add_argument("--profile", action="store_true",
                     help="decode steps only (no clock sampling, e2e, prefill or CPU baseline): for ncu captures")
     return ap.parse_args()
@@ -221,6 +224,23 @@ def job_throughput(world, units_per_rank, ms_per_step):
 
 
 # ============================================================================ reference arm
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def reference_sample(p, L, n=2, max_tokens=16384):
+    """Sequences of the workload the oracle steps cycle over: the first `n`
+    whose cache fits `max_tokens` (all of them at the uniform workloads)."""
+    picks = [b for b in range(len(L)) if L[b] + 1 <= max_tokens][:n]
+    return picks or [int(min(range(len(L)), key=lambda b: L[b]))]
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -230,12 +250,12 @@ def run_reference(args):
     from oracle import mla as om
     p, L = workload_lengths(args.workload, args.ctx, args.batch)
     Wh = synth.weights(p)
-    hs = {}
+    picks = reference_sample(p, L)
+    # inputs are drawn before the timed region: the steps time the oracle alone
+    hs = {b: synth.hidden(p, b, L[b] + 1) for b in picks}
 
     def step(i):
-        b = i % len(L)
-        if b not in hs:
-            hs[b] = synth.hidden(p, b, L[b] + 1)
+        b = picks[i % len(picks)]
         u = om.decode_unabsorbed(Wh, hs[b], p.dims)
         assert np.all(np.isfinite(u))
 
@@ -247,13 +267,15 @@ def run_reference(args):
     dt = (time.perf_counter() - t0) / args.steps
     value = 1.0 / dt  # one new token per step (one sequence of the batch)
     cores = blas_threads()
-    sample = f"{args.steps} steps, each the fp64 un-absorbed oracle on one whole sequence of the {args.workload} workload ({L[0] + 1} tokens)"
+    sample = (f"{args.steps} steps, each the fp64 un-absorbed oracle on one whole sequence of the {args.workload} "
+              f"workload (sequences {picks}, {[L[b] + 1 for b in picks]} tokens), inputs drawn before timing")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(args, args.gpus),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "cpu_model": cpu_model(),
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -261,6 +283,87 @@ def run_reference(args):
 
 
 # ============================================================================ our arm
+class DecodeSetup:
+    """Seeded synthetic decode workload resident on the device: random
+    N(0,0.02) bf16 weights, a latent cache filled through mla_cache_append
+    from N(0,1) hidden states, the new tokens' hidden states and seqlen."""
+
+    def __init__(self, m, dev, g, name, ctx=0, batch=0):
+        import torch
+        from mla_latent_kv_47_b200.cache import LatentCache
+        from synth import weight_shapes
+        self.m = m
+        self.p, self.L = workload_lengths(name, ctx, batch)
+        d = self.p.dims
+        self.dims = m.make_dims(d)
+        self.B = len(self.L)
+        self.Wd = {k: (torch.randn(s, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+                   for k, s in weight_shapes(d).items()}
+        self.wts = m.make_weights(self.Wd)
+        self.cache = LatentCache(self.dims, [x + 1 for x in self.L], device=dev)
+        self.ws = m.alloc_workspace(self.dims, self.B, 1, device=dev)
+        chunk = 16384
+        for b, n in enumerate(self.L):
+            for t0 in range(0, n, chunk):
+                k = min(chunk, n - t0)
+                h = torch.randn((k, d.d_model), generator=g, device=dev).to(torch.bfloat16)
+                m.cache_append(self.dims, self.wts, h, torch.full((k,), b, dtype=torch.int32, device=dev),
+                               torch.arange(t0, t0 + k, dtype=torch.int32, device=dev), self.cache.handle, self.ws)
+        self.h_new = torch.randn((self.B, d.d_model), generator=g, device=dev).to(torch.bfloat16)
+        self.seqlen = torch.tensor(self.L, dtype=torch.int32, device=dev)
+        self.u = torch.empty((self.B, d.d_model), dtype=torch.float32, device=dev)
+        torch.cuda.synchronize()
+        code, detail = m.device_status(self.ws)
+        assert code == 0, ("cache fill fault", code, detail)
+
+    def step(self):
+        self.m.decode(self.dims, self.wts, self.h_new, self.cache.handle, self.seqlen, self.u, self.ws)
+
+    def check(self):
+        code, detail = self.m.device_status(self.ws)
+        assert code == 0, ("decode fault", code, detail)
+
+
+def time_steps(m, step, K, barrier, ev_attn=True):
+    """K steps between CUDA events on the current stream, after a barrier and
+    a synchronize; the attention kernel of every step is bracketed by its own
+    events.  Returns (ms per step, mean attention ms, launches in the region)."""
+    import torch
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for e in ev_b + ev_e:  # torch creates the CUDA event on its first record
+        e.record()
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = m.kernel_launches()
+    t_start.record()
+    for i in range(K):
+        if ev_attn:
+            m.set_attention_events(ev_b[i], ev_e[i])
+        step()
+    t_end.record()
+    launches = m.kernel_launches() - launches0
+    torch.cuda.synchronize()
+    m.set_attention_events(None, None)
+    ms = t_start.elapsed_time(t_end) / K
+    attn = statistics.mean(ev_b[i].elapsed_time(ev_e[i]) for i in range(K)) if ev_attn else None
+    return ms, attn, launches
+
+
+def decode_summary(d, L, ms, attn_ms, world, hbm_gbs, bf16_tf):
+    """Throughput and roofline fractions of one decode workload."""
+    flops, bytes_total, cache_bytes, attn_flops = decode_flops_bytes(d, L)
+    roof_ms = max(bytes_total / (hbm_gbs * 1e9), flops / (bf16_tf * 1e12)) * 1e3
+    attn_roof_ms = max(cache_bytes / (hbm_gbs * 1e9), attn_flops / (bf16_tf * 1e12)) * 1e3
+    return {
+        "tokens_per_s": world * len(L) / (ms * 1e-3), "ms": ms, "batch": len(L), "cached_tokens": sum(L),
+        "attn_ms": attn_ms, "latent_cache_gbs": cache_bytes / (attn_ms * 1e-3) / 1e9,
+        "attn_roofline_frac": attn_roof_ms / attn_ms,
+        "step_roofline": {"bytes": bytes_total, "flops": flops, "roofline_ms": roof_ms, "frac": roof_ms / ms},
+    }
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -279,36 +382,7 @@ def run_ours(args):
     import mla_latent_kv_47_b200 as m
     from mla_latent_kv_47_b200.cache import LatentCache
 
-    p, L = workload_lengths(args.workload, args.ctx, args.batch)
-    d = p.dims
-    dims = m.make_dims(d)
-    B = len(L)
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = peaks()
-
-    # ---- inputs: seeded, synthetic, resident in HBM before timing
-    g = torch.Generator(device=dev)
-    g.manual_seed(1000 + rank)
-    from synth import weight_shapes
-    Wd = {k: (torch.randn(s, generator=g, device=dev) * 0.02).to(torch.bfloat16) for k, s in weight_shapes(d).items()}
-    wts = m.make_weights(Wd)
-    cache = LatentCache(dims, [x + 1 for x in L], device=dev)
-    chunk = 16384
-    ws = m.alloc_workspace(dims, B, 1, device=dev)
-    for b, n in enumerate(L):
-        for t0 in range(0, n, chunk):
-            k = min(chunk, n - t0)
-            h = torch.randn((k, d.d_model), generator=g, device=dev).to(torch.bfloat16)
-            m.cache_append(dims, wts, h, torch.full((k,), b, dtype=torch.int32, device=dev),
-                           torch.arange(t0, t0 + k, dtype=torch.int32, device=dev), cache.handle, ws)
-    h_new = torch.randn((B, d.d_model), generator=g, device=dev).to(torch.bfloat16)
-    seqlen = torch.tensor(L, dtype=torch.int32, device=dev)
-    u = torch.empty((B, d.d_model), dtype=torch.float32, device=dev)
-    torch.cuda.synchronize()
-    code, detail = m.device_status(ws)
-    assert code == 0, ("cache fill fault", code, detail)
-
-    def step():
-        m.decode(dims, wts, h_new, cache.handle, seqlen, u, ws)
 
     def barrier():
         if world > 1:
@@ -317,50 +391,42 @@ def run_ours(args):
     def max_over_ranks(x):
         return reduce_max(x, world, dev)
 
+    # ---- inputs: seeded, synthetic, resident in HBM before timing
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 + rank)
+    S = DecodeSetup(m, dev, g, args.workload, args.ctx, args.batch)
+    d, L, B = S.p.dims, S.L, S.B
+
     for _ in range(max(args.warmup, 3)):
-        step()
+        S.step()
     torch.cuda.synchronize()
     K = args.steps
-    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for e in ev_b + ev_e:  # torch creates the CUDA event on its first record
-        e.record()
-    barrier()
-    torch.cuda.synchronize()
     with ClockSampler(dev.index) as clk:
         # keep the GPU busy while the sampler starts, so its samples see load
         t0 = time.perf_counter()
         while not args.profile and time.perf_counter() - t0 < 0.5:
             for _ in range(20):
-                step()
+                S.step()
             torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
-        launches0 = m.kernel_launches()
-        t_start.record()
-        for i in range(K):
-            m.set_attention_events(ev_b[i], ev_e[i])
-            step()
-        t_end.record()
-        launches = m.kernel_launches() - launches0
-        torch.cuda.synchronize()
-    m.set_attention_events(None, None)
+        launches_before = m.kernel_launches()
+        ms, attn_ms, launches = time_steps(m, S.step, K, barrier)
     barrier()
-    ms = max_over_ranks(t_start.elapsed_time(t_end) / K)
-    attn_ms = max_over_ranks(statistics.mean(ev_b[i].elapsed_time(ev_e[i]) for i in range(K)))
-    code, detail = m.device_status(ws)
-    assert code == 0, ("decode fault", code, detail)
+    ms = max_over_ranks(ms)
+    attn_ms = max_over_ranks(attn_ms)
+    S.check()
 
     if args.profile:
         print(json.dumps({"profile_run": True, "ms_per_step": ms, "attn_ms": attn_ms,
-                          "launches_before_timing": launches0, "launches_per_step": launches // K}), flush=True)
+                          "launches_before_timing": launches_before, "launches_per_step": launches // K}),
+              flush=True)
         return 0
     # ---- end to end: host (pinned) inputs in, host output back, every step
-    h_host = h_new.cpu().pin_memory()
-    sl_host = seqlen.cpu().pin_memory()
+    h_host = S.h_new.cpu().pin_memory()
+    sl_host = S.seqlen.cpu().pin_memory()
     u_host = torch.empty((B, d.d_model), dtype=torch.float32).pin_memory()
-    h_dev, sl_dev = torch.empty_like(h_new), torch.empty_like(seqlen)
+    h_dev, sl_dev = torch.empty_like(S.h_new), torch.empty_like(S.seqlen)
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -368,50 +434,41 @@ def run_ours(args):
     for _ in range(K):
         h_dev.copy_(h_host, non_blocking=True)
         sl_dev.copy_(sl_host, non_blocking=True)
-        m.decode(dims, wts, h_dev, cache.handle, sl_dev, u, ws)
-        u_host.copy_(u, non_blocking=True)
+        m.decode(S.dims, S.wts, h_dev, S.cache.handle, sl_dev, S.u, S.ws)
+        u_host.copy_(S.u, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / K)
     h2d = h_host.numel() * h_host.element_size() + sl_host.numel() * 4
     d2h = u_host.numel() * 4
+    S.check()
 
-    flops, bytes_total, cache_bytes, attn_flops = decode_flops_bytes(d, L)
-    attn_gbs = cache_bytes / (attn_ms * 1e-3) / 1e9
-    roof_ms = max(bytes_total / (hbm_gbs * 1e9), flops / (bf16_tf * 1e12)) * 1e3
+    main = decode_summary(d, L, ms, attn_ms, world, hbm_gbs, bf16_tf)
+    cache_bytes = decode_flops_bytes(d, L)[2]
+    del S
+    torch.cuda.empty_cache()
 
-    # ---- prefill (secondary): 16384 tokens at the same dims
+    # ---- prefill (secondary): 16384 tokens at the DeepSeek-V2 dims
     prefill = None
     if not args.no_prefill and args.workload == "v2":
         import synth
+        from synth import weight_shapes
         T = synth.preset("prefill").prefill_T
-        del cache
-        torch.cuda.empty_cache()
+        Wd = {k: (torch.randn(s, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+              for k, s in weight_shapes(d).items()}
+        wts = m.make_weights(Wd)
+        dims = m.make_dims(d)
         pc = LatentCache(dims, [T], device=dev)
         wsp = m.alloc_workspace(dims, 1, T, device=dev)
         hp = torch.randn((T, d.d_model), generator=g, device=dev).to(torch.bfloat16)
         up = torch.empty((T, d.d_model), dtype=torch.float32, device=dev)
-        m.prefill(dims, wts, hp, 0, pc.handle, 0, up, wsp)
-        torch.cuda.synchronize()
-        KP = 2
-        pb = [torch.cuda.Event(enable_timing=True) for _ in range(KP)]
-        pe = [torch.cuda.Event(enable_timing=True) for _ in range(KP)]
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        for e in pb + pe:
-            e.record()
-        barrier()
-        torch.cuda.synchronize()
-        s0.record()
-        for i in range(KP):
-            m.set_attention_events(pb[i], pe[i])
+        for _ in range(3):
             m.prefill(dims, wts, hp, 0, pc.handle, 0, up, wsp)
-        s1.record()
         torch.cuda.synchronize()
-        m.set_attention_events(None, None)
-        barrier()
-        pms = max_over_ranks(s0.elapsed_time(s1) / KP)
-        pattn = max_over_ranks(statistics.mean(pb[i].elapsed_time(pe[i]) for i in range(KP)))
+        KP = 3
+        pms, pattn, _ = time_steps(m, lambda: m.prefill(dims, wts, hp, 0, pc.handle, 0, up, wsp), KP, barrier)
+        pms, pattn = max_over_ranks(pms), max_over_ranks(pattn)
         pf, pattn_flops = prefill_flops(d, T)
         assert m.device_status(wsp)[0] == 0
         prefill = {
@@ -421,6 +478,25 @@ def run_ours(args):
             "attention": {"ms": pattn, "tflops": pattn_flops / (pattn * 1e-3) / 1e12,
                           "frac": pattn_flops / (pattn * 1e-3) / 1e12 / bf16_tf},
         }
+        del pc, wsp, hp, up, Wd
+        torch.cuda.empty_cache()
+
+    # ---- the other decode workloads (secondary objects of the same line)
+    others = {}
+    if args.workload == "v2" and not args.ctx and not args.batch and not args.no_secondary:
+        for name in ("lite", "ragged"):
+            So = DecodeSetup(m, dev, g, name)
+            for _ in range(5):
+                So.step()
+            torch.cuda.synchronize()
+            K2 = max(10, min(K, 200))
+            oms, oattn, _ = time_steps(m, So.step, K2, barrier)
+            So.check()
+            others[name] = decode_summary(So.p.dims, So.L, max_over_ranks(oms), max_over_ranks(oattn), world,
+                                          hbm_gbs, bf16_tf)
+            others[name]["steps"] = K2
+            del So
+            torch.cuda.empty_cache()
 
     if rank != 0:
         if world > 1:
@@ -431,11 +507,12 @@ def run_ours(args):
     if world == 1 and not args.no_cpu_baseline:
         times, pp = oracle_decode_seconds(args.workload)
         cpu_baseline = {"value": len(times) / sum(times), "unit": "tokens/s", "cores": blas_threads(),
-                        "kind": "oracle",
+                        "cpu_model": cpu_model(), "kind": "oracle",
                         "sample": f"{len(times)} whole sequences of the {args.workload} workload "
                                   f"({pp.seqlen[0] + 1} tokens each) through the fp64 un-absorbed oracle"}
 
     traffic = traffic_record(ATTN_SOURCES)
+    attn_gbs = cache_bytes / (attn_ms * 1e-3) / 1e9
     value = job_throughput(world, B, ms)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
@@ -446,14 +523,15 @@ def run_ours(args):
                      "frac": attn_gbs / hbm_gbs, "traffic": traffic,
                      "kernel": "decode attention (latent-cache stream)",
                      "peak_source": peak_src, "attn_ms": attn_ms},
-        "step_roofline": {"bytes": bytes_total, "flops": flops, "roofline_ms": roof_ms,
-                          "frac": roof_ms / ms, "latent_cache_gbs": cache_bytes / (ms * 1e-3) / 1e9},
+        "step_roofline": dict(main["step_roofline"], latent_cache_gbs=cache_bytes / (ms * 1e-3) / 1e9),
         "e2e": {"value": world * B / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches,
         "clocks": clk.summary(),
         "cpu_baseline": cpu_baseline,
         "prefill": prefill,
+        "lite": others.get("lite"),
+        "ragged": others.get("ragged"),
     }
     print(json.dumps(line), flush=True)
     if world > 1:

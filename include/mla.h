@@ -33,6 +33,13 @@
  *    calls (apart from the diagnostic timing hook at the end of this file).
  *    Work is enqueued on `stream` and the calls return without synchronising.
  *  - Every device pointer must be 16-byte aligned (TMA requirement).
+ *  - Supported shapes.  bf16 storage runs on the tensor-core kernels, which
+ *    are built for the DeepSeek-V2 head shape: d_h = 128, d_R = 64,
+ *    d_c = 512, n_h <= 128, d_model and d_cq multiples of 64 (this covers
+ *    DeepSeek-V2 and DeepSeek-V2-Lite).  fp32 storage runs on CUDA-core
+ *    kernels for small layers: d_c <= 512 (a multiple of 4), d_h <= 256,
+ *    d_R even, 16-byte rows.  Anything else returns MLA_ERR_UNSUPPORTED
+ *    with nothing enqueued; no call switches to another kernel family.
  *  - Errors in arguments, shapes, alignment or workspace size are found on the
  *    host and returned before anything is enqueued.  Faults found on the
  *    device (a position at or beyond `capacity`, a pipeline wait that timed
@@ -174,8 +181,10 @@ size_t mla_workspace_offset(const mla_dims* dims, int max_batch, int max_tokens,
  *    larger batches.  A batch that does not fit returns MLA_ERR_WORKSPACE with
  *    nothing enqueued.
  *  - The first call on a device looks up the array's device address (once per
- *    device, with that device current).  Make that first call outside any
- *    stream capture.
+ *    device, with that device current) and keeps it for the life of the
+ *    process.  Make that first call outside any stream capture, and do not
+ *    reset the device (cudaDeviceReset) between calls: the kept address
+ *    would no longer be mapped.
  *  - All calls share the one array, and it keeps the previous call's contents;
  *    each call clears what must start at zero.  Calls whose work overlaps on the
  *    GPU (several streams or host threads) race on the array.

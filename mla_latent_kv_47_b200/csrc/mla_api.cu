@@ -24,9 +24,10 @@ constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Workspace: [status | split-K tickets | split-K partials] followed by ONE of
-// the decode region (sized by the batch) or the prefill region (sized by the
-// number of key tokens); a call uses only its own region.
+// Workspace: [status | split-K partials] followed by ONE of the decode region
+// (sized by the batch) or the prefill region (sized by the number of key
+// tokens); a call uses only its own region.  Apart from the status word, every
+// region is written in full by a kernel of the call before any kernel reads it.
 struct Layout {
   size_t status, gpart, base_end;
   size_t tile_start, seg_start, rope, cq, qc, qlat, olat, o, opart, ml, decode_end;
@@ -160,6 +161,23 @@ mla_status launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+constexpr int kMaxDevices = 64;
+
+// Raises a kernel's dynamic shared-memory limit on the current device.  The
+// attribute belongs to the device's context, so it is set once per device
+// (bit `dev` of `done`); devices beyond 64 set it on every call.
+template <typename Kern>
+mla_status set_smem_limit(Kern kern, int smem, std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  const unsigned long long bit = dev >= 0 && dev < kMaxDevices ? 1ull << dev : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return MLA_OK;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return MLA_OK;
+}
+
 // Tile width, pipeline depth, K blocks per stage, CTA target and 128-row tiles
 // per CTA (per-head modes) of one GEMM launch.
 struct GemmConfig {
@@ -170,12 +188,9 @@ template <int BN, bool AMN, int STAGES, int KBB, int MT = 1>
 mla_status launch_tc(const GemmArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
   constexpr int smem = GemmSmem<BN, STAGES, KBB, MT>::kBytes;
   auto kern = gemm_tc_kernel<BN, AMN, STAGES, KBB, MT>;
-  static bool attr_set = false;  // idempotent attribute set; races are harmless
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return MLA_ERR_CUDA;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  const mla_status s = set_smem_limit(kern, smem, attr_done);
+  if (s != MLA_OK) return s;
   return launch(kern, grid, dim3(192), smem, st, pdl, a);
 }
 
@@ -335,7 +350,8 @@ mla_status run_gemm(const Ctx& c, const GemmSpec& g) {
     if (g.mode != GEMM_DENSE && g.N <= 64 && g.rows[0] % 512 == 0) cfg = {64, 2, 1, c.num_sms, 4};
     return run_gemm_tc(c, g, cfg);
   }
-  return c.d.dtype == MLA_FP32 ? run_gemm_simt<float>(c, g) : run_gemm_simt<__nv_bfloat16>(c, g);
+  // fp32 storage (check_dims admits bf16 only with tensor-core shapes)
+  return c.d.dtype == MLA_FP32 ? run_gemm_simt<float>(c, g) : MLA_ERR_UNSUPPORTED;
 }
 
 // ------------------------------------------------------------------ checks
@@ -353,6 +369,12 @@ mla_status check_dims(const mla_dims* d) {
   // 16-byte rows for every tensor the kernels load
   const int es = d->dtype == MLA_FP32 ? 4 : 2;
   if ((row_elems(*d) * es) % 16 || (d->d_model * es) % 16 || (d->d_c * es) % 16) return MLA_ERR_UNSUPPORTED;
+  // bf16 storage runs on the tensor-core kernels only, which are built for the
+  // DeepSeek-V2 head shape (d_h = 128, d_R = 64, d_c = 512, up to 128 heads)
+  // and 64-wide K blocks; the CUDA-core kernels serve fp32 storage alone.
+  if (d->dtype == MLA_BF16 &&
+      (d->d_h != 128 || d->d_R != 64 || d->d_c != 512 || d->n_h > 128 || d->d_model % 64 != 0 || d->d_cq % 64 != 0))
+    return MLA_ERR_UNSUPPORTED;
   return MLA_OK;
 }
 
@@ -484,13 +506,9 @@ mla_status launch_attn_decode_tc(const __nv_bfloat16* qlat, const mla_cache* cac
   a.o_part = o_part;
   a.ml_part = ml;
   a.status = status;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, attn::kSmem) !=
-        cudaSuccess)
-      return MLA_ERR_CUDA;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  const mla_status s = set_smem_limit(attn_decode_tc_kernel, attn::kSmem, attr_done);
+  if (s != MLA_OK) return s;
   return launch(attn_decode_tc_kernel, dim3(2 * W), dim3(attn::kThreads), attn::kSmem, st, pdl, a);
 }
 
@@ -618,17 +636,13 @@ mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const 
                                    B, W, d.n_h, opart, ml, c.status, c.st, c.pdl)) != MLA_OK)
       return s;
   } else {
+    if (d.dtype != MLA_FP32) return MLA_ERR_UNSUPPORTED;  // bf16 is on the tensor-core kernel alone
     const size_t shm = (row + 4 * d.d_c + 8) * sizeof(float);
     dim3 grid(W, d.n_h);
     g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
-    if (d.dtype == MLA_FP32)
-      simt_decode_attn_kernel<float><<<grid, 128, shm, c.st>>>(
-          static_cast<const float*>(qlat), static_cast<const float*>(cache->base), cache->seq_start, seqlen,
-          tile_start, seg_start, B, W, d.n_h, d.d_c, d.d_R, tile_tokens, opart, ml);
-    else
-      simt_decode_attn_kernel<__nv_bfloat16><<<grid, 128, shm, c.st>>>(
-          static_cast<const __nv_bfloat16*>(qlat), static_cast<const __nv_bfloat16*>(cache->base), cache->seq_start,
-          seqlen, tile_start, seg_start, B, W, d.n_h, d.d_c, d.d_R, tile_tokens, opart, ml);
+    simt_decode_attn_kernel<float><<<grid, 128, shm, c.st>>>(
+        static_cast<const float*>(qlat), static_cast<const float*>(cache->base), cache->seq_start, seqlen,
+        tile_start, seg_start, B, W, d.n_h, d.d_c, d.d_R, tile_tokens, opart, ml);
     if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
   }
   attn_event(g_attn_end, c.st);
@@ -920,29 +934,19 @@ extern "C" mla_status mla_prefill(const mla_dims* dims, const mla_weights* w, co
     a.n_h = d.n_h;
     a.n_qt = (T + pf::kQ - 1) / pf::kQ;
     a.status = c.status;
-    static bool attr_set = false;
-    if (!attr_set) {
-      if (cudaFuncSetAttribute(attn_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pf::kSmem) !=
-          cudaSuccess)
-        return MLA_ERR_CUDA;
-      attr_set = true;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    if ((s = set_smem_limit(attn_prefill_tc_kernel, pf::kSmem, attr_done)) != MLA_OK) return s;
     g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
     attn_prefill_tc_kernel<<<dim3(a.n_qt, d.n_h), 192, pf::kSmem, c.st>>>(a);
     if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
   } else {
+    if (d.dtype != MLA_FP32) return MLA_ERR_UNSUPPORTED;  // bf16 is on the tensor-core kernel alone
     const size_t shm = (dq + 4 * d.d_h + 8) * sizeof(float);
     dim3 grid(T, d.n_h);
     g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
-    if (d.dtype == MLA_FP32)
-      simt_prefill_attn_kernel<float><<<grid, 128, shm, c.st>>>(
-          static_cast<const float*>(qp), static_cast<const float*>(kc), static_cast<const float*>(vv),
-          static_cast<const float*>(rows), T, start_pos, d.n_h, d.d_h, d.d_R, d.d_c, static_cast<float*>(att));
-    else
-      simt_prefill_attn_kernel<__nv_bfloat16><<<grid, 128, shm, c.st>>>(
-          static_cast<const __nv_bfloat16*>(qp), static_cast<const __nv_bfloat16*>(kc),
-          static_cast<const __nv_bfloat16*>(vv), static_cast<const __nv_bfloat16*>(rows), T, start_pos, d.n_h,
-          d.d_h, d.d_R, d.d_c, static_cast<__nv_bfloat16*>(att));
+    simt_prefill_attn_kernel<float><<<grid, 128, shm, c.st>>>(
+        static_cast<const float*>(qp), static_cast<const float*>(kc), static_cast<const float*>(vv),
+        static_cast<const float*>(rows), T, start_pos, d.n_h, d.d_h, d.d_R, d.d_c, static_cast<float*>(att));
     if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
   }
   attn_event(g_attn_end, c.st);
@@ -974,7 +978,6 @@ namespace {
 
 static __device__ __align__(256) uint8_t g_static_scratch[MLA_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
@@ -1015,8 +1018,9 @@ extern "C" mla_status mla_decode_static(const mla_dims* dims, const mla_weights*
   if ((s = static_scratch_address(dev, &scratch)) != MLA_OK) return s;
   c.ws = static_cast<uint8_t*>(scratch);
   c.status = reinterpret_cast<int*>(c.ws + c.L.status);
-  // the array keeps the previous call's contents: the status word is cleared
-  // here, the split-K tickets by the first kernel of the sequence
+  // the array keeps the previous call's contents: only the status word has to
+  // start at zero (cleared here); every other region is written in full by a
+  // kernel of this call before any kernel reads it
   if (cudaMemsetAsync(c.status, 0, sizeof(int), c.st) != cudaSuccess) return MLA_ERR_CUDA;
   return decode_run(c, w, h, B, cache, seqlen, u);
 }

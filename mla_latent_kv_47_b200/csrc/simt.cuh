@@ -1,8 +1,8 @@
 // simt.cuh -- CUDA-core kernels of the MLA path.  They serve fp32 storage
-// (the tiny preset, where tensor cores would need tf32 and the work is a few
-// kFLOP) and any dims the tensor-core kernels do not cover.  Also here: the
-// device-side split planner and the split-combine, shared by all attention
-// kernels.
+// only (small layers such as the tiny preset, where tensor cores would need
+// tf32 and the work is a few kFLOP); bf16 storage always runs on the
+// tensor-core kernels.  Also here: the device-side split planner and the
+// split-combine, shared by all attention kernels.
 #pragma once
 #include "epilogue.cuh"
 

@@ -122,3 +122,26 @@ def test_oracle_is_not_reachable_from_the_product():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src, f
+
+
+def test_bf16_shapes_outside_the_tensor_core_kernels_are_rejected(m):
+    """bf16 storage runs on the tensor-core kernels alone: a bf16 layer of
+    another head shape is refused on the host (nothing enqueued, the fake
+    device addresses are never touched) instead of running on other kernels."""
+    import synth
+    A = 1 << 20
+    W = m.Weights(*[A] * 8)
+    C = m.Cache(A, A, None, 1000)
+    base = synth.PRESETS["v2"].dims
+    for field, value in (("d_h", 64), ("d_c", 256), ("n_h", 256), ("d_model", 5120 + 32), ("d_cq", 1536 + 32)):
+        dims = m.make_dims(base)
+        setattr(dims, field, value)
+        assert _call_decode(m, dims, W, A, 4, C, A, A, A, 1 << 40) == -2, field
+        assert m.lib.mla_prefill(ctypes.byref(dims), ctypes.byref(W), A, 8, 0, ctypes.byref(C), 0, A, A,
+                                 1 << 40, None) == -2, field
+        assert m.lib.mla_cache_append(ctypes.byref(dims), ctypes.byref(W), A, 4, A, A, ctypes.byref(C), A,
+                                      1 << 40, None) == -2, field
+        assert m.workspace_bytes(dims, 4, 4) == 0, field
+    # the same head shapes in fp32 storage stay on the CUDA-core kernels
+    small = m.make_dims(synth.PRESETS["tiny"].dims)
+    assert m.workspace_bytes(small, 1, 64) > 0

@@ -87,6 +87,21 @@ def test_absorbed_equals_unabsorbed(dims, L):
     assert np.max(np.abs(u0 - u1)) <= 1e-12 * np.max(np.abs(u0))
 
 
+@pytest.mark.parametrize("preset,L", [("v2", 100), ("ragged", 40)])
+def test_absorbed_equals_unabsorbed_at_v2_dims(preset, L):
+    """The absorbed form, which the long ragged parity cases are checked
+    against, equals the un-absorbed App. C form at the DeepSeek-V2 dims and
+    with the presets' own weights and hidden states, not only on small
+    layers."""
+    import synth
+    p = synth.preset(preset)
+    W = synth.weights(p)
+    h = synth.hidden(p, 3, L + 1)
+    u0 = om.decode_unabsorbed(W, h, p.dims)
+    u1 = om.decode_absorbed(W, h, p.dims)
+    assert np.max(np.abs(u0 - u1)) <= 1e-12 * np.max(np.abs(u0))
+
+
 def test_softmax_rows_sum_to_one():
     dims = PRESETS["tiny"].dims
     W = rand_weights(dims, 3, std=0.3)
