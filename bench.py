@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-secondary", action="store_true", help="skip the V2-Lite and ragged decode objects")
     ap.add_argument("--profile", action="store_true",
                     help="decode steps only (no clock sampling, e2e, prefill or CPU baseline): for ncu captures")
+    ap.add_argument("--profile-prefill", type=int, default=0, metavar="T",
+                    help="only `--steps` prefill calls of T tokens at the DeepSeek-V2 dims (for ncu captures)")
     return ap.parse_args()
 
 
@@ -364,6 +366,30 @@ def decode_summary(d, L, ms, attn_ms, world, hbm_gbs, bf16_tf):
     }
 
 
+def profile_prefill(m, dev, g, T, steps, barrier):
+    """`steps` prefill calls of T tokens (V2 dims) after one warm-up call, for ncu."""
+    import torch
+    import synth
+    from synth import weight_shapes
+    from mla_latent_kv_47_b200.cache import LatentCache
+    d = synth.preset("prefill").dims
+    dims = m.make_dims(d)
+    Wd = {k: (torch.randn(s, generator=g, device=dev) * 0.02).to(torch.bfloat16) for k, s in weight_shapes(d).items()}
+    wts = m.make_weights(Wd)
+    pc = LatentCache(dims, [T], device=dev)
+    wsp = m.alloc_workspace(dims, 1, T, device=dev)
+    hp = torch.randn((T, d.d_model), generator=g, device=dev).to(torch.bfloat16)
+    up = torch.empty((T, d.d_model), dtype=torch.float32, device=dev)
+    m.prefill(dims, wts, hp, 0, pc.handle, 0, up, wsp)
+    torch.cuda.synchronize()
+    launches0 = m.kernel_launches()
+    ms, attn, launches = time_steps(m, lambda: m.prefill(dims, wts, hp, 0, pc.handle, 0, up, wsp), steps, barrier)
+    assert m.device_status(wsp)[0] == 0
+    print(json.dumps({"profile_run": True, "prefill_tokens": T, "ms_per_call": ms, "attn_ms": attn,
+                      "launches_before_timing": launches0, "launches_per_call": launches // steps}), flush=True)
+    return 0
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -394,6 +420,8 @@ def run_ours(args):
     # ---- inputs: seeded, synthetic, resident in HBM before timing
     g = torch.Generator(device=dev)
     g.manual_seed(1000 + rank)
+    if args.profile_prefill:
+        return profile_prefill(m, dev, g, args.profile_prefill, args.steps, barrier)
     S = DecodeSetup(m, dev, g, args.workload, args.ctx, args.batch)
     d, L, B = S.p.dims, S.L, S.B
 

@@ -42,8 +42,14 @@
  *    with nothing enqueued; no call switches to another kernel family.
  *  - Errors in arguments, shapes, alignment or workspace size are found on the
  *    host and returned before anything is enqueued.  Faults found on the
- *    device (a position at or beyond `capacity`, a pipeline wait that timed
- *    out) set a status word in the workspace; `mla_get_device_status` reads it.
+ *    device set bits of a status word in the workspace, which
+ *    `mla_get_device_status` reads: 1 = a cache write at a position at or
+ *    beyond `capacity` (or outside the cache) was skipped; 2 = a pipeline
+ *    wait timed out; 4 = the decode planner saw a negative seqlen; 8 = the
+ *    decode attention met scores of a sequence that rose, within one run of
+ *    64-token tiles, more than 96 (in units of log2, after the softmax
+ *    scale) above the maximum of the tiles before them, which is past the
+ *    kernel's range (that sequence's u is not valid).
  */
 #ifndef MLA_B200_H
 #define MLA_B200_H
@@ -78,6 +84,17 @@ typedef struct {
     int d_cq;          /* query compression dimension d_c'; 0 = no query compression (V2-Lite) */
     double rope_base;  /* RoPE base, e.g. 10000 */
     int dtype;         /* mla_dtype: storage type of h, weights and cache */
+    /* YaRN context extension (DeepSeek-V2 summary §3.1.4): 0 = off (plain
+     * RoPE, softmax scale 1/sqrt(d_h+d_R)).  With yarn_s >= 1 the rotary pairs
+     * of q^R and k^R use the YaRN frequencies: pair m keeps
+     * theta_m = rope_base^(-2m/d_R) when yarn_L0 (the pre-training length)
+     * spans more than yarn_beta of its wavelengths 2 pi / theta_m, takes
+     * theta_m / yarn_s below yarn_alpha of them and blends linearly in
+     * between; every attention score is multiplied by t with
+     * sqrt(t) = 0.0707 ln(yarn_s) + 1.  The pages give s = 40, alpha = 1,
+     * beta = 32 and a 4K pre-training length.  Requires yarn_beta > yarn_alpha
+     * >= 0 and yarn_L0 > 0. */
+    double yarn_s, yarn_alpha, yarn_beta, yarn_L0;
 } mla_dims;
 
 typedef struct {

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(HERE, "libmla_b200.so")
 MLA_BF16, MLA_FP32 = 0, 1
 STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3: "MLA_ERR_MISALIGNED",
           -4: "MLA_ERR_WORKSPACE", -5: "MLA_ERR_CUDA", -6: "MLA_ERR_DEVICE_FAULT"}
-FAULT_CAPACITY, FAULT_WAIT_TIMEOUT, FAULT_PLAN = 1, 2, 4
+FAULT_CAPACITY, FAULT_WAIT_TIMEOUT, FAULT_PLAN, FAULT_RANGE = 1, 2, 4, 8
 WS_CQ, WS_QC, WS_QLAT, WS_OLAT, WS_O = range(5)
 
 EXPORTS = ("mla_workspace_bytes", "mla_cache_append", "mla_decode", "mla_prefill",
@@ -35,7 +35,8 @@ class MLAError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [("d_model", ctypes.c_int), ("n_h", ctypes.c_int), ("d_h", ctypes.c_int), ("d_R", ctypes.c_int),
                 ("d_c", ctypes.c_int), ("d_cq", ctypes.c_int), ("rope_base", ctypes.c_double),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("yarn_s", ctypes.c_double), ("yarn_alpha", ctypes.c_double),
+                ("yarn_beta", ctypes.c_double), ("yarn_L0", ctypes.c_double)]
 
 
 class Weights(ctypes.Structure):
@@ -99,9 +100,11 @@ def status_string(code: int) -> str:
 
 
 def make_dims(d) -> Dims:
-    """ctypes dims from any object with the fields of synth.Dims."""
+    """ctypes dims from any object with the fields of synth.Dims (and, for
+    YaRN, a `yarn` = (s, alpha, beta, L0) attribute)."""
+    y = getattr(d, "yarn", None) or (0.0, 0.0, 0.0, 0.0)
     return Dims(d.d_model, d.n_h, d.d_h, d.d_R, d.d_c, d.d_cq, float(d.rope_base),
-                MLA_FP32 if getattr(d, "dtype", "bf16") == "fp32" else MLA_BF16)
+                MLA_FP32 if getattr(d, "dtype", "bf16") == "fp32" else MLA_BF16, *[float(v) for v in y])
 
 
 def _ptr(t):

@@ -24,6 +24,16 @@
 // retirement is committed to both CTAs' barriers (multicast commit), which
 // tells each side that both P buffers may take the next tile.
 //
+// The softmax never waits for the partner inside a piece.  Both CTAs form
+// P(j) against the same running max m, and decide whether tile j moves m
+// one tile later, once the partner's tile maxima (sent as soon as S(j) is
+// read) have long arrived: if the max over both halves of tile j exceeds m
+// by more than 2^8, both rescale O and l and take the new max from tile
+// j + 1 on.  Only a piece's first tile waits for the partner (it sets m).
+// Until a decision lands, P may exceed 1; the kernel's range is
+// P <= 2^96 (ample for fp32 O and l), and a tile whose scores jump past it
+// sets FAULT_RANGE.
+//
 // Warp roles (448 threads per CTA):
 //   warp 0      TMA producer (3-stage ring)
 //   warp 1      TMEM owner and MMA issuer: S(j) once tile j landed and the S
@@ -34,8 +44,9 @@
 //               16 heads each; two threads per head (rows 0-15 and 16-31 of
 //               this CTA's half, via the 16-lane TMEM access shape).  Online
 //               softmax with a lazily refreshed max (O is rescaled only when a
-//               tile's max exceeds the running one by more than 2^8), and the
-//               per-piece epilogue; CTA 1 sends its share of l to CTA 0.
+//               tile's max exceeds the running one by more than 2^8, decided
+//               one tile late as above), and the per-piece epilogue; CTA 1
+//               sends its share of l to CTA 0.
 #pragma once
 #include "mla.h"
 #include "ptx.cuh"
@@ -59,12 +70,15 @@ constexpr int kQSmemChunks = 9 - kQTmemChunks;
 constexpr int kQChunkBytes = 128 * 128;                // 128 heads x 64 columns, bf16
 constexpr int kPBytes = 128 * 128;                     // P: 128 heads x 64 rows, bf16 (CTA 0's rows first)
 constexpr int kPBufs = 2;
-constexpr int kAuxBytes = 2048;                        // partner maxima, CTA 1's l, barriers
+constexpr int kMaxSlots = 4;                           // partner tile maxima in flight (tile j in slot j % 4)
+constexpr int kPrefetchAhead = 6;                      // tiles brought into L2 ahead of their TMA load
+constexpr int kAuxBytes = 3072;                        // partner maxima, CTA 1's l, barriers
 // stages | Q chunks 7-8 | P x 2 | aux
 constexpr int kSmem = 1024 + kStages * kStageBytes + kQSmemChunks * kQChunkBytes + kPBufs * kPBytes + kAuxBytes;
 // TMEM columns: O half [0,256), S [256,288), Q chunks 0-6 (bf16 pairs) [288,512)
 constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 288, kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;
+constexpr float kRangeLog2 = 96.f;                     // largest exponent of P before the max catches up
 constexpr int kRow = 576;                              // d_c + d_R
 static_assert(kTmemQ + kQTmemChunks * 32 == kTmemCols, "TMEM budget");
 static_assert(kSmem <= 232448, "shared memory budget");
@@ -92,14 +106,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   uint8_t* qs = stages + kStages * kStageBytes;       // Q chunks 7-8, MMA A operand
   uint8_t* pbuf = qs + kQSmemChunks * kQChunkBytes;   // [2] P (bf16), MMA A operand
   uint8_t* aux = pbuf + kPBufs * kPBytes;
-  float* mx = reinterpret_cast<float*>(aux);          // [2][128] the partner's tile maxima (st.async)
-  float* lsh = mx + 256;                              // [128] CTA 1's share of l, in CTA 0 (st.async)
-  uint64_t* full = reinterpret_cast<uint64_t*>(aux + 1536);
+  float* mx = reinterpret_cast<float*>(aux);          // [4][128] the partner's tile maxima (st.async)
+  float* lsh = mx + kMaxSlots * 128;                  // [128] CTA 1's share of l, in CTA 0 (st.async)
+  uint64_t* full = reinterpret_cast<uint64_t*>(aux + 2560);
   uint64_t* empty = full + kStages;
   uint64_t* s_full = empty + kStages;  // S(j) in TMEM (MMA -> softmax)
   uint64_t* s_free = s_full + 1;       // S read out (softmax -> MMA)
-  uint64_t* mx_full = s_free + 1;      // [2] the partner's maxima of tile j landed (index j & 1)
-  uint64_t* p_full = mx_full + 2;      // [2] this CTA's half of P(j) written
+  uint64_t* mx_full = s_free + 1;      // [4] the partner's maxima of tile j landed (slot j % 4)
+  uint64_t* p_full = mx_full + kMaxSlots;  // [2] this CTA's half of P(j) written
   uint64_t* px_full = p_full + 2;      // [2] the partner's half of P(j) landed
   uint64_t* pv_done = px_full + 2;     // [2] PV(j) retired in both CTAs (one commit from each)
   uint64_t* q_full = pv_done + 2;
@@ -122,8 +136,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 8);        // one arrival per softmax warp
+    for (int i = 0; i < kMaxSlots; ++i) mbar_init(&mx_full[i], 1);  // armed per phase with the partner's 512 bytes
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&mx_full[i], 1);  // armed per phase with the partner's 512 bytes
       mbar_init(&p_full[i], 8);   // one arrival per softmax warp
       mbar_init(&px_full[i], 1);  // armed per phase with the partner's 8 KB
       mbar_init(&pv_done[i], 2);  // this CTA's and the partner's PV commit
@@ -135,10 +149,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    for (int i = 0; i < 2; ++i) {
-      mbar_arrive_expect_tx(&mx_full[i], 128 * 4);
-      mbar_arrive_expect_tx(&px_full[i], kPBytes / 2);
-    }
+    for (int i = 0; i < kMaxSlots; ++i) mbar_arrive_expect_tx(&mx_full[i], 128 * 4);
+    for (int i = 0; i < 2; ++i) mbar_arrive_expect_tx(&px_full[i], kPBytes / 2);
     if (rank == 0) mbar_arrive_expect_tx(l_full, 128 * 4);
   }
   if (warp == 0 && lane == 0) prefetch_tmap(&a.map_cache);
@@ -160,6 +172,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       // second read is an L2 hit; the rest is streamed with evict-first.
       const uint64_t pol_once = policy_evict_first();
       const uint64_t pol_twice = policy_evict_normal();
+      // A stage is held from its load until the tile's PV retires, so the
+      // ring alone keeps about one tile per CTA in flight from HBM.  This CTA's
+      // rows of the tiles kPrefetchAhead ahead are therefore pulled into L2
+      // first (the partner pulls its own rows, which this CTA also reads), and
+      // the ring's loads find them there.  Cursor: next worker tile to
+      // prefetch, as a global tile index and its sequence.
+      long long pf_g = 0, pf_end = 0;
+      int pf_b = 0;
+      {
+        const long long Tt = a.tile_start[a.B];
+        const int We = static_cast<int>(Tt < a.W ? Tt : a.W);
+        if (Tt > 0 && w < We) {
+          pf_g = worker_begin(w, Tt, We) + kStages;  // the first kStages tiles are loaded at once
+          pf_end = worker_begin(w + 1, Tt, We);
+          int lo = 0, hi = a.B - 1;                  // sequence of tile pf_g
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (a.tile_start[mid + 1] > pf_g) hi = mid; else lo = mid + 1;
+          }
+          pf_b = lo;
+        }
+      }
+      auto prefetch_next = [&]() {
+        if (pf_g >= pf_end) return;
+        while (pf_b + 1 < a.B && a.tile_start[pf_b + 1] <= pf_g) ++pf_b;
+        const long long y = a.seq_start[pf_b] + (pf_g - a.tile_start[pf_b]) * kAttnTileTokens + kHalf * rank;
+        for (int ci = 0; ci < kOwnChunks; ++ci) tma_prefetch_l2_2d(&a.map_cache, ci * 64, static_cast<int>(y));
+        ++pf_g;
+      };
+      for (int i = kStages; i < kStages + kPrefetchAhead; ++i) prefetch_next();
       int it = 0;
       for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
         if (*abort_flag) return;
@@ -167,6 +209,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         for (int t = p.t0; t < p.t1; ++t, ++it) {
           const int s = it % kStages;
           if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, wc)) return;
+          if (it >= kStages) prefetch_next();  // tile it + kPrefetchAhead
           mbar_arrive_expect_tx(&full[s], kStageBytes);
           uint8_t* dst = stages + s * kStageBytes;
           const long long y0 = row0 + static_cast<long long>(t) * kAttnTileTokens;
@@ -325,11 +368,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     const uint32_t mx_peer = mapa(smem_u32(mx), peer) + h * 4;
     const uint32_t mxfull_peer = mapa(smem_u32(mx_full), peer);
     int it = 0, piece = 0;
+    // The partner's maxima of tile g sit in slot g % kMaxSlots; reading them
+    // (and re-arming the slot) is the only per-tile wait on the partner.
+    auto partner_max = [&](int g, float& v) -> bool {
+      const int slot = g & (kMaxSlots - 1);
+      if (!mbar_wait<true>(&mx_full[slot], (g / kMaxSlots) & 1, wc)) return false;
+      v = mx[slot * 128 + h];
+      // next phase of the slot: the partner's maxima of tile g + 4, which it
+      // sends only after reading this CTA's maxima of tile g + 2 (sent later)
+      if (lead) mbar_arrive_expect_tx(&mx_full[slot], 128 * 4);
+      return true;
+    };
     for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
       if (*abort_flag) return;
       const bool head = h < a.n_h;
       const int L1 = a.seqlen[p.b] + 1;
       float m_run = -INFINITY, l_run = 0.f;  // l_run: this thread's 16 rows only
+      float mo_prev = -INFINITY;             // this CTA's max of the previous tile
       const int nt = p.t1 - p.t0;
       for (int k = 0; k < nt; ++k) {
         const int g = it + k;
@@ -357,47 +412,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
 #pragma unroll
         for (int j = 1; j < 16; ++j) mo = fmaxf(mo, sc[j]);
         mo = fmaxf(mo, __shfl_xor_sync(0xffffffffu, mo, 16));  // this CTA's 32 rows
-        if (th == 0) st_async_b32(mx_peer + b * 512, __float_as_uint(mo), mxfull_peer + b * 8);
-        // P of this thread's rows against max m; returns their sum
-        uint32_t pk[8];
-        auto exp_rows = [&](float m) {
-          float sum = 0.f;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float p0 = ex2_approx(sc[2 * j] - m), p1 = ex2_approx(sc[2 * j + 1] - m);
-            sum += p0 + p1;
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-            pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
-          }
-          return sum;
-        };
-        // Past a piece's first tile the max almost always stays, so P is formed
-        // against it while the partner's maxima are on their way, and formed
-        // again only if the tile's max does move it.
-        float lsum = k > 0 ? exp_rows(m_run) : 0.f;
-        if (!mbar_wait<true>(&mx_full[b], ph, wc)) return;
-        const float mt = fmaxf(mo, mx[b * 128 + h]);  // the tile's max, the same in both CTAs
-        // next phase: the partner's maxima of tile g + 2, which it sends only
-        // after this CTA's maxima of tile g + 1 (sent after this point) landed
-        if (lead) mbar_arrive_expect_tx(&mx_full[b], 128 * 4);
-        float m_new = m_run, alpha = 1.f;
+        if (th == 0) st_async_b32(mx_peer + (g & (kMaxSlots - 1)) * 512, __float_as_uint(mo), mxfull_peer + (g & (kMaxSlots - 1)) * 8);
         bool rescale = false;
+        float alpha = 1.f;
         if (k == 0) {
-          m_new = mt;
-          lsum = exp_rows(m_new);
-        } else if (mt > m_run + kRescaleLog2) {
-          m_new = mt;
-          alpha = ex2_approx(m_run - m_new);
-          rescale = true;
-          lsum = exp_rows(m_new);
+          // the piece's first tile sets the max: both halves are needed now
+          float pm;
+          if (!partner_max(g, pm)) return;
+          m_run = fmaxf(mo, pm);
+        } else if (k >= 2) {
+          // the decision for tile g - 1, whose partner maxima arrived a tile ago
+          float pm;
+          if (!partner_max(g - 1, pm)) return;
+          const float mt = fmaxf(mo_prev, pm);  // the same value in both CTAs
+          if (mt > m_run + kRescaleLog2) {
+            alpha = ex2_approx(m_run - mt);
+            m_run = mt;
+            rescale = true;
+          }
+        }
+        mo_prev = mo;
+        // P of this thread's rows against m_run, and their sum; exponents are
+        // capped at the kernel's range (a jump past it is reported)
+        if (__any_sync(0xffffffffu, mo > m_run + kRangeLog2)) {
+          if (mo > m_run + kRangeLog2) atomicOr(a.status, FAULT_RANGE);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) sc[j] = fminf(sc[j], m_run + kRangeLog2);
+        }
+        uint32_t pk[8];
+        float lsum = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float p0 = ex2_approx(sc[2 * j] - m_run), p1 = ex2_approx(sc[2 * j + 1] - m_run);
+          lsum += p0 + p1;
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+          pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
         }
         l_run = l_run * alpha + lsum;
-        m_run = m_new;
         // ---- P buffer b is free in both CTAs once PV(g-2) retired in both
         if (!mbar_wait_inline(&pv_done[b], ph ^ 1, wc)) return;
         tc_fence_after();
         if (__any_sync(0xffffffffu, rescale)) {
-          // O must hold PV(g-1) before it is scaled (k >= 1 here, so g >= 1)
+          // O must hold PV(g-1) before it is scaled (k >= 2 here, so g >= 1)
           if (!mbar_wait_inline(&pv_done[b ^ 1], ((g - 1) >> 1) & 1, wc)) return;
           tc_fence_after();
           for (int c = 0; c < 256; c += 32) {
@@ -436,6 +492,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[b]);
+      }
+      // the partner's maxima of the piece's last tile (if not read yet) must
+      // land before the slot is reused; O, l and m_run are already consistent
+      if (nt >= 2) {
+        float pm;
+        if (!partner_max(it + nt - 1, pm)) return;
       }
       // ---- epilogue of the piece: unnormalised O_r; CTA 0 writes m and l
       if (!mbar_wait(o_done, piece & 1, wc)) return;

@@ -42,6 +42,8 @@ struct TokenMap {
   int d_c, d_R;
   double log2_base;          // log2(rope_base)
   const float2* rope;        // NULL, or (cos, sin) of pair i at token n: rope[n * d_R / 2 + i]
+  double yarn_s;             // 0: plain RoPE; else the YaRN scale s (with alpha, beta, L0 below)
+  double yarn_alpha, yarn_beta, yarn_L0;
 };
 
 __device__ __forceinline__ int tok_pos(const TokenMap& t, int n) { return t.pos ? t.pos[n] : t.pos_base + n; }
@@ -53,8 +55,18 @@ __device__ __forceinline__ int tok_seq(const TokenMap& t, int n) {
 // product pos * base^(-2i/d_R) is formed and reduced in fp64 (positions reach
 // 1.3e5, where an fp32 angle would already be off by ~4e-3 rad), then sine and
 // cosine are taken in fp32.
-__device__ __forceinline__ double rope_inv_freq(int i, int d_R, double log2_base) {
-  return exp2(-(2.0 * i / d_R) * log2_base);
+// Rotary frequency of pair i: theta_i = base^(-2i/d_R) (RoFormer), or with
+// YaRN ("DeepSeek-V2 summary" (7shi.hateblo.jp) §3.1.4: s, alpha, beta and the
+// pre-training length L0) the published YaRN rule: a pair whose wavelength
+// 2 pi / theta_i fits more than beta times into L0 keeps theta_i, one that fits
+// fewer than alpha times takes theta_i / s, and in between the two blend
+// linearly in r = L0 theta_i / (2 pi).
+__device__ __forceinline__ double rope_inv_freq(const TokenMap& t, int i) {
+  const double theta = exp2(-(2.0 * i / t.d_R) * t.log2_base);
+  if (!(t.yarn_s > 0.0)) return theta;
+  const double r = t.yarn_L0 * theta * (1.0 / 6.283185307179586);
+  const double ramp = fmin(fmax((r - t.yarn_alpha) / (t.yarn_beta - t.yarn_alpha), 0.0), 1.0);
+  return (1.0 - ramp) * (theta / t.yarn_s) + ramp * theta;
 }
 __device__ __noinline__ void rope_cos_sin(int pos, double inv_freq, float& c, float& s) {
   const double two_pi_hi = 6.283185307179586;
@@ -223,7 +235,7 @@ __device__ __forceinline__ void epi_rope_run(const Epi& e, const TokenMap& tk, i
     c[0] = a.x; s[0] = a.y; c[1] = a.z; s[1] = a.w; c[2] = b.x; s[2] = b.y; c[3] = b.z; s[3] = b.w;
   } else {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) rope_cos_sin(tok_pos(tk, n), rope_inv_freq(i0 + q, tk.d_R, tk.log2_base), c[q], s[q]);
+    for (int q = 0; q < 4; ++q) rope_cos_sin(tok_pos(tk, n), rope_inv_freq(tk, i0 + q), c[q], s[q]);
   }
   const float sc = e.kind == EPI_CACHE_KR ? 1.f : e.scale;
 #pragma unroll
@@ -302,7 +314,7 @@ __device__ __forceinline__ bool epi_needs_rope(int kind) {
 __device__ __forceinline__ double epi_inv_freq(const Epi& e, const TokenMap& tk, int m) {
   if (!epi_needs_rope(e.kind)) return 0.0;
   const int j = (e.kind == EPI_CACHE_KR) ? m : (m % tk.d_R);
-  return rope_inv_freq(j >> 1, tk.d_R, tk.log2_base);
+  return rope_inv_freq(tk, j >> 1);
 }
 
 // (cos, sin) of every rotary pair of the call's T tokens, for the epilogues
@@ -317,7 +329,7 @@ __global__ void __launch_bounds__(256) rope_table_kernel(const TokenMap tk, int 
        idx += static_cast<long long>(gridDim.x) * 256) {
     const int n = static_cast<int>(idx / half), i = static_cast<int>(idx % half);
     float c, s;
-    rope_cos_sin(tok_pos(tk, n), rope_inv_freq(i, tk.d_R, tk.log2_base), c, s);
+    rope_cos_sin(tok_pos(tk, n), rope_inv_freq(tk, i), c, s);
     out[idx] = make_float2(c, s);
   }
 }

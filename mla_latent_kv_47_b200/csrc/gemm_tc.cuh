@@ -43,6 +43,7 @@ struct GemmArgs {
   int splits;
   float* partials;             // [tiles][splits][BN/4][128][4] fp32 (splits > 1)
   int* status;
+  int x_independent;           // 1: X is a call input no earlier kernel writes; only the epilogue waits
   TokenMap tok;
 };
 
@@ -150,13 +151,14 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                     head * args.b_head_stride + (kb0 + i * KBB + j) * 64, nt * BN, polB);
       };
       // Weights do not depend on earlier kernels: the first stages of A are
-      // fetched before waiting for the kernel that produces X.
+      // fetched before waiting for the kernel that produces X (no wait at all
+      // when X is a call input).
       const int pre = nk < STAGES ? nk : STAGES;
       for (int i = 0; i < pre; ++i) {
         mbar_arrive_expect_tx(&full[i], stage_kbs(i) * (bytesA + bytesB));
         for (int j = 0; j < stage_kbs(i); ++j) load_a(i, j);
       }
-      griddep_wait();
+      if (!args.x_independent) griddep_wait();
       for (int i = 0; i < pre; ++i)
         for (int j = 0; j < stage_kbs(i); ++j) load_b(i, j);
       for (int i = pre; i < nk; ++i) {
@@ -202,6 +204,9 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
     mbar_wait(accum, 0, wc);
     tc_fence_after();
+    // with an independent X the main loop ran alongside the previous kernel;
+    // the epilogue reads its tables and writes what it may still read
+    if (args.x_independent) griddep_wait();
     named_bar_sync(1, 128);            // every epilogue thread sees the same abort decision
     if (!*abort_flag) {
       const Epi& e = args.epi[seg];

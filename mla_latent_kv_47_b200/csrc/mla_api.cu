@@ -127,6 +127,7 @@ struct GemmSpec {
   int head_rows = 0;            // rows of A per head
   int b_head_stride = 0;        // X column offset per head
   TokenMap tok{};
+  bool x_independent = false;   // X is a call input (h): the GEMM need not wait for the kernel before it
 };
 
 struct Ctx {
@@ -231,6 +232,7 @@ mla_status run_gemm_tc(const Ctx& c, const GemmSpec& g, const GemmConfig& cfg) {
   a.b_head_stride = g.b_head_stride;
   a.status = c.status;
   a.tok = g.tok;
+  a.x_independent = g.x_independent ? 1 : 0;
   int m_tiles = 0, mt_per_cta = 1;
   if (g.mode == GEMM_DENSE) {
     a.nseg = g.nseg;
@@ -362,6 +364,11 @@ mla_status check_dims(const mla_dims* d) {
   if (d->d_model <= 0 || d->n_h <= 0 || d->d_h <= 0 || d->d_R <= 0 || d->d_c <= 0 || d->d_cq < 0)
     return MLA_ERR_INVALID_ARG;
   if (!(d->rope_base > 1.0) || !std::isfinite(d->rope_base)) return MLA_ERR_INVALID_ARG;
+  if (d->yarn_s != 0.0 &&
+      (!(d->yarn_s >= 1.0) || !std::isfinite(d->yarn_s) || !(d->yarn_alpha >= 0.0) ||
+       !(d->yarn_beta > d->yarn_alpha) || !std::isfinite(d->yarn_beta) || !(d->yarn_L0 > 0.0) ||
+       !std::isfinite(d->yarn_L0)))
+    return MLA_ERR_INVALID_ARG;
   if (d->dtype != MLA_BF16 && d->dtype != MLA_FP32) return MLA_ERR_UNSUPPORTED;
   if (d->d_R % 2 != 0) return MLA_ERR_UNSUPPORTED;
   // CUDA-core kernels hold d_c/32 <= 16 latent columns and d_h/32 <= 8 value columns per lane.
@@ -429,6 +436,10 @@ TokenMap cache_tokens(const mla_dims& d, const mla_cache* cache) {
   t.d_R = d.d_R;
   t.log2_base = std::log2(d.rope_base);
   t.seq_const = -1;
+  t.yarn_s = d.yarn_s;
+  t.yarn_alpha = d.yarn_alpha;
+  t.yarn_beta = d.yarn_beta;
+  t.yarn_L0 = d.yarn_L0;
   return t;
 }
 
@@ -466,8 +477,16 @@ Epi epi_kind(int kind, void* out = nullptr, long long ld = 0, long long hs = 0, 
   return e;
 }
 
+// Factor folded into the query: scores come out in log2 units (the softmax
+// uses exp2) and carry the softmax scale 1/sqrt(d_h + d_R) ("DeepSeek-V2
+// summary" App. C), times YaRN's t with sqrt(t) = 0.0707 ln s + 1 (§3.1.4).
 float qlat_scale(const mla_dims& d) {
-  return static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d.d_h + d.d_R)));
+  double t = 1.0;
+  if (d.yarn_s != 0.0) {
+    const double rt = 0.0707 * std::log(d.yarn_s) + 1.0;
+    t = rt * rt;
+  }
+  return static_cast<float>(1.4426950408889634 * t / std::sqrt(static_cast<double>(d.d_h + d.d_R)));
 }
 
 // Appends the [W_DKV; W_KR] segments (cache-row epilogues) to a dense GEMM.
@@ -560,12 +579,15 @@ mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const 
     return s;
   tk.rope = rope;
 
-  // ---- a1 (+a2): down-projections from h, cache append of the new token
+  // ---- a1 (+a2): down-projections from h, cache append of the new token.
+  // h is a call input, so the GEMM streams weights and h while the planner
+  // runs and waits for it only in the epilogue (RoPE table, cache rows).
   {
     GemmSpec g;
     g.K = d.d_model;
     g.a_ld = d.d_model;
     g.X = h;
+    g.x_independent = true;
     g.x_cols = d.d_model;
     g.x_ld = d.d_model;
     g.N = B;

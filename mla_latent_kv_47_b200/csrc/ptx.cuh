@@ -16,6 +16,8 @@ enum : int {
   FAULT_CAPACITY = 1,      // a cache write at pos >= capacity was skipped
   FAULT_WAIT_TIMEOUT = 2,  // a pipeline wait ran out of time
   FAULT_PLAN = 4,          // the device planner saw inconsistent sizes
+  FAULT_RANGE = 8,         // decode attention: a tile's scores exceeded the running max by more than
+                           // the kernel's range (2^96); the sequence's output is not valid
 };
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
@@ -182,6 +184,13 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
       "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
       : "memory");
+}
+
+// Brings the box at (x, y) of `map` into L2 without touching shared memory
+// (rows past the tensor are skipped).  x * elem_size must be a multiple of 16.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+               : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05

@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seqlen, int B
     const int half = tk.d_R >> 1;
     for (int idx = threadIdx.x; idx < B * half; idx += 1024) {
       float c, s;
-      rope_cos_sin(tok_pos(tk, idx / half), rope_inv_freq(idx % half, tk.d_R, tk.log2_base), c, s);
+      rope_cos_sin(tok_pos(tk, idx / half), rope_inv_freq(tk, idx % half), c, s);
       rope[idx] = make_float2(c, s);
     }
   }

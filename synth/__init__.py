@@ -39,6 +39,7 @@ class Dims:
     d_cq: int          # 0: no query compression (W_UQ / W_QR act on h directly)
     rope_base: float = 10000.0
     dtype: str = "bf16"  # storage dtype of h, weights and cache: "bf16" | "fp32"
+    yarn: tuple | None = None  # (s, alpha, beta, L0) of YaRN, or None for plain RoPE
 
     @property
     def row_elems(self) -> int:

@@ -145,3 +145,22 @@ def test_bf16_shapes_outside_the_tensor_core_kernels_are_rejected(m):
     # the same head shapes in fp32 storage stay on the CUDA-core kernels
     small = m.make_dims(synth.PRESETS["tiny"].dims)
     assert m.workspace_bytes(small, 1, 64) > 0
+
+
+def test_yarn_arguments_are_checked(m):
+    """YaRN is off at yarn_s = 0; otherwise s >= 1, beta > alpha >= 0 and
+    L0 > 0 are required (checked on the host, nothing enqueued)."""
+    import synth
+    A = 1 << 20
+    W = m.Weights(*[A] * 8)
+    C = m.Cache(A, A, None, 1000)
+    ok = m.make_dims(synth.PRESETS["v2"].dims)
+    assert m.workspace_bytes(ok, 4, 4) > 0
+    for y in ((0.5, 1.0, 32.0, 4096.0), (40.0, 32.0, 1.0, 4096.0), (40.0, 1.0, 32.0, 0.0),
+              (40.0, -1.0, 32.0, 4096.0), (float("nan"), 1.0, 32.0, 4096.0)):
+        d = m.make_dims(synth.PRESETS["v2"].dims)
+        d.yarn_s, d.yarn_alpha, d.yarn_beta, d.yarn_L0 = y
+        assert _call_decode(m, d, W, A, 4, C, A, A, A, 1 << 40) == -1, y
+    d = m.make_dims(synth.PRESETS["v2"].dims)
+    d.yarn_s, d.yarn_alpha, d.yarn_beta, d.yarn_L0 = 40.0, 1.0, 32.0, 4096.0
+    assert m.workspace_bytes(d, 4, 4) > 0

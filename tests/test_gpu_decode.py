@@ -26,14 +26,20 @@ def m():
     return mod
 
 
-def run_decode(m, preset, checked, lengths=None, pad=2, oracle="unabsorbed", dirty_workspace=False, h_scale=None):
+def run_decode(m, preset, checked, lengths=None, pad=2, oracle="unabsorbed", dirty_workspace=False, h_scale=None,
+               dims=None, weights=None):
+    """Fills a poisoned cache through mla_cache_append, runs one mla_decode and
+    checks layout, cache rows and u.  `dims` replaces the preset's dims (same
+    shapes, e.g. with YaRN on); `weights` (host, device) replaces its weights.
+    `oracle` names the fp64 form u is compared with, per sequence when it is a
+    callable of the sequence's length."""
     from mla_latent_kv_47_b200.cache import LatentCache
     p = synth.preset(preset)
-    d = p.dims
+    d = p.dims if dims is None else dims
     dims = m.make_dims(d)
     L = list(lengths if lengths is not None else p.seqlen)
     B = len(L)
-    Wh, Wd = gu.device_weights(p)
+    Wh, Wd = gu.device_weights(p) if weights is None else weights
     cache = LatentCache(dims, [x + 1 + pad for x in L], poison=True, gap=1)
     ws = m.alloc_workspace(dims, B, 1)
     if dirty_workspace:
@@ -83,7 +89,8 @@ def run_decode(m, preset, checked, lengths=None, pad=2, oracle="unabsorbed", dir
             rows_ref = np.concatenate([c_kv, k_r], axis=1)
             gotf = got.view(np.float32).astype(np.float64)
             assert np.max(np.abs(gotf - rows_ref)) <= 1e-5 * np.max(np.abs(rows_ref))
-        u_ref = (om.decode_unabsorbed if oracle == "unabsorbed" else om.decode_absorbed)(Wh, hb, d)
+        form = oracle(L[b]) if callable(oracle) else oracle
+        u_ref = (om.decode_unabsorbed if form == "unabsorbed" else om.decode_absorbed)(Wh, hb, d)
         stats[b] = gu.gate(u_h[b], u_ref)
     return stats
 
@@ -252,3 +259,31 @@ def test_decode_intermediates(m, preset):
                                ("o_lat", olat[b], parts["o_lat"])):
             s = gu.gate(got, ref)
             assert s["max_rel"] <= 1e-2 and s["mean_rel"] <= 2e-3, (name, b, s)
+
+
+def test_score_jump_past_the_kernel_range_is_reported(m):
+    """Inside a run of tiles the attention kernel forms P against the running
+    max and learns a tile's max one tile late, so P may exceed 1 until then;
+    its range is P <= 2^96.  Cached tokens 192..255 of sequence 0 scaled by 64
+    put that tile's scores ~200 log2 units above the earlier tiles' (its piece
+    starts at tile 0: 8 sequences of 4096 tokens give ~7 tiles per attention
+    worker), past the range, so the call reports FAULT_RANGE through the
+    status word instead of returning a silently wrong u; the status is
+    cleared by reading it."""
+    from mla_latent_kv_47_b200.cache import LatentCache
+    p = synth.preset("v2")
+    d = p.dims
+    dims = m.make_dims(d)
+    L = [4096] * 8
+    Wh, Wd = gu.device_weights(p)
+    cache = LatentCache(dims, [x + 1 for x in L])
+    ws = m.alloc_workspace(dims, len(L), 1)
+    h0 = synth.hidden(p, 0, L[0] + 1)
+    h0[192:256] *= 64.0
+    gu.fill_cache(m, dims, Wd, cache, ws, {0: h0}, L, p)
+    h_new = gu.to_dev(np.stack([h0[L[0]]] + [synth.hidden(p, b, 1, first=L[b])[0] for b in range(1, 8)]), "bf16")
+    u = torch.empty((len(L), d.d_model), dtype=torch.float32, device="cuda")
+    m.decode(dims, m.make_weights(Wd), h_new, cache.handle, torch.tensor(L, dtype=torch.int32, device="cuda"), u, ws)
+    code, detail = m.device_status(ws)
+    assert code == -6 and detail & m.FAULT_RANGE, (code, detail)
+    assert m.device_status(ws) == (0, 0)

@@ -17,12 +17,12 @@ def m():
     return mod
 
 
-def run_prefill(m, preset, T, start_pos=0, rows=None, seq=1, n_seq=3, pad=3):
+def run_prefill(m, preset, T, start_pos=0, rows=None, seq=1, n_seq=3, pad=3, dims=None, weights=None):
     from mla_latent_kv_47_b200.cache import LatentCache
     p = synth.preset(preset)
-    d = p.dims
+    d = p.dims if dims is None else dims
     dims = m.make_dims(d)
-    Wh, Wd = gu.device_weights(p)
+    Wh, Wd = gu.device_weights(p) if weights is None else weights
     S = start_pos + T
     cache = LatentCache(dims, [S + pad] * n_seq, poison=True, gap=1)
     ws = m.alloc_workspace(dims, 1, S)

@@ -151,3 +151,17 @@ def test_planted_mistake_is_caught(name, monkeypatch):
     monkeypatch.setattr(om, attr, fn)
     with pytest.raises(AssertionError):
         pin()
+
+
+def test_yarn_moves_v2_decode_by_more_than_the_gpu_gate():
+    """At DeepSeek-V2 dims and positions past the 4K pre-training length, YaRN
+    changes u by several times the GPU parity gate (1e-2 of max|u|), so the GPU
+    YaRN parity tests cannot pass with plain RoPE."""
+    import dataclasses
+    import synth
+    p = synth.preset("v2")
+    W = synth.weights(p)
+    h = synth.hidden(p, 1, 6001)
+    a = om.decode_absorbed(W, h, dataclasses.replace(p.dims, yarn=V2_YARN))
+    b = om.decode_absorbed(W, h, p.dims)
+    assert np.max(np.abs(a - b)) > 5e-2 * np.max(np.abs(a))
