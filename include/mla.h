@@ -106,15 +106,32 @@ typedef struct {
     const void* W_UV;
     const void* W_KR;
     const void* W_O;
+    /* RMSNorm gains of the compressed latents (DeepSeek-V2 summary §3.1.2,
+     * which adds RMSNorm layers after them; App. C has none).  NULL = no norm.
+     * g_kv [d_c]: c^KV is normalised, x / sqrt(mean(x^2) + 1e-6) * g_kv, before
+     * it is cached.  g_q [d_cq]: c^Q is normalised the same way before the
+     * up-projections (only with query compression: g_q with d_cq == 0 is
+     * MLA_ERR_INVALID_ARG).  Storage dtype, 16-byte aligned. */
+    const void* g_kv;
+    const void* g_q;
 } mla_weights;
 
 typedef struct {
     void* base;                 /* device: rows of (d_c + d_R) elements */
-    const int64_t* seq_start;   /* device [n_seq]: row of token 0 of each sequence */
+    const int64_t* seq_start;   /* device [n_seq]: row of token 0 of each sequence (contiguous
+                                   layout; unused, may be NULL, when block_table is given) */
     const int32_t* capacity;    /* device [n_seq] or NULL: rows reserved per sequence; a write at
                                    pos >= capacity[s] is skipped and raises MLA_ERR_DEVICE_FAULT */
     int64_t n_rows;             /* rows allocated at `base` (> 0): bounds of every tile load; a
                                    write at a row >= n_rows is skipped and raises MLA_ERR_DEVICE_FAULT */
+    /* Paged layout (optional; NULL = contiguous per sequence).  The cache is a
+     * pool of pages of block_size rows (a multiple of 64); token p of sequence
+     * s lives in row block_table[s * max_blocks + p / block_size] * block_size
+     * + p % block_size.  device int32 [n_seq x max_blocks], caller-owned.  A
+     * position p >= max_blocks * block_size is treated as beyond capacity. */
+    const int32_t* block_table;
+    int32_t block_size;
+    int32_t max_blocks;
 } mla_cache;
 
 /* Bytes of workspace needed by mla_decode for batches up to `max_batch` and by

@@ -39,13 +39,17 @@ class Dims(ctypes.Structure):
                 ("yarn_beta", ctypes.c_double), ("yarn_L0", ctypes.c_double)]
 
 
+WEIGHT_FIELDS = ("W_DQ", "W_UQ", "W_QR", "W_DKV", "W_UK", "W_UV", "W_KR", "W_O", "g_kv", "g_q")
+
+
 class Weights(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("W_DQ", "W_UQ", "W_QR", "W_DKV", "W_UK", "W_UV", "W_KR", "W_O")]
+    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS]
 
 
 class Cache(ctypes.Structure):
     _fields_ = [("base", ctypes.c_void_p), ("seq_start", ctypes.c_void_p), ("capacity", ctypes.c_void_p),
-                ("n_rows", ctypes.c_int64)]
+                ("n_rows", ctypes.c_int64), ("block_table", ctypes.c_void_p), ("block_size", ctypes.c_int32),
+                ("max_blocks", ctypes.c_int32)]
 
 
 def _load():
@@ -115,14 +119,21 @@ def _ptr(t):
 
 
 def make_weights(W: dict) -> Weights:
-    return Weights(*[_ptr(W.get(n)) for n in ("W_DQ", "W_UQ", "W_QR", "W_DKV", "W_UK", "W_UV", "W_KR", "W_O")])
+    """Device weight tensors by name (the RMSNorm gains g_kv / g_q are optional)."""
+    return Weights(*[_ptr(W.get(n)) for n in WEIGHT_FIELDS])
 
 
-def make_cache(base, seq_start, capacity=None) -> Cache:
-    """base: [n_rows, d_c + d_R] device tensor; seq_start int64 [n_seq]; capacity int32 [n_seq] or None."""
-    assert seq_start.dtype == torch.int64
+def make_cache(base, seq_start=None, capacity=None, block_table=None, block_size=0) -> Cache:
+    """base: [n_rows, d_c + d_R] device tensor; seq_start int64 [n_seq] (contiguous layout) or
+    block_table int32 [n_seq, max_blocks] with block_size rows per page (paged layout);
+    capacity int32 [n_seq] or None."""
+    assert seq_start is None or seq_start.dtype == torch.int64
     assert capacity is None or capacity.dtype == torch.int32
-    return Cache(_ptr(base), _ptr(seq_start), _ptr(capacity), int(base.shape[0]))
+    if block_table is not None:
+        assert block_table.dtype == torch.int32 and block_table.dim() == 2
+        return Cache(_ptr(base), _ptr(seq_start), _ptr(capacity), int(base.shape[0]), _ptr(block_table),
+                     int(block_size), int(block_table.shape[1]))
+    return Cache(_ptr(base), _ptr(seq_start), _ptr(capacity), int(base.shape[0]), None, 0, 0)
 
 
 def _stream(stream):

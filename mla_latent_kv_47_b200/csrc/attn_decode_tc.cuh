@@ -87,7 +87,8 @@ static_assert(kSmem <= 232448, "shared memory budget");
 struct AttnArgs {
   CUtensorMap map_cache;       // cache rows [n_rows x 576] bf16, box {64 columns, 32 rows}, 128B swizzle
   const __nv_bfloat16* qlat;   // [B][n_h][576]
-  const int64_t* seq_start;
+  CacheLayout lay;             // cache rows of each sequence (contiguous or paged)
+  long long n_rows;            // rows of the cache tensor
   const int32_t* seqlen;
   const int* tile_start;
   const int* seg_start;
@@ -197,22 +198,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       auto prefetch_next = [&]() {
         if (pf_g >= pf_end) return;
         while (pf_b + 1 < a.B && a.tile_start[pf_b + 1] <= pf_g) ++pf_b;
-        const long long y = a.seq_start[pf_b] + (pf_g - a.tile_start[pf_b]) * kAttnTileTokens + kHalf * rank;
-        for (int ci = 0; ci < kOwnChunks; ++ci) tma_prefetch_l2_2d(&a.map_cache, ci * 64, static_cast<int>(y));
+        const long long y = a.lay.row(pf_b, (pf_g - a.tile_start[pf_b]) * kAttnTileTokens) + kHalf * rank;
+        if (y >= 0)
+          for (int ci = 0; ci < kOwnChunks; ++ci) tma_prefetch_l2_2d(&a.map_cache, ci * 64, static_cast<int>(y));
         ++pf_g;
       };
       for (int i = kStages; i < kStages + kPrefetchAhead; ++i) prefetch_next();
       int it = 0;
       for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
         if (*abort_flag) return;
-        const long long row0 = a.seq_start[p.b];
         for (int t = p.t0; t < p.t1; ++t, ++it) {
           const int s = it % kStages;
           if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, wc)) return;
           if (it >= kStages) prefetch_next();  // tile it + kPrefetchAhead
           mbar_arrive_expect_tx(&full[s], kStageBytes);
           uint8_t* dst = stages + s * kStageBytes;
-          const long long y0 = row0 + static_cast<long long>(t) * kAttnTileTokens;
+          // a tile lies within one page; a tile without a page (a capacity
+          // fault of the call) loads rows past the tensor, which read as zero
+          long long y0 = a.lay.row(p.b, static_cast<long long>(t) * kAttnTileTokens);
+          if (y0 < 0) y0 = a.n_rows;
           const int y_own = static_cast<int>(y0 + kHalf * rank), y_peer = static_cast<int>(y0 + kHalf * peer);
           for (int ci = 0; ci < kOwnChunks; ++ci) {
             const bool shared = ci >= 4 * static_cast<int>(peer) && ci < 4 * static_cast<int>(peer) + 4;

@@ -28,13 +28,35 @@ struct Epi {
   float scale;
 };
 
+// Where the cache rows of each sequence live: contiguous from seq_start[s],
+// or, with a block table, in pages of block_size rows (a multiple of the
+// 64-token attention tile, so a tile never straddles two pages).
+struct CacheLayout {
+  const int64_t* seq_start;
+  const int32_t* block_table;  // NULL: contiguous; else [n_seq][max_blocks] page numbers
+  int block_size, max_blocks;
+
+  // Positions the layout can hold for one sequence (paged), else no limit.
+  __device__ __forceinline__ bool holds(long long p) const {
+    return !block_table || p < static_cast<long long>(max_blocks) * block_size;
+  }
+  // Row of position p of sequence s; negative when the block table has no
+  // page for it (a position past max_blocks pages, or a negative entry).
+  __device__ __forceinline__ long long row(int s, long long p) const {
+    if (!block_table) return seq_start[s] + p;
+    if (!holds(p)) return -1;
+    const long long page = block_table[static_cast<long long>(s) * max_blocks + p / block_size];
+    return page < 0 ? -1 : page * block_size + p % block_size;
+  }
+};
+
 // Where token n of a GEMM sits: its sequence, its position, its cache row.
 struct TokenMap {
   const int32_t* pos;        // position of token n, or NULL: pos_base + n
   int pos_base;
   const int32_t* seq;        // sequence of token n, or NULL: seq_const (>= 0) or n (seq_const < 0)
   int seq_const;
-  const int64_t* seq_start;  // cache row of token 0 of each sequence
+  CacheLayout lay;           // cache rows of each sequence
   const int32_t* capacity;   // NULL or rows reserved per sequence
   long long n_rows;          // rows allocated in the cache
   void* cache;
@@ -110,11 +132,11 @@ __device__ __forceinline__ void store_elem(void* base, long long idx, float v, i
 __device__ __forceinline__ long long cache_row(const TokenMap& t, int n, int* status) {
   const int s = tok_seq(t, n);
   const int p = tok_pos(t, n);
-  if (p < 0 || (t.capacity && p >= t.capacity[s])) {
+  if (p < 0 || (t.capacity && p >= t.capacity[s]) || !t.lay.holds(p)) {
     atomicOr(status, FAULT_CAPACITY);
     return -1;
   }
-  const long long row = t.seq_start[s] + p;
+  const long long row = t.lay.row(s, p);
   if (row < 0 || row >= t.n_rows) {
     atomicOr(status, FAULT_CAPACITY);
     return -1;

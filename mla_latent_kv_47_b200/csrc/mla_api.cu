@@ -30,8 +30,8 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // region is written in full by a kernel of the call before any kernel reads it.
 struct Layout {
   size_t status, gpart, base_end;
-  size_t tile_start, seg_start, rope, cq, qc, qlat, olat, o, opart, ml, decode_end;
-  size_t p_rope, p_cq, p_qp, p_rows, p_kc, p_v, p_out, prefill_end;
+  size_t tile_start, seg_start, rope, cq, qc, qlat, olat, o, opart, ml, nkv, nq, decode_end;
+  size_t p_rope, p_cq, p_qp, p_rows, p_kc, p_v, p_out, p_nkv, p_nq, prefill_end;
 };
 
 int elem_size(const mla_dims& d) { return d.dtype == MLA_FP32 ? 4 : 2; }
@@ -62,6 +62,8 @@ Layout make_layout_sized(const mla_dims& d, int max_batch, int max_tokens, int g
   L.o = take(B * nh * dh * es);
   L.opart = take((B + workers) * nh * d.d_c * sizeof(float));
   L.ml = take((B + workers) * nh * 2 * sizeof(float));
+  L.nkv = take(B * d.d_c * sizeof(float));                      // c^KV before the RMSNorm (with g_kv)
+  L.nq = take(B * (d.d_cq ? d.d_cq : 1) * sizeof(float));       // c^Q before the RMSNorm (with g_q)
   L.decode_end = off;
   off = L.base_end;
   L.p_rope = take(T * (d.d_R / 2 + 1) * 2 * sizeof(float));
@@ -71,6 +73,11 @@ Layout make_layout_sized(const mla_dims& d, int max_batch, int max_tokens, int g
   L.p_kc = take(T * nh * dh * es);
   L.p_v = take(T * nh * dh * es);
   L.p_out = take(T * nh * dh * es);
+  // the latents before the RMSNorm are consumed before K^C and V are formed,
+  // so they share those buffers when they fit
+  const size_t kv_bytes = T * nh * dh * es;
+  L.p_nq = T * d.d_cq * sizeof(float) <= kv_bytes ? L.p_kc : take(T * (d.d_cq ? d.d_cq : 1) * sizeof(float));
+  L.p_nkv = T * d.d_c * sizeof(float) <= kv_bytes ? L.p_v : take(T * d.d_c * sizeof(float));
   L.prefill_end = off;
   return L;
 }
@@ -396,13 +403,30 @@ mla_status check_weights(const mla_dims* d, const mla_weights* w) {
     if (!w->W_DQ) return MLA_ERR_INVALID_ARG;
     if (!aligned16(w->W_DQ)) return MLA_ERR_MISALIGNED;
   }
+  if (w->g_q && !d->d_cq) return MLA_ERR_INVALID_ARG;  // no c^Q to normalise without query compression
+  if ((w->g_kv && !aligned16(w->g_kv)) || (w->g_q && !aligned16(w->g_q))) return MLA_ERR_MISALIGNED;
   return MLA_OK;
 }
 
 mla_status check_cache(const mla_cache* c) {
-  if (!c || !c->base || !c->seq_start || c->n_rows <= 0) return MLA_ERR_INVALID_ARG;
+  if (!c || !c->base || c->n_rows <= 0) return MLA_ERR_INVALID_ARG;
+  if (c->block_table) {
+    if (c->block_size <= 0 || c->block_size % 64 != 0 || c->max_blocks <= 0) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(c->block_table)) return MLA_ERR_MISALIGNED;
+  } else if (!c->seq_start) {
+    return MLA_ERR_INVALID_ARG;
+  }
   if (!aligned16(c->base)) return MLA_ERR_MISALIGNED;
   return MLA_OK;
+}
+
+CacheLayout cache_layout(const mla_cache* c) {
+  CacheLayout l{};
+  l.seq_start = c->seq_start;
+  l.block_table = c->block_table;
+  l.block_size = c->block_table ? c->block_size : 0;
+  l.max_blocks = c->block_table ? c->max_blocks : 0;
+  return l;
 }
 
 enum Region { REGION_BASE, REGION_DECODE, REGION_PREFILL };
@@ -427,7 +451,7 @@ mla_status make_ctx(Ctx& c, const mla_dims* d, int max_batch, int max_tokens, Re
 
 TokenMap cache_tokens(const mla_dims& d, const mla_cache* cache) {
   TokenMap t{};
-  t.seq_start = cache->seq_start;
+  t.lay = cache_layout(cache);
   t.capacity = cache->capacity;
   t.n_rows = cache->n_rows;
   t.cache = cache->base;
@@ -490,15 +514,33 @@ float qlat_scale(const mla_dims& d) {
 }
 
 // Appends the [W_DKV; W_KR] segments (cache-row epilogues) to a dense GEMM.
-void add_cache_segments(GemmSpec& g, const mla_dims& d, const mla_weights* w) {
+// With an RMSNorm gain on c^KV the W_DKV segment leaves c^KV in fp32 at `nkv`
+// ([tokens x d_c]) for launch_latent_norm, which writes the cache rows.
+void add_cache_segments(GemmSpec& g, const mla_dims& d, const mla_weights* w, void* nkv) {
   g.A[g.nseg] = w->W_DKV;
   g.rows[g.nseg] = d.d_c;
-  g.epi[g.nseg] = epi_kind(EPI_CACHE_CKV);
+  g.epi[g.nseg] = w->g_kv ? epi_store(nkv, d.d_c, 0, 1.f, 1) : epi_kind(EPI_CACHE_CKV);
   ++g.nseg;
   g.A[g.nseg] = w->W_KR;
   g.rows[g.nseg] = d.d_R;
   g.epi[g.nseg] = epi_kind(EPI_CACHE_KR);
   ++g.nseg;
+}
+
+// RMSNorm of the latents of T tokens (no-op without gains): c^KV from `nkv`
+// into the tokens' cache rows, c^Q from `nq` into `cq_out` (storage dtype).
+mla_status launch_latent_norm(const Ctx& c, const mla_weights* w, const TokenMap& tk, int T, const void* nkv,
+                              const void* nq, void* cq_out) {
+  if (!w->g_kv && !w->g_q) return MLA_OK;
+  const float* fk = static_cast<const float*>(nkv);
+  const float* fq = static_cast<const float*>(nq);
+  if (c.d.dtype == MLA_FP32)
+    return launch(latent_norm_kernel<float>, dim3(T), dim3(256), 0, c.st, c.pdl, fk,
+                  static_cast<const float*>(w->g_kv), fq, static_cast<const float*>(w->g_q), c.d.d_cq,
+                  static_cast<float*>(cq_out), tk, c.status);
+  return launch(latent_norm_kernel<__nv_bfloat16>, dim3(T), dim3(256), 0, c.st, c.pdl, fk,
+                static_cast<const __nv_bfloat16*>(w->g_kv), fq, static_cast<const __nv_bfloat16*>(w->g_q), c.d.d_cq,
+                static_cast<__nv_bfloat16*>(cq_out), tk, c.status);
 }
 
 cudaEvent_t g_attn_begin = nullptr, g_attn_end = nullptr;  // diagnostic hook (mla_set_attention_events)
@@ -515,7 +557,8 @@ mla_status launch_attn_decode_tc(const __nv_bfloat16* qlat, const mla_cache* cac
   if (cache->n_rows > (1ll << 31) - 128) return MLA_ERR_UNSUPPORTED;  // tile rows are int32 TMA coordinates
   if (!make_map_2d(&a.map_cache, cache->base, attn::kRow, cache->n_rows, attn::kRow, attn::kHalf)) return MLA_ERR_CUDA;
   a.qlat = qlat;
-  a.seq_start = cache->seq_start;
+  a.lay = cache_layout(cache);
+  a.n_rows = cache->n_rows;
   a.seqlen = seqlen;
   a.tile_start = tile_start;
   a.seg_start = seg_start;
@@ -595,7 +638,7 @@ mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const 
     if (d.d_cq) {
       g.A[0] = w->W_DQ;
       g.rows[0] = d.d_cq;
-      g.epi[0] = epi_store(cq, d.d_cq, 0, 1.f);
+      g.epi[0] = w->g_q ? epi_store(ws + c.L.nq, d.d_cq, 0, 1.f, 1) : epi_store(cq, d.d_cq, 0, 1.f);
       g.nseg = 1;
     } else {
       g.A[0] = w->W_UQ;
@@ -606,8 +649,9 @@ mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const 
       g.epi[1] = epi_kind(EPI_QLAT_ROPE, qlat, static_cast<long long>(d.n_h) * row, row, 0, 0, qs);
       g.nseg = 2;
     }
-    add_cache_segments(g, d, w);
+    add_cache_segments(g, d, w, ws + c.L.nkv);
     if ((s = run_gemm(c, g)) != MLA_OK) return s;
+    if ((s = launch_latent_norm(c, w, tk, B, ws + c.L.nkv, ws + c.L.nq, cq)) != MLA_OK) return s;
   }
   // ---- a3: query up-projection from c^Q (+ RoPE on q^R)
   if (d.d_cq) {
@@ -663,7 +707,7 @@ mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const 
     dim3 grid(W, d.n_h);
     g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
     simt_decode_attn_kernel<float><<<grid, 128, shm, c.st>>>(
-        static_cast<const float*>(qlat), static_cast<const float*>(cache->base), cache->seq_start, seqlen,
+        static_cast<const float*>(qlat), static_cast<const float*>(cache->base), cache_layout(cache), seqlen,
         tile_start, seg_start, B, W, d.n_h, d.d_c, d.d_R, tile_tokens, opart, ml);
     if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
   }
@@ -790,7 +834,10 @@ mla_status mla_cache_append(const mla_dims* dims, const mla_weights* w, const vo
   if (!h || !seq_idx || !pos) return MLA_ERR_INVALID_ARG;
   if (!aligned16(h)) return MLA_ERR_MISALIGNED;
   Ctx c;
-  if ((s = make_ctx(c, dims, 1, 1, REGION_BASE, workspace, workspace_bytes, stream)) != MLA_OK) return s;
+  // with an RMSNorm on c^KV the raw latents of the T tokens need the prefill region
+  if ((s = make_ctx(c, dims, 1, T, w->g_kv ? REGION_PREFILL : REGION_BASE, workspace, workspace_bytes, stream)) !=
+      MLA_OK)
+    return s;
   const mla_dims& d = *dims;
   GemmSpec g;
   g.K = d.d_model;
@@ -802,8 +849,12 @@ mla_status mla_cache_append(const mla_dims* dims, const mla_weights* w, const vo
   g.tok = cache_tokens(d, cache);
   g.tok.pos = pos;
   g.tok.seq = seq_idx;
-  add_cache_segments(g, d, w);
-  return run_gemm(c, g);
+  add_cache_segments(g, d, w, c.ws + c.L.p_nkv);
+  if ((s = run_gemm(c, g)) != MLA_OK) return s;
+  if (!w->g_kv) return MLA_OK;
+  mla_weights kv_only = *w;
+  kv_only.g_q = nullptr;  // appending caches c^KV only
+  return launch_latent_norm(c, &kv_only, g.tok, T, c.ws + c.L.p_nkv, nullptr, nullptr);
 }
 
 mla_status mla_decode(const mla_dims* dims, const mla_weights* w, const void* h, int B, const mla_cache* cache,
@@ -823,14 +874,22 @@ mla_status mla_decode(const mla_dims* dims, const mla_weights* w, const void* h,
 
 namespace {
 
-template <typename T>
-__global__ void gather_rows_kernel(const T* __restrict__ cache, const int64_t* __restrict__ seq_start, int seq,
-                                   long long nrows, int row, T* __restrict__ out) {
-  const T* src = cache + seq_start[seq] * row;
-  const long long n = nrows * row;
+// Copies the first nrows cache rows of sequence `seq` (contiguous or paged)
+// into one contiguous block, 16 bytes per thread and step (row_bytes is a
+// multiple of 16).
+__global__ void gather_rows_kernel(const uint8_t* __restrict__ cache, const CacheLayout lay, int seq, long long nrows,
+                                   int row_bytes, uint8_t* __restrict__ out) {
+  const int v = row_bytes >> 4;  // 16-byte pieces per row
+  const long long n = nrows * v;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * blockDim.x)
-    out[i] = src[i];
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long r = i / v;
+    const int q = static_cast<int>(i - r * v);
+    const long long src = lay.row(seq, r);  // negative: no page (reported by the call's cache write)
+    reinterpret_cast<uint4*>(out)[i] =
+        src < 0 ? make_uint4(0, 0, 0, 0)
+                : *reinterpret_cast<const uint4*>(cache + src * row_bytes + static_cast<long long>(q) * 16);
+  }
 }
 
 }  // namespace
@@ -876,7 +935,7 @@ extern "C" mla_status mla_prefill(const mla_dims* dims, const mla_weights* w, co
     if (d.d_cq) {
       g.A[0] = w->W_DQ;
       g.rows[0] = d.d_cq;
-      g.epi[0] = epi_store(cq, d.d_cq, 0, 1.f);
+      g.epi[0] = w->g_q ? epi_store(ws + c.L.p_nq, d.d_cq, 0, 1.f, 1) : epi_store(cq, d.d_cq, 0, 1.f);
       g.nseg = 1;
     } else {
       g.A[0] = w->W_UQ;
@@ -887,8 +946,9 @@ extern "C" mla_status mla_prefill(const mla_dims* dims, const mla_weights* w, co
       g.epi[1] = epi_kind(EPI_QP_ROPE, qp, static_cast<long long>(d.n_h) * dq, dq, d.d_h, 0, qs);
       g.nseg = 2;
     }
-    add_cache_segments(g, d, w);
+    add_cache_segments(g, d, w, ws + c.L.p_nkv);
     if ((s = run_gemm(c, g)) != MLA_OK) return s;
+    if ((s = launch_latent_norm(c, w, tk, T, ws + c.L.p_nkv, ws + c.L.p_nq, cq)) != MLA_OK) return s;
   }
   // ---- p2: queries [q^C ; RoPE(q^R)] per head
   if (d.d_cq) {
@@ -911,15 +971,11 @@ extern "C" mla_status mla_prefill(const mla_dims* dims, const mla_weights* w, co
   }
   // ---- the sequence's cache rows (prefix + new) as one contiguous block
   {
-    const int blocks = std::min<long long>(4096, (static_cast<long long>(S) * row + 255) / 256);
+    const int row_bytes = row * elem_size(d);
+    const int blocks = static_cast<int>(std::min<long long>(8 * c.num_sms, (static_cast<long long>(S) * (row_bytes / 16) + 255) / 256));
     g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
-    if (d.dtype == MLA_FP32)
-      gather_rows_kernel<float><<<blocks, 256, 0, c.st>>>(static_cast<const float*>(cache->base), cache->seq_start,
-                                                          seq, S, row, static_cast<float*>(rows));
-    else
-      gather_rows_kernel<__nv_bfloat16><<<blocks, 256, 0, c.st>>>(
-          static_cast<const __nv_bfloat16*>(cache->base), cache->seq_start, seq, S, row,
-          static_cast<__nv_bfloat16*>(rows));
+    gather_rows_kernel<<<blocks, 256, 0, c.st>>>(static_cast<const uint8_t*>(cache->base), cache_layout(cache), seq, S,
+                                                 row_bytes, static_cast<uint8_t*>(rows));
     if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
   }
   // ---- p3: un-absorbed keys and values of every key token: K^C = W_UK c, V = W_UV c

@@ -177,7 +177,7 @@ __device__ __forceinline__ void for_each_piece(int w, int W, int B, const int* t
 // l = sum_j 2^(s_j - m).
 template <typename T>
 __global__ void __launch_bounds__(128) simt_decode_attn_kernel(
-    const T* __restrict__ qlat, const T* __restrict__ cache, const int64_t* __restrict__ seq_start,
+    const T* __restrict__ qlat, const T* __restrict__ cache, const CacheLayout lay,
     const int32_t* __restrict__ seqlen, const int* tile_start, const int* seg_start, int B, int W, int n_h,
     int d_c, int d_R, int tile_tokens, float* __restrict__ o_part, float* __restrict__ ml_part) {
   extern __shared__ float sm[];
@@ -194,13 +194,14 @@ __global__ void __launch_bounds__(128) simt_decode_attn_kernel(
     __syncthreads();
     const int L1 = seqlen[p.b] + 1;
     const int j0 = p.t0 * tile_tokens, j1 = min(L1, p.t1 * tile_tokens);
-    const T* base = cache + seq_start[p.b] * row;
     float m = -INFINITY, l = 0.f;
     float o[16];
     const int per = (d_c + 31) / 32;
     for (int i = 0; i < 16; ++i) o[i] = 0.f;
     for (int j = j0 + warp; j < j1; j += 4) {
-      const T* r = base + static_cast<long long>(j) * row;
+      const long long rj = lay.row(p.b, j);
+      if (rj < 0) continue;  // no page for this position (reported by the call's cache write)
+      const T* r = cache + rj * row;
       float s = 0.f;
       for (int i = lane; i < row; i += 32) s += q[i] * to_f32(r[i]);
       for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
@@ -241,6 +242,57 @@ __global__ void __launch_bounds__(128) simt_decode_attn_kernel(
       ml_part[(static_cast<long long>(p.slot) * n_h + h) * 2 + 1] = Lsum;
     }
   });
+}
+
+// ---------------------------------------------------------------- latent RMSNorm
+// RMSNorm after the compressed latents ("DeepSeek-V2 summary" (7shi.hateblo.jp)
+// §3.1.2), one block per token: c^KV, as the down-projection left it in fp32,
+// becomes x / sqrt(mean(x^2) + eps) * g_kv in the token's cache row, and c^Q
+// likewise with g_q becomes the input of the query up-projection.
+constexpr float kRmsEps = 1e-6f;
+
+__device__ __forceinline__ float block_sum_256(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();  // red may still be read by the previous call
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t += red[i];
+  return t;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) latent_norm_kernel(const float* __restrict__ ckv, const T* __restrict__ g_kv,
+                                                          const float* __restrict__ cq, const T* __restrict__ g_q,
+                                                          int d_cq, T* __restrict__ cq_out, const TokenMap tk,
+                                                          int* status) {
+  __shared__ float red[8];
+  __shared__ long long s_row;
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  const int n = blockIdx.x;
+  if (g_kv) {
+    const float* x = ckv + static_cast<long long>(n) * tk.d_c;
+    float ss = 0.f;
+    for (int c = threadIdx.x; c < tk.d_c; c += 256) ss += x[c] * x[c];
+    const float inv = rsqrtf(block_sum_256(ss, red) / tk.d_c + kRmsEps);
+    if (threadIdx.x == 0) s_row = cache_row(tk, n, status);
+    __syncthreads();
+    if (s_row >= 0) {
+      T* dst = static_cast<T*>(tk.cache) + s_row * tk.row_elems;
+      for (int c = threadIdx.x; c < tk.d_c; c += 256) dst[c] = static_cast<T>(x[c] * inv * to_f32(g_kv[c]));
+    }
+  }
+  if (g_q) {
+    const float* x = cq + static_cast<long long>(n) * d_cq;
+    float ss = 0.f;
+    for (int c = threadIdx.x; c < d_cq; c += 256) ss += x[c] * x[c];
+    const float inv = rsqrtf(block_sum_256(ss, red) / d_cq + kRmsEps);
+    T* dst = cq_out + static_cast<long long>(n) * d_cq;
+    for (int c = threadIdx.x; c < d_cq; c += 256) dst[c] = static_cast<T>(x[c] * inv * to_f32(g_q[c]));
+  }
 }
 
 // ---------------------------------------------------------------- split combine

@@ -90,6 +90,13 @@ def cache_value_check(got_bits: np.ndarray, Wh: dict, h: np.ndarray, pos: np.nda
     u = 2.0 ** -24
     h2 = np.asarray(h, np.float64) ** 2
     noise_c = np.sqrt(h2 @ (np.asarray(Wh["W_DKV"], np.float64) ** 2).T)
+    if "g_kv" in Wh:
+        # RMSNorm on c^KV: the fp32 noise of each element is divided by the
+        # row's RMS and multiplied by its gain
+        raw = np.asarray(h, np.float64) @ np.asarray(Wh["W_DKV"], np.float64).T
+        rms = np.sqrt(np.mean(raw * raw, axis=1, keepdims=True) + 1e-6)
+        g = np.abs(np.asarray(Wh["g_kv"], np.float64))[None, :]
+        noise_c = noise_c * g / rms
     pre_r = np.asarray(h, np.float64) @ np.asarray(Wh["W_KR"], np.float64).T
     noise_r = np.sqrt(h2 @ (np.asarray(Wh["W_KR"], np.float64) ** 2).T)
     pair = noise_r.reshape(noise_r.shape[0], -1, 2).sum(-1).repeat(2, axis=1)
@@ -97,4 +104,8 @@ def cache_value_check(got_bits: np.ndarray, Wh: dict, h: np.ndarray, pos: np.nda
     acc = 16.0 * np.sqrt(K) * u * np.concatenate([noise_c, pair], axis=1)
     rot = np.concatenate([np.zeros_like(noise_c), 8 * u * pair_mag], axis=1)
     bound = 2.0 ** -8 * np.abs(exact) + (1 + 2.0 ** -8) * acc + rot
+    if "g_kv" in Wh:
+        # the norm's own fp32 arithmetic (a sum of squares over d_c, rsqrt, two
+        # products) and the noise of the RMS itself: well under 2^-14 relative
+        bound[:, :c_kv.shape[1]] += 2.0 ** -14 * np.abs(c_kv)
     return float(np.max(np.abs(got - exact) / bound))

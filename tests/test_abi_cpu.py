@@ -164,3 +164,27 @@ def test_yarn_arguments_are_checked(m):
     d = m.make_dims(synth.PRESETS["v2"].dims)
     d.yarn_s, d.yarn_alpha, d.yarn_beta, d.yarn_L0 = 40.0, 1.0, 32.0, 4096.0
     assert m.workspace_bytes(d, 4, 4) > 0
+
+
+def test_paged_cache_arguments_are_checked(m):
+    """A block table needs block_size a positive multiple of 64 and
+    max_blocks > 0; without one, seq_start is required."""
+    import synth
+    A = 1 << 20
+    W = m.Weights(*[A] * 8, None, None)
+    dims = m.make_dims(synth.PRESETS["v2"].dims)
+    assert _call_decode(m, dims, W, A, 4, m.Cache(A, None, None, 1000, None, 0, 0), A, A, A, 1 << 40) == -1
+    for bs, mb in ((0, 4), (96, 4), (64, 0), (-64, 4)):
+        assert _call_decode(m, dims, W, A, 4, m.Cache(A, None, None, 1000, A, bs, mb), A, A, A, 1 << 40) == -1, (bs, mb)
+    assert _call_decode(m, dims, W, A, 4, m.Cache(A, None, None, 1000, A + 4, 64, 4), A, A, A, 1 << 40) == -3
+
+
+def test_rmsnorm_gain_arguments_are_checked(m):
+    """g_q needs query compression; gains must be 16-byte aligned."""
+    import synth
+    A = 1 << 20
+    C = m.Cache(A, A, None, 1000, None, 0, 0)
+    lite = m.make_dims(synth.PRESETS["lite"].dims)
+    assert _call_decode(m, lite, m.Weights(*[A] * 8, None, A), A, 4, C, A, A, A, 1 << 40) == -1
+    v2 = m.make_dims(synth.PRESETS["v2"].dims)
+    assert _call_decode(m, v2, m.Weights(*[A] * 8, A + 2, None), A, 4, C, A, A, A, 1 << 40) == -3

@@ -27,12 +27,13 @@ def m():
 
 
 def run_decode(m, preset, checked, lengths=None, pad=2, oracle="unabsorbed", dirty_workspace=False, h_scale=None,
-               dims=None, weights=None):
+               dims=None, weights=None, chunk=None):
     """Fills a poisoned cache through mla_cache_append, runs one mla_decode and
     checks layout, cache rows and u.  `dims` replaces the preset's dims (same
     shapes, e.g. with YaRN on); `weights` (host, device) replaces its weights.
     `oracle` names the fp64 form u is compared with, per sequence when it is a
-    callable of the sequence's length."""
+    callable of the sequence's length.  `chunk`: tokens per mla_cache_append
+    call, with a workspace sized for them (the latent RMSNorm needs it)."""
     from mla_latent_kv_47_b200.cache import LatentCache
     p = synth.preset(preset)
     d = p.dims if dims is None else dims
@@ -41,14 +42,14 @@ def run_decode(m, preset, checked, lengths=None, pad=2, oracle="unabsorbed", dir
     B = len(L)
     Wh, Wd = gu.device_weights(p) if weights is None else weights
     cache = LatentCache(dims, [x + 1 + pad for x in L], poison=True, gap=1)
-    ws = m.alloc_workspace(dims, B, 1)
+    ws = m.alloc_workspace(dims, B, chunk or 1)
     if dirty_workspace:
         ws.fill_(0xFF)      # NaN floats, -1 counters: nothing may be read before it is written
         ws[:256].zero_()    # except the status word, zeroed once by contract
     seqs_h = {b: synth.hidden(p, b, L[b] + 1) for b in checked}
     if h_scale is not None:   # per-token scale of the checked sequences (powers of two keep bf16 values exact)
         seqs_h = {b: h * h_scale(np.arange(h.shape[0]))[:, None].astype(h.dtype) for b, h in seqs_h.items()}
-    gu.fill_cache(m, dims, Wd, cache, ws, seqs_h, L, p)
+    gu.fill_cache(m, dims, Wd, cache, ws, seqs_h, L, p, chunk=chunk or 32768)
     tdt = torch.float32 if d.dtype == "fp32" else torch.bfloat16
     g = torch.Generator(device="cuda")
     g.manual_seed(99)

@@ -106,3 +106,19 @@ def test_planted_mistake_is_caught(name, monkeypatch):
     monkeypatch.setattr(om, "rmsnorm", MUTANTS[name])
     with pytest.raises(AssertionError):
         test_rmsnorm_matches_brute_force()
+
+
+def test_gains_move_v2_decode_by_more_than_the_gpu_gate():
+    """At DeepSeek-V2 dims, RMSNorm with gains in [0.5, 1.5) changes u by
+    several times the GPU parity gate (1e-2 of max|u|), so the GPU RMSNorm
+    tests cannot pass with the norm skipped."""
+    import synth
+    p = synth.preset("v2")
+    W = synth.weights(p)
+    rng = np.random.default_rng(17)
+    Wg = dict(W, g_kv=synth.round_bf16((0.5 + rng.random(p.dims.d_c)).astype(np.float32)),
+              g_q=synth.round_bf16((0.5 + rng.random(p.dims.d_cq)).astype(np.float32)))
+    h = synth.hidden(p, 2, 700)
+    a = om.decode_absorbed(Wg, h, p.dims)
+    b = om.decode_absorbed(W, h, p.dims)
+    assert np.max(np.abs(a - b)) > 5e-2 * np.max(np.abs(a))
