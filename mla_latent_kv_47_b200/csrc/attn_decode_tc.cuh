@@ -71,7 +71,6 @@ constexpr int kQChunkBytes = 128 * 128;                // 128 heads x 64 columns
 constexpr int kPBytes = 128 * 128;                     // P: 128 heads x 64 rows, bf16 (CTA 0's rows first)
 constexpr int kPBufs = 2;
 constexpr int kMaxSlots = 4;                           // partner tile maxima in flight (tile j in slot j % 4)
-constexpr int kPrefetchAhead = 6;                      // tiles brought into L2 ahead of their TMA load
 constexpr int kAuxBytes = 3072;                        // partner maxima, CTA 1's l, barriers
 // stages | Q chunks 7-8 | P x 2 | aux
 constexpr int kSmem = 1024 + kStages * kStageBytes + kQSmemChunks * kQChunkBytes + kPBufs * kPBytes + kAuxBytes;
@@ -173,50 +172,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       // second read is an L2 hit; the rest is streamed with evict-first.
       const uint64_t pol_once = policy_evict_first();
       const uint64_t pol_twice = policy_evict_normal();
-      // A stage is held from its load until the tile's PV retires, so the
-      // ring alone keeps about one tile per CTA in flight from HBM.  This CTA's
-      // rows of the tiles kPrefetchAhead ahead are therefore pulled into L2
-      // first (the partner pulls its own rows, which this CTA also reads), and
-      // the ring's loads find them there.  Cursor: next worker tile to
-      // prefetch, as a global tile index and its sequence.
-      long long pf_g = 0, pf_end = 0;
-      int pf_b = 0;
-      {
-        const long long Tt = a.tile_start[a.B];
-        const int We = static_cast<int>(Tt < a.W ? Tt : a.W);
-        if (Tt > 0 && w < We) {
-          pf_g = worker_begin(w, Tt, We) + kStages;  // the first kStages tiles are loaded at once
-          pf_end = worker_begin(w + 1, Tt, We);
-          int lo = 0, hi = a.B - 1;                  // sequence of tile pf_g
-          while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (a.tile_start[mid + 1] > pf_g) hi = mid; else lo = mid + 1;
-          }
-          pf_b = lo;
-        }
-      }
-      auto prefetch_next = [&]() {
-        if (pf_g >= pf_end) return;
-        while (pf_b + 1 < a.B && a.tile_start[pf_b + 1] <= pf_g) ++pf_b;
-        const long long y = a.lay.row(pf_b, (pf_g - a.tile_start[pf_b]) * kAttnTileTokens) + kHalf * rank;
-        if (y >= 0)
-          for (int ci = 0; ci < kOwnChunks; ++ci) tma_prefetch_l2_2d(&a.map_cache, ci * 64, static_cast<int>(y));
-        ++pf_g;
-      };
-      for (int i = kStages; i < kStages + kPrefetchAhead; ++i) prefetch_next();
       int it = 0;
       for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
         if (*abort_flag) return;
+        const long long row0 = a.lay.block_table ? 0 : a.lay.seq_start[p.b];  // contiguous layout
         for (int t = p.t0; t < p.t1; ++t, ++it) {
           const int s = it % kStages;
-          if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, wc)) return;
-          if (it >= kStages) prefetch_next();  // tile it + kPrefetchAhead
-          mbar_arrive_expect_tx(&full[s], kStageBytes);
-          uint8_t* dst = stages + s * kStageBytes;
           // a tile lies within one page; a tile without a page (a capacity
           // fault of the call) loads rows past the tensor, which read as zero
-          long long y0 = a.lay.row(p.b, static_cast<long long>(t) * kAttnTileTokens);
+          long long y0 = a.lay.block_table ? a.lay.row(p.b, static_cast<long long>(t) * kAttnTileTokens)
+                                           : row0 + static_cast<long long>(t) * kAttnTileTokens;
           if (y0 < 0) y0 = a.n_rows;
+          if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, wc)) return;
+          mbar_arrive_expect_tx(&full[s], kStageBytes);
+          uint8_t* dst = stages + s * kStageBytes;
           const int y_own = static_cast<int>(y0 + kHalf * rank), y_peer = static_cast<int>(y0 + kHalf * peer);
           for (int ci = 0; ci < kOwnChunks; ++ci) {
             const bool shared = ci >= 4 * static_cast<int>(peer) && ci < 4 * static_cast<int>(peer) + 4;
