@@ -86,18 +86,20 @@ def workload_config(args, world):
 
 
 def decode_flops_bytes(d, L):
-    """Algorithmic FLOPs and HBM bytes of one decode step (bf16 storage)."""
+    """Algorithmic FLOPs and HBM bytes of one decode step (bf16 weights; the
+    cache rows in their format: bf16, or E4M3 c^KV + bf16 k^R + 16 bytes)."""
     B = len(L)
     ctx = sum(x + 1 for x in L)
     row = d.d_c + d.d_R
+    row_bytes = d.d_c + 2 * d.d_R + 16 if getattr(d, "cache", "dtype") == "e4m3" else row * 2
     qin = d.d_cq if d.d_cq else d.d_model
     wrows = {
         "W_DQ": (d.d_cq, d.d_model), "W_UQ": (d.n_h * d.d_h, qin), "W_QR": (d.n_h * d.d_R, qin),
         "W_DKV": (d.d_c, d.d_model), "W_KR": (d.d_R, d.d_model), "W_UK": (d.n_h * d.d_h, d.d_c),
         "W_UV": (d.n_h * d.d_h, d.d_c), "W_O": (d.d_model, d.n_h * d.d_h)}
     welem = sum(a * b for a, b in wrows.values())
-    cache_bytes = ctx * row * 2
-    bytes_total = cache_bytes + welem * 2 + B * d.d_model * (2 + 4) + B * row * 2
+    cache_bytes = ctx * row_bytes
+    bytes_total = cache_bytes + welem * 2 + B * d.d_model * (2 + 4) + B * row_bytes
     attn_flops = ctx * d.n_h * (2 * row + 2 * d.d_c)
     flops = attn_flops + 2 * welem * B
     return flops, bytes_total, cache_bytes, attn_flops
@@ -290,13 +292,14 @@ class DecodeSetup:
     N(0,0.02) bf16 weights, a latent cache filled through mla_cache_append
     from N(0,1) hidden states, the new tokens' hidden states and seqlen."""
 
-    def __init__(self, m, dev, g, name, ctx=0, batch=0):
+    def __init__(self, m, dev, g, name, ctx=0, batch=0, cache="dtype"):
+        import dataclasses
         import torch
         from mla_latent_kv_47_b200.cache import LatentCache
         from synth import weight_shapes
         self.m = m
         self.p, self.L = workload_lengths(name, ctx, batch)
-        d = self.p.dims
+        d = self.d = dataclasses.replace(self.p.dims, cache=cache)
         self.dims = m.make_dims(d)
         self.B = len(self.L)
         self.Wd = {k: (torch.randn(s, generator=g, device=dev) * 0.02).to(torch.bfloat16)
@@ -305,18 +308,21 @@ class DecodeSetup:
         self.cache = LatentCache(self.dims, [x + 1 for x in self.L], device=dev)
         self.ws = m.alloc_workspace(self.dims, self.B, 1, device=dev)
         chunk = 16384
+        # E4M3 rows are encoded from the fp32 latents, which need room for a chunk of tokens
+        fill_ws = m.alloc_workspace(self.dims, self.B, chunk, device=dev) if cache == "e4m3" else self.ws
         for b, n in enumerate(self.L):
             for t0 in range(0, n, chunk):
                 k = min(chunk, n - t0)
                 h = torch.randn((k, d.d_model), generator=g, device=dev).to(torch.bfloat16)
                 m.cache_append(self.dims, self.wts, h, torch.full((k,), b, dtype=torch.int32, device=dev),
-                               torch.arange(t0, t0 + k, dtype=torch.int32, device=dev), self.cache.handle, self.ws)
+                               torch.arange(t0, t0 + k, dtype=torch.int32, device=dev), self.cache.handle, fill_ws)
         self.h_new = torch.randn((self.B, d.d_model), generator=g, device=dev).to(torch.bfloat16)
         self.seqlen = torch.tensor(self.L, dtype=torch.int32, device=dev)
         self.u = torch.empty((self.B, d.d_model), dtype=torch.float32, device=dev)
         torch.cuda.synchronize()
-        code, detail = m.device_status(self.ws)
+        code, detail = m.device_status(fill_ws)
         assert code == 0, ("cache fill fault", code, detail)
+        del fill_ws
 
     def step(self):
         self.m.decode(self.dims, self.wts, self.h_new, self.cache.handle, self.seqlen, self.u, self.ws)
@@ -509,20 +515,21 @@ def run_ours(args):
         del pc, wsp, hp, up, Wd
         torch.cuda.empty_cache()
 
-    # ---- the other decode workloads (secondary objects of the same line)
+    # ---- the other decode workloads (secondary objects of the same line):
+    # V2-Lite, ragged long context, and the V2 workload over an E4M3 cache
     others = {}
     if args.workload == "v2" and not args.ctx and not args.batch and not args.no_secondary:
-        for name in ("lite", "ragged"):
-            So = DecodeSetup(m, dev, g, name)
+        for key, name, fmt in (("lite", "lite", "dtype"), ("ragged", "ragged", "dtype"), ("e4m3", "v2", "e4m3")):
+            So = DecodeSetup(m, dev, g, name, cache=fmt)
             for _ in range(5):
                 So.step()
             torch.cuda.synchronize()
             K2 = max(10, min(K, 200))
             oms, oattn, _ = time_steps(m, So.step, K2, barrier)
             So.check()
-            others[name] = decode_summary(So.p.dims, So.L, max_over_ranks(oms), max_over_ranks(oattn), world,
-                                          hbm_gbs, bf16_tf)
-            others[name]["steps"] = K2
+            others[key] = decode_summary(So.d, So.L, max_over_ranks(oms), max_over_ranks(oattn), world,
+                                         hbm_gbs, bf16_tf)
+            others[key]["steps"] = K2
             del So
             torch.cuda.empty_cache()
 
@@ -560,6 +567,7 @@ def run_ours(args):
         "prefill": prefill,
         "lite": others.get("lite"),
         "ragged": others.get("ragged"),
+        "v2_e4m3_cache": others.get("e4m3"),
     }
     print(json.dumps(line), flush=True)
     if world > 1:

@@ -26,8 +26,9 @@
  *  - RoPE rotates interleaved pairs (2m, 2m+1) by pos * rope_base^(-2m/d_R);
  *    pos is the token's 0-based index in its sequence.
  *  - Cache row of a token: [c^KV (d_c) | RoPE'd k^R (d_R)], dtype
- *    `mla_dims.dtype`, row stride (d_c + d_R) elements, contiguous per sequence:
- *    token p of sequence s lives in row seq_start[s] + p.
+ *    `mla_dims.dtype`, row stride (d_c + d_R) elements (or the E4M3 row of
+ *    `mla_cache_format`), contiguous per sequence (token p of sequence s in
+ *    row seq_start[s] + p) or paged through a block table.
  *  - All pointers except the structs themselves are device pointers owned by
  *    the caller.  The library allocates nothing and keeps no state between
  *    calls (apart from the diagnostic timing hook at the end of this file).
@@ -95,7 +96,25 @@ typedef struct {
      * beta = 32 and a 4K pre-training length.  Requires yarn_beta > yarn_alpha
      * >= 0 and yarn_L0 > 0. */
     double yarn_s, yarn_alpha, yarn_beta, yarn_L0;
+    /* mla_cache_format of the latent cache (0 = storage dtype rows). */
+    int cache_format;
 } mla_dims;
+
+/* Latent cache row formats.
+ *  MLA_CACHE_DTYPE: [c^KV (d_c) | k^R (d_R)] in the storage dtype; row stride
+ *    (d_c + d_R) elements.
+ *  MLA_CACHE_E4M3: the low-bit cache of DeepSeek-V2 summary §3.2.3 (about 6
+ *    bits per element there; FP8 here, the serving example's format family):
+ *    bytes [0, d_c) c^KV as OCP E4M3 codes, [d_c, d_c + 2 d_R) k^R in bf16,
+ *    byte d_c + 2 d_R the row's scale exponent k (int8), then zeros to
+ *    d_c + 2 d_R + 16 (the row stride, 656 bytes at DeepSeek-V2 dims against
+ *    1152 for bf16).  Element j of c^KV is code_value * 2^k, with k the
+ *    smallest integer for which max_j |c^KV_j| / 2^k <= 448 (the largest E4M3
+ *    value; k = 0 for an all-zero row), and the code the E4M3 value nearest
+ *    to c^KV_j / 2^k, ties to even.  bf16 storage only; mla_prefill does not
+ *    take it (MLA_ERR_UNSUPPORTED) — fill such a cache with mla_cache_append
+ *    and mla_decode. */
+typedef enum { MLA_CACHE_DTYPE = 0, MLA_CACHE_E4M3 = 1 } mla_cache_format;
 
 typedef struct {
     const void* W_DQ;  /* [d_cq x d]; ignored when d_cq == 0 */
@@ -186,12 +205,15 @@ mla_status mla_get_device_status(void* workspace, mla_stream_t stream, int* deta
 const char* mla_status_string(mla_status s);
 
 /* Byte offset inside the workspace of an intermediate left by the last
- * mla_decode call with batch `max_batch` (`max_tokens` is ignored), for
- * inspection in tests.  All are in the storage dtype: 0 = c^Q [B x d_cq],
+ * mla_decode call with batch `max_batch` (ids 0-4) or by the last
+ * mla_cache_append / mla_prefill call of up to `max_tokens` tokens (id 5),
+ * for inspection in tests.  0-4 are in the storage dtype: 0 = c^Q [B x d_cq],
  * 1 = q^C [B x n_h d_h], 2 = Q_lat [B x n_h x (d_c+d_R)] = [W_UK_i^T q^C_i ; q^R_i]
  * pre-multiplied by log2(e)/sqrt(d_h+d_R), 3 = O_lat [B x n_h x d_c]
- * (normalised latent output), 4 = o [B x n_h d_h].  Returns (size_t)-1 for an
- * unknown id or invalid dims. */
+ * (normalised latent output), 4 = o [B x n_h d_h].  5 = c^KV of the tokens
+ * in fp32 [T x d_c] as the down-projection produced it, before the RMSNorm
+ * and the E4M3 encoding (written only when one of them is on).  Returns
+ * (size_t)-1 for an unknown id or invalid dims. */
 size_t mla_workspace_offset(const mla_dims* dims, int max_batch, int max_tokens, int which);
 
 /* ---------------------------------------------------------------------------

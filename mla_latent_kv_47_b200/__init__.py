@@ -16,10 +16,11 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libmla_b200.so")
 
 MLA_BF16, MLA_FP32 = 0, 1
+CACHE_DTYPE, CACHE_E4M3 = 0, 1
 STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3: "MLA_ERR_MISALIGNED",
           -4: "MLA_ERR_WORKSPACE", -5: "MLA_ERR_CUDA", -6: "MLA_ERR_DEVICE_FAULT"}
 FAULT_CAPACITY, FAULT_WAIT_TIMEOUT, FAULT_PLAN, FAULT_RANGE = 1, 2, 4, 8
-WS_CQ, WS_QC, WS_QLAT, WS_OLAT, WS_O = range(5)
+WS_CQ, WS_QC, WS_QLAT, WS_OLAT, WS_O, WS_CKV_RAW = range(6)
 
 EXPORTS = ("mla_workspace_bytes", "mla_cache_append", "mla_decode", "mla_prefill",
            "mla_get_device_status", "mla_status_string", "mla_workspace_offset", "mla_set_attention_events",
@@ -36,7 +37,7 @@ class Dims(ctypes.Structure):
     _fields_ = [("d_model", ctypes.c_int), ("n_h", ctypes.c_int), ("d_h", ctypes.c_int), ("d_R", ctypes.c_int),
                 ("d_c", ctypes.c_int), ("d_cq", ctypes.c_int), ("rope_base", ctypes.c_double),
                 ("dtype", ctypes.c_int), ("yarn_s", ctypes.c_double), ("yarn_alpha", ctypes.c_double),
-                ("yarn_beta", ctypes.c_double), ("yarn_L0", ctypes.c_double)]
+                ("yarn_beta", ctypes.c_double), ("yarn_L0", ctypes.c_double), ("cache_format", ctypes.c_int)]
 
 
 WEIGHT_FIELDS = ("W_DQ", "W_UQ", "W_QR", "W_DKV", "W_UK", "W_UV", "W_KR", "W_O", "g_kv", "g_q")
@@ -107,8 +108,16 @@ def make_dims(d) -> Dims:
     """ctypes dims from any object with the fields of synth.Dims (and, for
     YaRN, a `yarn` = (s, alpha, beta, L0) attribute)."""
     y = getattr(d, "yarn", None) or (0.0, 0.0, 0.0, 0.0)
+    fmt = {"dtype": CACHE_DTYPE, "e4m3": CACHE_E4M3}[getattr(d, "cache", "dtype")]
     return Dims(d.d_model, d.n_h, d.d_h, d.d_R, d.d_c, d.d_cq, float(d.rope_base),
-                MLA_FP32 if getattr(d, "dtype", "bf16") == "fp32" else MLA_BF16, *[float(v) for v in y])
+                MLA_FP32 if getattr(d, "dtype", "bf16") == "fp32" else MLA_BF16, *[float(v) for v in y], fmt)
+
+
+def cache_row_bytes(dims: Dims) -> int:
+    """Bytes of one cache row (the layouts of mla_cache_format)."""
+    if dims.cache_format == CACHE_E4M3:
+        return dims.d_c + 2 * dims.d_R + 16
+    return (dims.d_c + dims.d_R) * (4 if dims.dtype == MLA_FP32 else 2)
 
 
 def _ptr(t):
@@ -152,6 +161,11 @@ def workspace_bytes(dims: Dims, max_batch: int, max_tokens: int) -> int:
 
 def workspace_offset(dims: Dims, batch: int, which: int) -> int:
     return int(_lib().mla_workspace_offset(ctypes.byref(dims), int(batch), 0, int(which)))
+
+
+def workspace_offset_tokens(dims: Dims, max_tokens: int, which: int) -> int:
+    """Offset of an append / prefill intermediate (WS_CKV_RAW) for up to max_tokens tokens."""
+    return int(_lib().mla_workspace_offset(ctypes.byref(dims), 1, int(max_tokens), int(which)))
 
 
 def alloc_workspace(dims: Dims, max_batch: int, max_tokens: int, device="cuda") -> torch.Tensor:

@@ -1,24 +1,41 @@
 """Contiguous per-sequence latent cache on the device (allocation and bookkeeping).
 
-Row layout per token: [c^KV (d_c) | k^R (d_R)] in the storage dtype; sequence s
-owns rows [seq_start[s], seq_start[s] + capacity[s]).  Writes go through the
+Row layout per token: [c^KV (d_c) | k^R (d_R)] in the storage dtype, or the
+E4M3 row of mla_cache_format (bytes); sequence s owns rows
+[seq_start[s], seq_start[s] + capacity[s]).  Writes go through the
 library (mla_cache_append / mla_decode / mla_prefill).
 """
 from __future__ import annotations
 
 import torch
 
-from . import make_cache, MLA_FP32
+from . import make_cache, MLA_FP32, CACHE_E4M3, cache_row_bytes
 
 POISON_BF16 = 0x7FC1          # a quiet NaN; rows never written keep this pattern
 POISON_FP32 = 0x7FC00001
+POISON_BYTE = 0x7F            # E4M3 rows: a NaN code (and a NaN-free pattern elsewhere)
+
+
+def _row_storage(dims):
+    """(torch dtype, elements per row) of a cache row of these dims."""
+    if dims.cache_format == CACHE_E4M3:
+        return torch.uint8, cache_row_bytes(dims)
+    return (torch.float32 if dims.dtype == MLA_FP32 else torch.bfloat16), dims.d_c + dims.d_R
+
+
+def _poison(data):
+    if data.dtype == torch.bfloat16:
+        data.view(torch.int16).fill_(POISON_BF16)
+    elif data.dtype == torch.uint8:
+        data.fill_(POISON_BYTE)
+    else:
+        data.view(torch.int32).fill_(POISON_FP32)
 
 
 class LatentCache:
     def __init__(self, dims, capacities, device="cuda", poison=False, gap=0):
         self.dims = dims
-        self.dtype = torch.float32 if dims.dtype == MLA_FP32 else torch.bfloat16
-        self.row = dims.d_c + dims.d_R
+        self.dtype, self.row = _row_storage(dims)
         caps = [int(c) for c in capacities]
         starts, s = [], 0
         for c in caps:
@@ -33,10 +50,7 @@ class LatentCache:
         self.handle = make_cache(self.data, self.seq_start, self.capacity)
 
     def poison_(self):
-        if self.dtype == torch.bfloat16:
-            self.data.view(torch.int16).fill_(POISON_BF16)
-        else:
-            self.data.view(torch.int32).fill_(POISON_FP32)
+        _poison(self.data)
 
     def rows_of(self, seq, n):
         s = int(self.seq_start[seq].item())
@@ -56,8 +70,7 @@ class PagedLatentCache:
     def __init__(self, dims, capacities, block_size=64, device="cuda", poison=False, spare_pages=0,
                  page_order=None):
         self.dims = dims
-        self.dtype = torch.float32 if dims.dtype == MLA_FP32 else torch.bfloat16
-        self.row = dims.d_c + dims.d_R
+        self.dtype, self.row = _row_storage(dims)
         self.block_size = int(block_size)
         caps = [int(c) for c in capacities]
         need = [(c + self.block_size - 1) // self.block_size for c in caps]
@@ -82,10 +95,7 @@ class PagedLatentCache:
                                  block_size=self.block_size)
 
     def poison_(self):
-        if self.dtype == torch.bfloat16:
-            self.data.view(torch.int16).fill_(POISON_BF16)
-        else:
-            self.data.view(torch.int32).fill_(POISON_FP32)
+        _poison(self.data)
 
     def row_of(self, seq, p):
         return self.table_host[seq][p // self.block_size] * self.block_size + p % self.block_size

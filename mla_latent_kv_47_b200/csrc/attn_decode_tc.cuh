@@ -58,13 +58,10 @@ constexpr int kAttnTileTokens = 64;
 constexpr bool kAttnTcReady = true;
 
 namespace attn {
-constexpr int kStages = 3;
 constexpr int kThreads = 448;
 constexpr int kHalf = 32;                              // rows of a tile whose scores one CTA computes
 constexpr int kChunkBytes = kHalf * 128;               // 32 token rows x 64 latent columns, bf16, 128B swizzle
-constexpr int kOwnChunks = 9;                          // own rows: all 576 columns
 constexpr int kPeerChunks = 4;                         // partner's rows: this CTA's 256 c^KV columns
-constexpr int kStageBytes = (kOwnChunks + kPeerChunks) * kChunkBytes;
 constexpr int kQTmemChunks = 7;                        // Q chunks held in TMEM; the rest in shared memory
 constexpr int kQSmemChunks = 9 - kQTmemChunks;
 constexpr int kQChunkBytes = 128 * 128;                // 128 heads x 64 columns, bf16
@@ -72,19 +69,45 @@ constexpr int kPBytes = 128 * 128;                     // P: 128 heads x 64 rows
 constexpr int kPBufs = 2;
 constexpr int kMaxSlots = 4;                           // partner tile maxima in flight (tile j in slot j % 4)
 constexpr int kAuxBytes = 3072;                        // partner maxima, CTA 1's l, barriers
-// stages | Q chunks 7-8 | P x 2 | aux
-constexpr int kSmem = 1024 + kStages * kStageBytes + kQSmemChunks * kQChunkBytes + kPBufs * kPBytes + kAuxBytes;
 // TMEM columns: O half [0,256), S [256,288), Q chunks 0-6 (bf16 pairs) [288,512)
 constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 288, kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;
 constexpr float kRangeLog2 = 96.f;                     // largest exponent of P before the max catches up
 constexpr int kRow = 576;                              // d_c + d_R
 static_assert(kTmemQ + kQTmemChunks * 32 == kTmemCols, "TMEM budget");
-static_assert(kSmem <= 232448, "shared memory budget");
+
+// Stage layouts of the two cache formats.  The MMAs always read bf16 stages:
+// own rows' c^KV chunks 0-7 (and, for bf16 rows, the k^R chunk 8), then the
+// partner rows' chunks in this CTA's c^KV columns.  For E4M3 rows the TMA
+// fills a raw stage (k^R chunk in bf16 with the 128B swizzle, the own rows'
+// 512 code bytes as two boxes of 256, the partner rows' 256 code bytes in
+// this CTA's columns, and the scale bytes of both), and the converter warps
+// decode it into the bf16 stage; the S MMAs take k^R from the raw stage.
+template <bool kFp8>
+struct Cfg {
+  static constexpr int kStages = kFp8 ? 2 : 3;           // bf16 stages
+  static constexpr int kOwnChunks = kFp8 ? 8 : 9;        // own-row chunks in a bf16 stage
+  static constexpr int kStageBytes = (kOwnChunks + kPeerChunks) * kChunkBytes;
+  static constexpr int kRawStages = kFp8 ? 2 : 0;
+  // raw stage: k^R chunk | own codes 0-255 | own codes 256-511 | partner codes | own scales | partner scales
+  static constexpr int kRawKr = 0, kRawOwn0 = 4096, kRawOwn1 = 4096 + 8192, kRawPeer = 4096 + 2 * 8192;
+  static constexpr int kRawOwnS = 4096 + 3 * 8192, kRawPeerS = kRawOwnS + 512;
+  static constexpr int kRawTx = kRawPeerS + 512;         // bytes the TMA brings per raw stage
+  static constexpr int kRawBytes = kFp8 ? 30720 : 0;     // rounded up to 1 KB (the swizzled chunk's alignment)
+  // bf16 stages | raw stages | Q chunks 7-8 | P x 2 | aux
+  static constexpr int kSmem = 1024 + kStages * kStageBytes + kRawStages * kRawBytes + kQSmemChunks * kQChunkBytes +
+                               kPBufs * kPBytes + kAuxBytes;
+  static_assert(kSmem <= 232448, "shared memory budget");
+  static_assert(!kFp8 || kRawTx <= kRawBytes, "raw stage");
+};
 }  // namespace attn
 
 struct AttnArgs {
-  CUtensorMap map_cache;       // cache rows [n_rows x 576] bf16, box {64 columns, 32 rows}, 128B swizzle
+  CUtensorMap map_cache;       // bf16 view of the rows, box {64 columns, 32 rows}, 128B swizzle (E4M3 rows: k^R only)
+  CUtensorMap map_code;        // E4M3 rows: bytes, box {256, 32}, no swizzle
+  CUtensorMap map_scale;       // E4M3 rows: bytes, box {16, 32} at the scale byte, no swizzle
+  int kr_x;                    // E4M3 rows: k^R's column in the bf16 view (d_c / 2)
+  int scale_x;                 // E4M3 rows: byte of the scale exponent
   const __nv_bfloat16* qlat;   // [B][n_h][576]
   CacheLayout lay;             // cache rows of each sequence (contiguous or paged)
   long long n_rows;            // rows of the cache tensor
@@ -97,13 +120,36 @@ struct AttnArgs {
   int* status;
 };
 
+// Decodes 8 E4M3 codes scaled by 2^k into 8 bf16 (exact: a code value times
+// a power of two fits bf16's 8-bit significand).
+__device__ __forceinline__ uint4 e4m3x8_to_bf16(uint2 raw, float scale) {
+  uint32_t out[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t word = i < 2 ? raw.x : raw.y;
+    const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((word >> (16 * (i & 1))) & 0xFFFFu);
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+    const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * scale, f.y * scale);
+    out[i] = *reinterpret_cast<const uint32_t*>(&b);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+template <bool kFp8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     attn_decode_tc_kernel(const __grid_constant__ AttnArgs a) {
   using namespace attn;
+  using C = Cfg<kFp8>;
+  constexpr int kStages = C::kStages;
+  constexpr int kOwnChunks = C::kOwnChunks;
+  constexpr int kStageBytes = C::kStageBytes;
+  constexpr int kRS = C::kRawStages > 0 ? C::kRawStages : 1;  // raw-stage modulus (unused for bf16 rows)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* stages = smem;
-  uint8_t* qs = stages + kStages * kStageBytes;       // Q chunks 7-8, MMA A operand
+  uint8_t* raws = stages + kStages * kStageBytes;     // E4M3 rows: raw stages (TMA)
+  uint8_t* qs = raws + C::kRawStages * C::kRawBytes;  // Q chunks 7-8, MMA A operand
   uint8_t* pbuf = qs + kQSmemChunks * kQChunkBytes;   // [2] P (bf16), MMA A operand
   uint8_t* aux = pbuf + kPBufs * kPBytes;
   float* mx = reinterpret_cast<float*>(aux);          // [4][128] the partner's tile maxima (st.async)
@@ -121,7 +167,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   uint64_t* o_done = q_free + 1;
   uint64_t* l_full = o_done + 1;       // CTA 0: CTA 1's l of the piece landed
   uint64_t* drain = l_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* raw_full = drain + 1;      // [2] E4M3 rows: raw stage loaded (TMA)
+  uint64_t* raw_empty = raw_full + 2;  // [2] E4M3 rows: raw stage read by the converter and by S's k^R MMAs
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(raw_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t rank = cluster_ctarank();
@@ -131,8 +179,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], kFp8 ? 4 : 1);  // E4M3 rows: one arrival per converter warp
       mbar_init(&empty[s], 1);
+    }
+    for (int r = 0; r < C::kRawStages; ++r) {
+      mbar_init(&raw_full[r], 1);
+      mbar_init(&raw_empty[r], 5);        // four converter warps and the commit after S
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 8);        // one arrival per softmax warp
@@ -153,7 +205,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     for (int i = 0; i < 2; ++i) mbar_arrive_expect_tx(&px_full[i], kPBytes / 2);
     if (rank == 0) mbar_arrive_expect_tx(l_full, 128 * 4);
   }
-  if (warp == 0 && lane == 0) prefetch_tmap(&a.map_cache);
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&a.map_cache);
+    if (kFp8) {
+      prefetch_tmap(&a.map_code);
+      prefetch_tmap(&a.map_scale);
+    }
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -177,12 +235,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         if (*abort_flag) return;
         const long long row0 = a.lay.block_table ? 0 : a.lay.seq_start[p.b];  // contiguous layout
         for (int t = p.t0; t < p.t1; ++t, ++it) {
-          const int s = it % kStages;
           // a tile lies within one page; a tile without a page (a capacity
           // fault of the call) loads rows past the tensor, which read as zero
           long long y0 = a.lay.block_table ? a.lay.row(p.b, static_cast<long long>(t) * kAttnTileTokens)
                                            : row0 + static_cast<long long>(t) * kAttnTileTokens;
           if (y0 < 0) y0 = a.n_rows;
+          if constexpr (kFp8) {
+            const int r = it % kRS;
+            if (!mbar_wait(&raw_empty[r], ((it / kRS) & 1) ^ 1, wc)) return;
+            mbar_arrive_expect_tx(&raw_full[r], C::kRawTx);
+            uint8_t* dst = raws + r * C::kRawBytes;
+            const int y_own = static_cast<int>(y0 + kHalf * rank), y_peer = static_cast<int>(y0 + kHalf * peer);
+            tma_load_2d(dst + C::kRawKr, &a.map_cache, &raw_full[r], a.kr_x, y_own, pol_once);
+            // the partner reads this CTA's rows in its own half of the codes too
+            tma_load_2d(dst + C::kRawOwn0, &a.map_code, &raw_full[r], 0, y_own, peer == 0 ? pol_twice : pol_once);
+            tma_load_2d(dst + C::kRawOwn1, &a.map_code, &raw_full[r], 256, y_own, peer == 1 ? pol_twice : pol_once);
+            tma_load_2d(dst + C::kRawPeer, &a.map_code, &raw_full[r], 256 * static_cast<int>(rank), y_peer, pol_twice);
+            tma_load_2d(dst + C::kRawOwnS, &a.map_scale, &raw_full[r], a.scale_x, y_own, pol_twice);
+            tma_load_2d(dst + C::kRawPeerS, &a.map_scale, &raw_full[r], a.scale_x, y_peer, pol_twice);
+            continue;
+          }
+          const int s = it % kStages;
           if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, wc)) return;
           mbar_arrive_expect_tx(&full[s], kStageBytes);
           uint8_t* dst = stages + s * kStageBytes;
@@ -257,13 +330,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
                 }
               }
               for (int ci = 0; ci < kQSmemChunks; ++ci) {
+                const int chunk = kQTmemChunks + ci;
+                // E4M3 rows: k^R (chunk 8) stays in the raw stage, already bf16
+                const uint32_t bchunk = (kFp8 && chunk == 8) ? smem_u32(raws + (g % kRS) * C::kRawBytes + C::kRawKr)
+                                                             : st + chunk * kChunkBytes;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                   mma_ss(dS, sdesc_sw128(smem_u32(qs) + ci * kQChunkBytes + kk * 32, 16, 1024),
-                         sdesc_sw128(st + (kQTmemChunks + ci) * kChunkBytes + kk * 32, 16, 1024), idesc_s, 1u);
+                         sdesc_sw128(bchunk + kk * 32, 16, 1024), idesc_s, 1u);
                 }
               }
               mma_commit(s_full);
+              if constexpr (kFp8) mma_commit(&raw_empty[g % kRS]);  // the raw stage's k^R was read
               if (ns == nt - 1) mma_commit(q_free);  // no MMA of this piece reads Q any more
               ++ns;
               issued = true;
@@ -290,13 +368,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       mma_commit(drain);
     }
   } else if (warp < 6) {
-    // ------------------------------------------------------------ Q_lat of each piece
+    // ------------------------------------------------------------ Q_lat of each piece (and, for
+    // E4M3 rows, the decode of every raw stage of the piece)
     const int q4 = warp & 3;
     const int h = q4 * 32 + lane;  // head = TMEM lane
     const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int sw = h & 7;
     const uint32_t q_row = smem_u32(qs) + h * 128;
     int piece = 0;
+    int cv = 0;  // E4M3 rows: tiles converted so far
     for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
       if (*abort_flag) return;
       // the previous piece's S products have retired: nothing reads Q now
@@ -325,6 +405,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       tc_fence_before();
       mbar_arrive(q_full);
       ++piece;
+      if constexpr (kFp8) {
+        // ---- E4M3 rows: decode each raw stage of the piece into its bf16
+        // stage.  A warp takes one (row, 256-code segment) at a time: 32 lanes
+        // read 8 codes each (256 contiguous bytes) and write 16 bytes into one
+        // of the segment's four 128-byte swizzled chunk rows.
+        const int cw = warp - 2;  // converter warp 0..3
+        const int cc = lane >> 3, u = lane & 7;
+        for (int t = p.t0; t < p.t1; ++t, ++cv) {
+          const int r = cv % kRS, s = cv % kStages;
+          if (!mbar_wait(&raw_full[r], (cv / kRS) & 1, wc)) return;
+          if (!mbar_wait(&empty[s], ((cv / kStages) & 1) ^ 1, wc)) return;
+          const uint8_t* raw = raws + r * C::kRawBytes;
+          uint8_t* st = stages + s * kStageBytes;
+          for (int task = cw; task < 3 * kHalf; task += 4) {
+            const int row = task % kHalf, seg = task / kHalf;  // seg 0, 1: own codes; 2: the partner's
+            const uint8_t* src = raw + (seg == 0 ? C::kRawOwn0 : seg == 1 ? C::kRawOwn1 : C::kRawPeer) + row * 256;
+            const int k = static_cast<int8_t>(raw[(seg < 2 ? C::kRawOwnS : C::kRawPeerS) + row * 16]);
+            const uint2 codes = *reinterpret_cast<const uint2*>(src + lane * 8);
+            const uint4 v = e4m3x8_to_bf16(codes, ldexpf(1.f, k));
+            const int chunk = (seg < 2 ? 4 * seg : kOwnChunks) + cc;
+            *reinterpret_cast<uint4*>(st + chunk * kChunkBytes + row * 128 + ((u ^ (row & 7)) << 4)) = v;
+          }
+          fence_proxy_async_smem();  // the MMAs read the stage through the async proxy
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&full[s]);
+            mbar_arrive(&raw_empty[r]);
+          }
+        }
+      }
     });
   } else {
     // ------------------------------------------------------------ softmax + epilogue

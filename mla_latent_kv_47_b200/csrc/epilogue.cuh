@@ -60,7 +60,9 @@ struct TokenMap {
   const int32_t* capacity;   // NULL or rows reserved per sequence
   long long n_rows;          // rows allocated in the cache
   void* cache;
-  int row_elems;             // d_c + d_R
+  int row_bytes;             // bytes of one cache row
+  int kr_off;                // byte offset of k^R inside a row
+  int fp8;                   // rows hold E4M3 c^KV (written by the latent finish kernel, not the GEMM)
   int d_c, d_R;
   double log2_base;          // log2(rope_base)
   const float2* rope;        // NULL, or (cos, sin) of pair i at token n: rope[n * d_R / 2 + i]
@@ -167,7 +169,7 @@ __device__ __forceinline__ void epi_apply(const Epi& e, const TokenMap& tk, int 
       break;
     case EPI_CACHE_CKV: {
       const long long row = cache_row(tk, n, status);
-      if (row >= 0) store_elem<T>(tk.cache, row * tk.row_elems + m, y, 0);
+      if (row >= 0) store_elem<T>(static_cast<uint8_t*>(tk.cache) + row * tk.row_bytes, m, y, 0);
       break;
     }
     case EPI_CACHE_KR: {
@@ -175,7 +177,7 @@ __device__ __forceinline__ void epi_apply(const Epi& e, const TokenMap& tk, int 
       float c, s;
       rope_cs(tk, n, m >> 1, inv_freq, c, s);
       const float r = rope_apply(m, y, yp, c, s);
-      if (row >= 0) store_elem<T>(tk.cache, row * tk.row_elems + tk.d_c + m, r, 0);
+      if (row >= 0) store_elem<T>(static_cast<uint8_t*>(tk.cache) + row * tk.row_bytes + tk.kr_off, m, r, 0);
       break;
     }
     case EPI_QP_ROPE: {
@@ -240,7 +242,7 @@ __device__ __forceinline__ uint8_t* epi_addr(const Epi& e, const TokenMap& tk, i
     case EPI_CACHE_KR: {
       const long long row = cache_row(tk, n, status);
       if (row < 0) return nullptr;
-      return static_cast<uint8_t*>(tk.cache) + (row * tk.row_elems + (e.kind == EPI_CACHE_KR ? tk.d_c : 0) + m) * 2;
+      return static_cast<uint8_t*>(tk.cache) + row * tk.row_bytes + (e.kind == EPI_CACHE_KR ? tk.kr_off : 0) + m * 2;
     }
     default: idx = static_cast<long long>(n) * e.ld + e.col0 + m; break;
   }

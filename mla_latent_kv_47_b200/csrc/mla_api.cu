@@ -36,6 +36,11 @@ struct Layout {
 
 int elem_size(const mla_dims& d) { return d.dtype == MLA_FP32 ? 4 : 2; }
 int row_elems(const mla_dims& d) { return d.d_c + d.d_R; }
+bool cache_fp8(const mla_dims& d) { return d.cache_format == MLA_CACHE_E4M3; }
+// Bytes of one cache row (the layouts of mla_cache_format).
+int row_bytes(const mla_dims& d) {
+  return cache_fp8(d) ? d.d_c + 2 * d.d_R + 16 : row_elems(d) * elem_size(d);
+}
 
 int pick_bn(int N) { return N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256; }
 
@@ -102,6 +107,20 @@ EncodeTiledFn get_encode() {
       fn = reinterpret_cast<EncodeTiledFn>(p);
   });
   return fn;
+}
+
+// 2-D byte tensor [rows x cols] with row stride `ld` bytes; box {box_cols, box_rows}, no swizzle.
+bool make_map_2d_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t ld, uint32_t box_cols,
+                    uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 2-D bf16 tensor [rows x cols] with row stride `ld` elements; box {64, box_rows}; 128-byte swizzle.
@@ -377,12 +396,14 @@ mla_status check_dims(const mla_dims* d) {
        !std::isfinite(d->yarn_L0)))
     return MLA_ERR_INVALID_ARG;
   if (d->dtype != MLA_BF16 && d->dtype != MLA_FP32) return MLA_ERR_UNSUPPORTED;
+  if (d->cache_format != MLA_CACHE_DTYPE && d->cache_format != MLA_CACHE_E4M3) return MLA_ERR_UNSUPPORTED;
+  if (d->cache_format == MLA_CACHE_E4M3 && d->dtype != MLA_BF16) return MLA_ERR_UNSUPPORTED;
   if (d->d_R % 2 != 0) return MLA_ERR_UNSUPPORTED;
   // CUDA-core kernels hold d_c/32 <= 16 latent columns and d_h/32 <= 8 value columns per lane.
   if (d->d_c > 512 || d->d_h > 256 || d->d_c % 4 != 0) return MLA_ERR_UNSUPPORTED;
   // 16-byte rows for every tensor the kernels load
   const int es = d->dtype == MLA_FP32 ? 4 : 2;
-  if ((row_elems(*d) * es) % 16 || (d->d_model * es) % 16 || (d->d_c * es) % 16) return MLA_ERR_UNSUPPORTED;
+  if (row_bytes(*d) % 16 || (d->d_model * es) % 16 || (d->d_c * es) % 16) return MLA_ERR_UNSUPPORTED;
   // bf16 storage runs on the tensor-core kernels only, which are built for the
   // DeepSeek-V2 head shape (d_h = 128, d_R = 64, d_c = 512, up to 128 heads)
   // and 64-wide K blocks; the CUDA-core kernels serve fp32 storage alone.
@@ -455,7 +476,9 @@ TokenMap cache_tokens(const mla_dims& d, const mla_cache* cache) {
   t.capacity = cache->capacity;
   t.n_rows = cache->n_rows;
   t.cache = cache->base;
-  t.row_elems = row_elems(d);
+  t.row_bytes = row_bytes(d);
+  t.kr_off = cache_fp8(d) ? d.d_c : d.d_c * elem_size(d);
+  t.fp8 = cache_fp8(d) ? 1 : 0;
   t.d_c = d.d_c;
   t.d_R = d.d_R;
   t.log2_base = std::log2(d.rope_base);
@@ -514,12 +537,13 @@ float qlat_scale(const mla_dims& d) {
 }
 
 // Appends the [W_DKV; W_KR] segments (cache-row epilogues) to a dense GEMM.
-// With an RMSNorm gain on c^KV the W_DKV segment leaves c^KV in fp32 at `nkv`
-// ([tokens x d_c]) for launch_latent_norm, which writes the cache rows.
+// With an RMSNorm gain on c^KV, or an E4M3 cache, the W_DKV segment leaves
+// c^KV in fp32 at `nkv` ([tokens x d_c]) for launch_latent_norm, which
+// writes the cache rows' c^KV part.
 void add_cache_segments(GemmSpec& g, const mla_dims& d, const mla_weights* w, void* nkv) {
   g.A[g.nseg] = w->W_DKV;
   g.rows[g.nseg] = d.d_c;
-  g.epi[g.nseg] = w->g_kv ? epi_store(nkv, d.d_c, 0, 1.f, 1) : epi_kind(EPI_CACHE_CKV);
+  g.epi[g.nseg] = (w->g_kv || cache_fp8(d)) ? epi_store(nkv, d.d_c, 0, 1.f, 1) : epi_kind(EPI_CACHE_CKV);
   ++g.nseg;
   g.A[g.nseg] = w->W_KR;
   g.rows[g.nseg] = d.d_R;
@@ -531,8 +555,8 @@ void add_cache_segments(GemmSpec& g, const mla_dims& d, const mla_weights* w, vo
 // into the tokens' cache rows, c^Q from `nq` into `cq_out` (storage dtype).
 mla_status launch_latent_norm(const Ctx& c, const mla_weights* w, const TokenMap& tk, int T, const void* nkv,
                               const void* nq, void* cq_out) {
-  if (!w->g_kv && !w->g_q) return MLA_OK;
-  const float* fk = static_cast<const float*>(nkv);
+  if (!w->g_kv && !w->g_q && !tk.fp8) return MLA_OK;
+  const float* fk = (w->g_kv || tk.fp8) ? static_cast<const float*>(nkv) : nullptr;
   const float* fq = static_cast<const float*>(nq);
   if (c.d.dtype == MLA_FP32)
     return launch(latent_norm_kernel<float>, dim3(T), dim3(256), 0, c.st, c.pdl, fk,
@@ -549,13 +573,31 @@ void attn_event(cudaEvent_t e, cudaStream_t st) {
   if (e) cudaEventRecord(e, st);
 }
 
-mla_status launch_attn_decode_tc(const __nv_bfloat16* qlat, const mla_cache* cache, const int32_t* seqlen,
-                                 const int* tile_start, const int* seg_start, int B, int W, int n_h, float* o_part,
-                                 float* ml, int* status, cudaStream_t st, bool pdl) {
+template <bool kFp8>
+mla_status launch_attn_kernel(const AttnArgs& a, int W, cudaStream_t st, bool pdl) {
+  static std::atomic<unsigned long long> attr_done{0};
+  const mla_status s = set_smem_limit(attn_decode_tc_kernel<kFp8>, attn::Cfg<kFp8>::kSmem, attr_done);
+  if (s != MLA_OK) return s;
+  return launch(attn_decode_tc_kernel<kFp8>, dim3(2 * W), dim3(attn::kThreads), attn::Cfg<kFp8>::kSmem, st, pdl, a);
+}
+
+mla_status launch_attn_decode_tc(const mla_dims& d, const __nv_bfloat16* qlat, const mla_cache* cache,
+                                 const int32_t* seqlen, const int* tile_start, const int* seg_start, int B, int W,
+                                 int n_h, float* o_part, float* ml, int* status, cudaStream_t st, bool pdl) {
   AttnArgs a;
   memset(&a, 0, sizeof(a));
   if (cache->n_rows > (1ll << 31) - 128) return MLA_ERR_UNSUPPORTED;  // tile rows are int32 TMA coordinates
-  if (!make_map_2d(&a.map_cache, cache->base, attn::kRow, cache->n_rows, attn::kRow, attn::kHalf)) return MLA_ERR_CUDA;
+  const bool fp8 = cache_fp8(d);
+  const int rb = row_bytes(d);
+  // bf16 view of the rows (the whole row for bf16 rows; k^R for E4M3 rows)
+  if (!make_map_2d(&a.map_cache, cache->base, rb / 2, cache->n_rows, rb / 2, attn::kHalf)) return MLA_ERR_CUDA;
+  if (fp8) {
+    if (!make_map_2d_u8(&a.map_code, cache->base, rb, cache->n_rows, rb, 256, attn::kHalf) ||
+        !make_map_2d_u8(&a.map_scale, cache->base, rb, cache->n_rows, rb, 16, attn::kHalf))
+      return MLA_ERR_CUDA;
+    a.kr_x = d.d_c / 2;
+    a.scale_x = d.d_c + 2 * d.d_R;
+  }
   a.qlat = qlat;
   a.lay = cache_layout(cache);
   a.n_rows = cache->n_rows;
@@ -568,10 +610,7 @@ mla_status launch_attn_decode_tc(const __nv_bfloat16* qlat, const mla_cache* cac
   a.o_part = o_part;
   a.ml_part = ml;
   a.status = status;
-  static std::atomic<unsigned long long> attr_done{0};
-  const mla_status s = set_smem_limit(attn_decode_tc_kernel, attn::kSmem, attr_done);
-  if (s != MLA_OK) return s;
-  return launch(attn_decode_tc_kernel, dim3(2 * W), dim3(attn::kThreads), attn::kSmem, st, pdl, a);
+  return fp8 ? launch_attn_kernel<true>(a, W, st, pdl) : launch_attn_kernel<false>(a, W, st, pdl);
 }
 
 bool prefill_tc_ok(const mla_dims& d) {
@@ -698,8 +737,8 @@ mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const 
   float* ml = reinterpret_cast<float*>(ws + c.L.ml);
   attn_event(g_attn_begin, c.st);
   if (tc_attn) {
-    if ((s = launch_attn_decode_tc(reinterpret_cast<const __nv_bfloat16*>(qlat), cache, seqlen, tile_start, seg_start,
-                                   B, W, d.n_h, opart, ml, c.status, c.st, c.pdl)) != MLA_OK)
+    if ((s = launch_attn_decode_tc(d, reinterpret_cast<const __nv_bfloat16*>(qlat), cache, seqlen, tile_start,
+                                   seg_start, B, W, d.n_h, opart, ml, c.status, c.st, c.pdl)) != MLA_OK)
       return s;
   } else {
     if (d.dtype != MLA_FP32) return MLA_ERR_UNSUPPORTED;  // bf16 is on the tensor-core kernel alone
@@ -789,6 +828,7 @@ size_t mla_workspace_offset(const mla_dims* dims, int max_batch, int max_tokens,
     case 2: return L.qlat;
     case 3: return L.olat;
     case 4: return L.o;
+    case 5: return L.p_nkv;
     default: return static_cast<size_t>(-1);
   }
 }
@@ -834,8 +874,10 @@ mla_status mla_cache_append(const mla_dims* dims, const mla_weights* w, const vo
   if (!h || !seq_idx || !pos) return MLA_ERR_INVALID_ARG;
   if (!aligned16(h)) return MLA_ERR_MISALIGNED;
   Ctx c;
-  // with an RMSNorm on c^KV the raw latents of the T tokens need the prefill region
-  if ((s = make_ctx(c, dims, 1, T, w->g_kv ? REGION_PREFILL : REGION_BASE, workspace, workspace_bytes, stream)) !=
+  // with an RMSNorm on c^KV or an E4M3 cache the raw latents of the T tokens
+  // need the prefill region
+  const bool raw_ckv = w->g_kv || cache_fp8(*dims);
+  if ((s = make_ctx(c, dims, 1, T, raw_ckv ? REGION_PREFILL : REGION_BASE, workspace, workspace_bytes, stream)) !=
       MLA_OK)
     return s;
   const mla_dims& d = *dims;
@@ -851,7 +893,7 @@ mla_status mla_cache_append(const mla_dims* dims, const mla_weights* w, const vo
   g.tok.seq = seq_idx;
   add_cache_segments(g, d, w, c.ws + c.L.p_nkv);
   if ((s = run_gemm(c, g)) != MLA_OK) return s;
-  if (!w->g_kv) return MLA_OK;
+  if (!raw_ckv) return MLA_OK;
   mla_weights kv_only = *w;
   kv_only.g_q = nullptr;  // appending caches c^KV only
   return launch_latent_norm(c, &kv_only, g.tok, T, c.ws + c.L.p_nkv, nullptr, nullptr);
@@ -903,6 +945,7 @@ extern "C" mla_status mla_prefill(const mla_dims* dims, const mla_weights* w, co
   if ((s = check_cache(cache)) != MLA_OK) return s;
   if (T <= 0 || start_pos < 0 || seq < 0 || !h || !u) return MLA_ERR_INVALID_ARG;
   if (!aligned16(h) || !aligned16(u)) return MLA_ERR_MISALIGNED;
+  if (cache_fp8(*dims)) return MLA_ERR_UNSUPPORTED;  // prefill reads and writes storage-dtype rows only
   const int S = start_pos + T;  // keys of the last token
   Ctx c;
   if ((s = make_ctx(c, dims, 1, S, REGION_PREFILL, workspace, workspace_bytes, stream)) != MLA_OK) return s;

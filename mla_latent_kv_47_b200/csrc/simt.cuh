@@ -263,6 +263,21 @@ __device__ __forceinline__ float block_sum_256(float v, float* red) {
   return t;
 }
 
+__device__ __forceinline__ float block_max_256(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t = fmaxf(t, red[i]);
+  return t;
+}
+
+// Finishes the latents of one token per block: the RMSNorm of c^KV (with
+// g_kv) and its store into the cache row, as the storage dtype or as an E4M3
+// row with its scale exponent; the RMSNorm of c^Q (with g_q).
 template <typename T>
 __global__ void __launch_bounds__(256) latent_norm_kernel(const float* __restrict__ ckv, const T* __restrict__ g_kv,
                                                           const float* __restrict__ cq, const T* __restrict__ g_q,
@@ -273,16 +288,49 @@ __global__ void __launch_bounds__(256) latent_norm_kernel(const float* __restric
   griddep_wait();
   if (threadIdx.x == 0) griddep_launch_dependents();
   const int n = blockIdx.x;
-  if (g_kv) {
+  if (g_kv || tk.fp8) {
     const float* x = ckv + static_cast<long long>(n) * tk.d_c;
-    float ss = 0.f;
-    for (int c = threadIdx.x; c < tk.d_c; c += 256) ss += x[c] * x[c];
-    const float inv = rsqrtf(block_sum_256(ss, red) / tk.d_c + kRmsEps);
+    float inv = 1.f;
+    if (g_kv) {
+      float ss = 0.f;
+      for (int c = threadIdx.x; c < tk.d_c; c += 256) ss += x[c] * x[c];
+      inv = rsqrtf(block_sum_256(ss, red) / tk.d_c + kRmsEps);
+    }
     if (threadIdx.x == 0) s_row = cache_row(tk, n, status);
     __syncthreads();
     if (s_row >= 0) {
-      T* dst = static_cast<T*>(tk.cache) + s_row * tk.row_elems;
-      for (int c = threadIdx.x; c < tk.d_c; c += 256) dst[c] = static_cast<T>(x[c] * inv * to_f32(g_kv[c]));
+      uint8_t* rowp = static_cast<uint8_t*>(tk.cache) + s_row * tk.row_bytes;
+      if (!tk.fp8) {
+        T* dst = reinterpret_cast<T*>(rowp);
+        for (int c = threadIdx.x; c < tk.d_c; c += 256)
+          dst[c] = static_cast<T>(g_kv ? x[c] * inv * to_f32(g_kv[c]) : x[c]);
+      } else {
+        // E4M3 row: scale exponent k = the smallest integer with amax / 2^k <= 448
+        // (amax = max |c|; frexp gives amax = f 2^e, f in [0.5, 1), and
+        // amax <= 448 2^k  <=>  k >= e - 9 + (f > 0.875)), codes = RNE(c / 2^k)
+        float am = 0.f;
+        for (int c = threadIdx.x; c < tk.d_c; c += 256) am = fmaxf(am, fabsf(g_kv ? x[c] * inv * to_f32(g_kv[c]) : x[c]));
+        am = block_max_256(am, red);
+        int k = 0;
+        if (am > 0.f) {
+          int e;
+          const float f = frexpf(am, &e);
+          k = e - 9 + (f > 0.875f ? 1 : 0);
+        }
+        const float descale = ldexpf(1.f, -k);
+        for (int c = 2 * threadIdx.x; c < tk.d_c; c += 512) {
+          float v0 = x[c], v1 = x[c + 1];
+          if (g_kv) {
+            v0 = v0 * inv * to_f32(g_kv[c]);
+            v1 = v1 * inv * to_f32(g_kv[c + 1]);
+          }
+          const __nv_fp8x2_storage_t q = __nv_cvt_float2_to_fp8x2(make_float2(v0 * descale, v1 * descale), __NV_SATFINITE, __NV_E4M3);
+          *reinterpret_cast<__nv_fp8x2_storage_t*>(rowp + c) = q;
+        }
+        // scale byte, then zeros to the end of the row (16 bytes after k^R)
+        const int sb = tk.kr_off + 2 * tk.d_R;
+        if (threadIdx.x < 16) rowp[sb + threadIdx.x] = threadIdx.x == 0 ? static_cast<uint8_t>(static_cast<int8_t>(k)) : 0;
+      }
     }
   }
   if (g_q) {

@@ -34,7 +34,7 @@ import math
 
 import numpy as np
 
-from oracle.mla import decode_unabsorbed, latent_rows, round_bf16_f64
+from oracle.mla import decode_absorbed, decode_unabsorbed, latent_rows, round_bf16_f64
 
 __all__ = ["FORMATS", "code_values", "max_finite", "encode", "decode", "row_scale_exp",
            "quantize_rows", "dequantize_rows", "store_rows", "decode_lowbit"]
@@ -155,11 +155,15 @@ def store_rows(c_kv, k_r, fmt_c: str, fmt_r: str | None = None):
     return c_store, r_store
 
 
-def decode_lowbit(W: dict, h_seq, dims, fmt_c: str, fmt_r: str | None = None):
+def decode_lowbit(W: dict, h_seq, dims, fmt_c: str, fmt_r: str | None = None, absorbed: bool = False):
     """u of the App. C decode step over a cache stored in the low-bit format:
     the exact latent rows, stored and read back by store_rows, then the
-    un-absorbed formulas of oracle.mla."""
+    un-absorbed formulas of oracle.mla (or, with `absorbed`, the absorbed form,
+    which is pinned to them and far cheaper for long sequences)."""
     h_seq = np.asarray(h_seq, dtype=np.float64)
     pos = np.arange(h_seq.shape[0], dtype=np.float64)
     c_kv, k_r = latent_rows(W, h_seq, pos, dims)
-    return decode_unabsorbed(W, h_seq, dims, cache_rows=store_rows(c_kv, k_r, fmt_c, fmt_r))
+    rows = store_rows(c_kv, k_r, fmt_c, fmt_r)
+    if absorbed:
+        return decode_absorbed(W, h_seq, dims, cache_rows=rows)
+    return decode_unabsorbed(W, h_seq, dims, cache_rows=rows)

@@ -213,18 +213,20 @@ def decode_unabsorbed(W: dict, h_seq, dims, cache_rows=None):
     return _output(W, o, dims)
 
 
-def decode_absorbed(W: dict, h_seq, dims, return_parts=False):
+def decode_absorbed(W: dict, h_seq, dims, return_parts=False, cache_rows=None):
     """Same result as decode_unabsorbed, with W^{UK} and W^{UV} absorbed.
 
     Associativity (App. C, last paragraph): q^C_i . (W^{UK}_i c_j) =
     (W^{UK}_i^T q^C_i) . c_j, and W^{UV}_i sum_j p_j c_j = sum_j p_j W^{UV}_i c_j,
     so keys and values are never formed: every head scores against the cached
-    [c^KV_j ; k^R_j] row with q_lat_i = [W^{UK}_i^T q^C_i ; q^R_i].
+    [c^KV_j ; k^R_j] row with q_lat_i = [W^{UK}_i^T q^C_i ; q^R_i].  The
+    identity holds for any cached rows, so `cache_rows` = (c_kv, k_r) may
+    replace the recomputed latents as in decode_unabsorbed.
     """
     h_seq = _f64(h_seq)
     L1 = h_seq.shape[0]
     pos = np.arange(L1, dtype=np.float64)
-    c_kv, k_r = latent_rows(W, h_seq, pos, dims)
+    c_kv, k_r = latent_rows(W, h_seq, pos, dims) if cache_rows is None else (_f64(cache_rows[0]), _f64(cache_rows[1]))
     q_c, q_r = queries(W, h_seq[-1:], pos[-1:], dims)
     W_UK = _f64(W["W_UK"]).reshape(dims.n_h, dims.d_h, dims.d_c)
     W_UV = _f64(W["W_UV"]).reshape(dims.n_h, dims.d_h, dims.d_c)

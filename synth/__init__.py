@@ -40,6 +40,7 @@ class Dims:
     rope_base: float = 10000.0
     dtype: str = "bf16"  # storage dtype of h, weights and cache: "bf16" | "fp32"
     yarn: tuple | None = None  # (s, alpha, beta, L0) of YaRN, or None for plain RoPE
+    cache: str = "dtype"       # latent cache rows: "dtype" (storage dtype) or "e4m3" (low-bit c^KV)
 
     @property
     def row_elems(self) -> int:

@@ -109,3 +109,37 @@ def cache_value_check(got_bits: np.ndarray, Wh: dict, h: np.ndarray, pos: np.nda
         # products) and the noise of the RMS itself: well under 2^-14 relative
         bound[:, :c_kv.shape[1]] += 2.0 ** -14 * np.abs(c_kv)
     return float(np.max(np.abs(got - exact) / bound))
+
+
+def e4m3_row_check(got_bytes: np.ndarray, Wh: dict, h: np.ndarray, pos: np.ndarray, dims) -> float:
+    """Checks stored E4M3 cache rows (bytes of the mla_cache_format layout)
+    against the exact rows.  c^KV: the decoded value code * 2^k must be within
+    half a code spacing of the exact value (2^-4 relative for normal codes,
+    2^(k-10) absolute below the smallest normal, 2^(k-6)) plus the fp32 noise
+    of the down-projection; the scale exponent must be the oracle's rule
+    applied to the row; the 15 padding bytes must be zero.  k^R: bf16 within
+    half an ulp plus the rotation's fp32 noise.  Returns the largest
+    |error| / bound (must be <= 1)."""
+    from oracle import lowbit as lb
+    from oracle import mla as om
+    d_c, d_R = dims.d_c, dims.d_R
+    c_kv, k_r = om.latent_rows(Wh, h, pos, dims)
+    g = np.asarray(got_bytes, dtype=np.uint8)
+    k = g[:, d_c + 2 * d_R].view(np.int8).astype(np.int64)
+    assert np.all(g[:, d_c + 2 * d_R + 1:d_c + 2 * d_R + 16] == 0), "padding bytes"
+    # the scale rule on the exact row may differ by one where amax sits on a power-of-two edge
+    k_ref = lb.row_scale_exp(np.max(np.abs(c_kv), axis=1), "e4m3")
+    assert np.all(np.abs(k - k_ref) <= 1), "scale exponent"
+    dec = lb.dequantize_rows(g[:, :d_c], k, "e4m3")
+    u = 2.0 ** -24
+    h2 = np.asarray(h, np.float64) ** 2
+    noise = 16.0 * np.sqrt(dims.d_model) * u * np.sqrt(h2 @ (np.asarray(Wh["W_DKV"], np.float64) ** 2).T)
+    bound_c = 2.0 ** -4 * np.abs(c_kv) + np.ldexp(1.0, k - 10)[:, None] + 2 * noise
+    ratio = float(np.max(np.abs(dec - c_kv) / bound_c))
+    kr = bf16_bits_to_f64(g[:, d_c:d_c + 2 * d_R].copy().view(np.uint16))
+    bound_r = 2.0 ** -8 * np.abs(k_r) + 1e-4 * (1.0 + np.abs(k_r))
+    return max(ratio, float(np.max(np.abs(kr - k_r) / bound_r)))
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    return synth.bf16_bits_to_f32(bits).astype(np.float64)

@@ -188,3 +188,23 @@ def test_rmsnorm_gain_arguments_are_checked(m):
     assert _call_decode(m, lite, m.Weights(*[A] * 8, None, A), A, 4, C, A, A, A, 1 << 40) == -1
     v2 = m.make_dims(synth.PRESETS["v2"].dims)
     assert _call_decode(m, v2, m.Weights(*[A] * 8, A + 2, None), A, 4, C, A, A, A, 1 << 40) == -3
+
+
+def test_e4m3_cache_arguments_are_checked(m):
+    """The E4M3 cache format needs bf16 storage; mla_prefill does not take it;
+    an unknown format is refused."""
+    import dataclasses
+    import synth
+    A = 1 << 20
+    W = m.Weights(*[A] * 8, None, None)
+    C = m.Cache(A, A, None, 1000, None, 0, 0)
+    e4 = m.make_dims(dataclasses.replace(synth.PRESETS["v2"].dims, cache="e4m3"))
+    assert e4.cache_format == m.CACHE_E4M3 and m.cache_row_bytes(e4) == 656
+    assert m.workspace_bytes(e4, 4, 4) > 0
+    assert m.lib.mla_prefill(ctypes.byref(e4), ctypes.byref(W), A, 8, 0, ctypes.byref(C), 0, A, A, 1 << 40, None) == -2
+    tiny = m.make_dims(synth.PRESETS["tiny"].dims)
+    tiny.cache_format = m.CACHE_E4M3
+    assert m.workspace_bytes(tiny, 1, 4) == 0
+    bad = m.make_dims(synth.PRESETS["v2"].dims)
+    bad.cache_format = 5
+    assert _call_decode(m, bad, W, A, 4, C, A, A, A, 1 << 40) == -2

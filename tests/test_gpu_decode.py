@@ -16,6 +16,7 @@ pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
 import synth  # noqa: E402
+from oracle import lowbit as lb  # noqa: E402
 from oracle import mla as om  # noqa: E402
 from tests import gpu_util as gu  # noqa: E402
 
@@ -69,7 +70,11 @@ def run_decode(m, preset, checked, lengths=None, pad=2, oracle="unabsorbed", dir
     for b in range(B):
         written[ss[b]:ss[b] + L[b] + 1] = True
     data = cache.data.cpu()
-    if d.dtype == "bf16":
+    e4m3 = getattr(d, "cache", "dtype") == "e4m3"
+    if e4m3:
+        bits = data.numpy()
+        pois = np.uint8(0x7F)
+    elif d.dtype == "bf16":
         bits = data.view(torch.int16).numpy().astype(np.uint16)
         pois = np.uint16(0x7FC1)
     else:
@@ -82,7 +87,10 @@ def run_decode(m, preset, checked, lengths=None, pad=2, oracle="unabsorbed", dir
     for b in checked:
         hb = seqs_h[b]
         got = bits[ss[b]:ss[b] + L[b] + 1]
-        if d.dtype == "bf16":
+        if e4m3:
+            ratio = gu.e4m3_row_check(got, Wh, hb, np.arange(L[b] + 1.0), d)
+            assert ratio <= 1.0, f"seq {b}: E4M3 cache row error at {ratio:.3g} of its bound"
+        elif d.dtype == "bf16":
             ratio = gu.cache_value_check(got, Wh, hb, np.arange(L[b] + 1.0), d)
             assert ratio <= 1.0, f"seq {b}: cache row error at {ratio:.3g} of its bound"
         else:
@@ -91,7 +99,10 @@ def run_decode(m, preset, checked, lengths=None, pad=2, oracle="unabsorbed", dir
             gotf = got.view(np.float32).astype(np.float64)
             assert np.max(np.abs(gotf - rows_ref)) <= 1e-5 * np.max(np.abs(rows_ref))
         form = oracle(L[b]) if callable(oracle) else oracle
-        u_ref = (om.decode_unabsorbed if form == "unabsorbed" else om.decode_absorbed)(Wh, hb, d)
+        if e4m3:   # the oracle over the same low-bit rows (codes and scales of the exact latents)
+            u_ref = lb.decode_lowbit(Wh, hb, d, "e4m3", absorbed=(form == "absorbed"))
+        else:
+            u_ref = (om.decode_unabsorbed if form == "unabsorbed" else om.decode_absorbed)(Wh, hb, d)
         stats[b] = gu.gate(u_h[b], u_ref)
     return stats
 

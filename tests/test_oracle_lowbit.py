@@ -218,3 +218,18 @@ def test_planted_mistake_is_caught(name, monkeypatch):
     with pytest.raises(AssertionError):
         for fmt in FMTS:
             globals()[pin](fmt)
+
+
+@pytest.mark.parametrize("preset,L", [("tiny", 40), ("v2", 90)])
+def test_absorbed_lowbit_equals_unabsorbed_lowbit(preset, L):
+    """The absorbed form over low-bit rows equals the un-absorbed one (the
+    absorption identity of App. C holds for whatever rows are cached), so the
+    long GPU parity cases may use the cheaper form."""
+    import synth
+    p = synth.preset(preset)
+    W = synth.weights(p)
+    h = synth.hidden(p, 1, L + 1)
+    for fmt in ("e4m3", "e5m2"):
+        a = lb.decode_lowbit(W, h, p.dims, fmt, absorbed=True)
+        b = lb.decode_lowbit(W, h, p.dims, fmt)
+        assert np.max(np.abs(a - b)) <= 1e-12 * np.max(np.abs(b))
