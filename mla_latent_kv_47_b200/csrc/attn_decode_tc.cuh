@@ -24,15 +24,12 @@
 // retirement is committed to both CTAs' barriers (multicast commit), which
 // tells each side that both P buffers may take the next tile.
 //
-// The softmax never waits for the partner inside a piece.  Both CTAs form
-// P(j) against the same running max m, and decide whether tile j moves m
-// one tile later, once the partner's tile maxima (sent as soon as S(j) is
-// read) have long arrived: if the max over both halves of tile j exceeds m
-// by more than 2^8, both rescale O and l and take the new max from tile
-// j + 1 on.  Only a piece's first tile waits for the partner (it sets m).
-// Until a decision lands, P may exceed 1; the kernel's range is
-// P <= 2^96 (ample for fp32 O and l), and a tile whose scores jump past it
-// sets FAULT_RANGE.
+// The softmax waits for the partner once per piece.  The max over both
+// halves of a piece's first tile is the piece's reference m, and every P of
+// the piece is 2^(s - m).  The reference cancels in O / l, so it need not be
+// the running max: later tiles may give P > 1, and O and l are never
+// rescaled.  The kernel's range is P <= 2^96 (ample for fp32 O and l); a
+// tile whose scores rise past it sets FAULT_RANGE.
 //
 // Warp roles (448 threads per CTA):
 //   warp 0      TMA producer (3-stage ring)
@@ -42,11 +39,9 @@
 //               7-8 into shared memory, both MMA A operands
 //   warps 6-13  softmax: warp 6+i and warp 10+i share lane quarter i mod 4,
 //               16 heads each; two threads per head (rows 0-15 and 16-31 of
-//               this CTA's half, via the 16-lane TMEM access shape).  Online
-//               softmax with a lazily refreshed max (O is rescaled only when a
-//               tile's max exceeds the running one by more than 2^8, decided
-//               one tile late as above), and the per-piece epilogue; CTA 1
-//               sends its share of l to CTA 0.
+//               this CTA's half, via the 16-lane TMEM access shape).  Softmax
+//               against the piece's reference max (above), and the per-piece
+//               epilogue; CTA 1 sends its share of l to CTA 0.
 #pragma once
 #include "mla.h"
 #include "ptx.cuh"
@@ -71,7 +66,6 @@ constexpr int kMaxSlots = 4;                           // partner tile maxima in
 constexpr int kAuxBytes = 3072;                        // partner maxima, CTA 1's l, barriers
 // TMEM columns: O half [0,256), S [256,288), Q chunks 0-6 (bf16 pairs) [288,512)
 constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 288, kTmemCols = 512;
-constexpr float kRescaleLog2 = 8.f;
 constexpr float kRangeLog2 = 96.f;                     // largest exponent of P before the max catches up
 constexpr int kRow = 576;                              // d_c + d_R
 static_assert(kTmemQ + kQTmemChunks * 32 == kTmemCols, "TMEM budget");
@@ -451,14 +445,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     const uint32_t mx_peer = mapa(smem_u32(mx), peer) + h * 4;
     const uint32_t mxfull_peer = mapa(smem_u32(mx_full), peer);
     int it = 0, piece = 0;
-    // The partner's maxima of tile g sit in slot g % kMaxSlots; reading them
-    // (and re-arming the slot) is the only per-tile wait on the partner.
-    auto partner_max = [&](int g, float& v) -> bool {
-      const int slot = g & (kMaxSlots - 1);
-      if (!mbar_wait<true>(&mx_full[slot], (g / kMaxSlots) & 1, wc)) return false;
+    // The partner's maxima of the first tile of piece j sit in slot j % kMaxSlots.
+    auto partner_max = [&](int j, float& v) -> bool {
+      const int slot = j & (kMaxSlots - 1);
+      if (!mbar_wait<true>(&mx_full[slot], (j / kMaxSlots) & 1, wc)) return false;
       v = mx[slot * 128 + h];
-      // next phase of the slot: the partner's maxima of tile g + 4, which it
-      // sends only after reading this CTA's maxima of tile g + 2 (sent later)
+      // next phase of the slot: the partner's maxima of piece j + 4, which it
+      // sends only after it received P of piece j + 1 from this CTA
       if (lead) mbar_arrive_expect_tx(&mx_full[slot], 128 * 4);
       return true;
     };
@@ -467,7 +460,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       const bool head = h < a.n_h;
       const int L1 = a.seqlen[p.b] + 1;
       float m_run = -INFINITY, l_run = 0.f;  // l_run: this thread's 16 rows only
-      float mo_prev = -INFINITY;             // this CTA's max of the previous tile
       const int nt = p.t1 - p.t0;
       for (int k = 0; k < nt; ++k) {
         const int g = it + k;
@@ -495,28 +487,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
 #pragma unroll
         for (int j = 1; j < 16; ++j) mo = fmaxf(mo, sc[j]);
         mo = fmaxf(mo, __shfl_xor_sync(0xffffffffu, mo, 16));  // this CTA's 32 rows
-        if (th == 0) st_async_b32(mx_peer + (g & (kMaxSlots - 1)) * 512, __float_as_uint(mo), mxfull_peer + (g & (kMaxSlots - 1)) * 8);
-        bool rescale = false;
-        float alpha = 1.f;
         if (k == 0) {
-          // the piece's first tile sets the max: both halves are needed now
+          // the piece's first tile sets its reference max: both halves of the
+          // tile are needed, so the pair swaps its maxima once per piece
+          if (th == 0)
+            st_async_b32(mx_peer + (piece & (kMaxSlots - 1)) * 512, __float_as_uint(mo),
+                         mxfull_peer + (piece & (kMaxSlots - 1)) * 8);
           float pm;
-          if (!partner_max(g, pm)) return;
+          if (!partner_max(piece, pm)) return;
           m_run = fmaxf(mo, pm);
-        } else if (k >= 2) {
-          // the decision for tile g - 1, whose partner maxima arrived a tile ago
-          float pm;
-          if (!partner_max(g - 1, pm)) return;
-          const float mt = fmaxf(mo_prev, pm);  // the same value in both CTAs
-          if (mt > m_run + kRescaleLog2) {
-            alpha = ex2_approx(m_run - mt);
-            m_run = mt;
-            rescale = true;
-          }
         }
-        mo_prev = mo;
-        // P of this thread's rows against m_run, and their sum; exponents are
-        // capped at the kernel's range (a jump past it is reported)
+        // P of this thread's rows against the piece's reference max, and their
+        // sum; exponents are capped at the kernel's range (a jump past it is
+        // reported)
         if (__any_sync(0xffffffffu, mo > m_run + kRangeLog2)) {
           if (mo > m_run + kRangeLog2) atomicOr(a.status, FAULT_RANGE);
 #pragma unroll
@@ -531,24 +514,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
           pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
         }
-        l_run = l_run * alpha + lsum;
+        l_run += lsum;
         // ---- P buffer b is free in both CTAs once PV(g-2) retired in both
         if (!mbar_wait_inline(&pv_done[b], ph ^ 1, wc)) return;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
-          // O must hold PV(g-1) before it is scaled (k >= 2 here, so g >= 1)
-          if (!mbar_wait_inline(&pv_done[b ^ 1], ((g - 1) >> 1) & 1, wc)) return;
-          tc_fence_after();
-          for (int c = 0; c < 256; c += 32) {
-            uint32_t o[16];
-            tmem_ld16x2(tl + kTmemO + c, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st16x2(tl + kTmemO + c, o);
-          }
-          tmem_wait_st();
-        }
         const int v64 = min(kAttnTileTokens, L1 - tile0);  // valid rows of the tile
         if (v64 < kAttnTileTokens) {
           // rows past the sequence may hold anything (even NaN); 0 * NaN would
@@ -575,12 +544,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[b]);
-      }
-      // the partner's maxima of the piece's last tile (if not read yet) must
-      // land before the slot is reused; O, l and m_run are already consistent
-      if (nt >= 2) {
-        float pm;
-        if (!partner_max(it + nt - 1, pm)) return;
       }
       // ---- epilogue of the piece: unnormalised O_r; CTA 0 writes m and l
       if (!mbar_wait(o_done, piece & 1, wc)) return;

@@ -81,8 +81,24 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   constexpr uint32_t kTmemCols = BN * MT < 32 ? 32 : BN * MT;
   static_assert(BN * MT <= 512 && (BN * MT & (BN * MT - 1)) == 0, "TMEM columns: a power of two <= 512");
 
-  // ---- which tile
-  const int mt = blockIdx.x, nt = blockIdx.y, split = blockIdx.z;
+  // ---- which tile.  With several token tiles (prefill, long appends) the
+  // grid is walked in groups of kRasterGroup weight tiles: consecutive CTAs
+  // take the same few weight tiles against successive token tiles, so a
+  // weight tile is read from HBM once and then from L2, instead of once per
+  // token tile when all weight tiles run before the next token tile.
+  int mt = blockIdx.x, nt = blockIdx.y;
+  const int split = blockIdx.z;
+  if (gridDim.y > 1) {
+    constexpr int kRasterGroup = 8;
+    const int num_m = gridDim.x, num_n = gridDim.y;
+    const int lin = blockIdx.x + num_m * blockIdx.y;
+    const int group = lin / (kRasterGroup * num_n);
+    const int first_m = group * kRasterGroup;
+    const int gm = min(num_m - first_m, kRasterGroup);  // weight tiles in this group
+    const int in_group = lin - group * kRasterGroup * num_n;
+    mt = first_m + in_group % gm;
+    nt = in_group / gm;
+  }
   int seg = 0, head = 0, m0;
   if (args.mode == GEMM_DENSE) {
     while (seg + 1 < args.nseg && mt >= args.seg_tile0[seg + 1]) ++seg;

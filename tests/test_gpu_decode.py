@@ -161,16 +161,17 @@ def test_decode_with_dirty_workspace(m, preset, L):
             gu.assert_gate(s)
 
 
-def test_lazy_rescale_of_o(m):
+def test_scores_above_the_piece_reference(m):
     """Cached tokens scaled by 1 and 4 in alternate 64-token tiles (the query
     row unscaled) put the max score of a scaled tile ~11.5 log2 units above an
-    unscaled tile's (~15 against ~3.5), past the kernel's 2^8 rescale
-    threshold, so the lazy rescale of O and l runs inside most pieces;
-    unscaled inputs never reach it.  The lengths give ~2.8 tiles per worker,
-    so pieces span several tiles.  With scores this large the bf16 operands
-    alone (Q_lat, cache rows, P) cost up to 0.72% max / 0.15% mean of max|u|
-    (fp64 emulation of those roundings), inside the gate; larger scales push
-    that bound past it."""
+    unscaled tile's (~15 against ~3.5).  The attention kernel forms P against
+    the max of a piece's first tile, so inside most pieces P rises to ~2^11
+    (never rescaled; the reference cancels in O / l), which unscaled inputs
+    never reach.  The lengths give ~2.8 tiles per worker, so pieces span
+    several tiles.  With scores this large the bf16 operands alone (Q_lat,
+    cache rows, P) cost up to 0.72% max / 0.15% mean of max|u| (fp64
+    emulation of those roundings), inside the gate; larger scales push that
+    bound past it."""
     L = [8192, 4000, 777]
 
     def scale(pos):
@@ -274,9 +275,8 @@ def test_decode_intermediates(m, preset):
 
 
 def test_score_jump_past_the_kernel_range_is_reported(m):
-    """Inside a run of tiles the attention kernel forms P against the running
-    max and learns a tile's max one tile late, so P may exceed 1 until then;
-    its range is P <= 2^96.  Cached tokens 192..255 of sequence 0 scaled by 64
+    """Inside a run of tiles the attention kernel forms P against the max of
+    the run's first tile, so P may exceed 1; its range is P <= 2^96.  Cached tokens 192..255 of sequence 0 scaled by 64
     put that tile's scores ~200 log2 units above the earlier tiles' (its piece
     starts at tile 0: 8 sequences of 4096 tokens give ~7 tiles per attention
     worker), past the range, so the call reports FAULT_RANGE through the
