@@ -360,6 +360,10 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* dst, float4
 
 // One warp per (sequence, head): lane l owns columns 4l + 128k.  The pieces
 // are merged in order, weights 2^(m_s - M), then normalised by the merged l.
+// The weights of up to kCombineUnroll pieces are formed first, so that all
+// of a lane's partial loads of a column group are in flight together.
+constexpr int kCombineUnroll = 4;
+
 template <typename T>
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ o_part, const float* __restrict__ ml_part,
                                                      const int* seg_start, int n_h, int d_c, T* __restrict__ olat) {
@@ -376,16 +380,34 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
     Ls += exp2f(ml_part[i] - M) * ml_part[i + 1];
   }
   const float inv = 1.f / Ls;
-  for (int c = lane * 4; c < d_c; c += 128) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = s0; s < s1; ++s) {
-      const float wgt = exp2f(ml_part[(static_cast<long long>(s) * n_h + h) * 2] - M);
-      const float4 v = *reinterpret_cast<const float4*>(o_part + (static_cast<long long>(s) * n_h + h) * d_c + c);
-      acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
+  float4 acc[4];  // columns lane * 4 + 128 k, k < d_c / 128 (d_c <= 512)
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int nk = lane * 4 < d_c ? (d_c - lane * 4 + 127) / 128 : 0;  // this lane's column groups
+  for (int sb = s0; sb < s1; sb += kCombineUnroll) {
+    float wgt[kCombineUnroll];
+#pragma unroll
+    for (int u = 0; u < kCombineUnroll; ++u)
+      wgt[u] = sb + u < s1 ? exp2f(ml_part[(static_cast<long long>(sb + u) * n_h + h) * 2] - M) : 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (k >= nk) break;
+      float4 v[kCombineUnroll];
+#pragma unroll
+      for (int u = 0; u < kCombineUnroll; ++u)
+        v[u] = sb + u < s1 ? __ldcs(reinterpret_cast<const float4*>(
+                                 o_part + (static_cast<long long>(sb + u) * n_h + h) * d_c + lane * 4 + 128 * k))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < kCombineUnroll; ++u) {
+        acc[k].x += wgt[u] * v[u].x; acc[k].y += wgt[u] * v[u].y;
+        acc[k].z += wgt[u] * v[u].z; acc[k].w += wgt[u] * v[u].w;
+      }
     }
-    store4<T>(olat + (static_cast<long long>(b) * n_h + h) * d_c + c,
-              make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv));
   }
+  for (int k = 0; k < nk; ++k)
+    store4<T>(olat + (static_cast<long long>(b) * n_h + h) * d_c + lane * 4 + 128 * k,
+              make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv));
 }
 
 // ---------------------------------------------------------------- prefill attention (CUDA cores)
