@@ -253,6 +253,14 @@ mla_status mla_decode_static(const mla_dims* dims, const mla_weights* w,
                              const mla_cache* cache, const int32_t* seqlen,
                              float* u, mla_stream_t stream);
 
+/* Diagnostic: exercises the bounded pipeline waits every kernel uses.  Runs a
+ * one-thread-block kernel whose wait on a shared-memory barrier is never
+ * satisfied; after the time limit (2 s) the wait gives up, sets
+ * FAULT_WAIT_TIMEOUT (2) in the workspace's status word and the kernel exits,
+ * leaving the context usable.  Read the result with mla_get_device_status.
+ * workspace: as for the other calls (256-byte aligned, status word zeroed). */
+mla_status mla_check_wait_timeout(void* workspace, mla_stream_t stream);
+
 /* Diagnostic: number of kernels this library has launched in this process
  * (all entry points, all threads).  The difference across a call counts the
  * call's kernel launches. */

@@ -24,7 +24,7 @@ WS_CQ, WS_QC, WS_QLAT, WS_OLAT, WS_O, WS_CKV_RAW = range(6)
 
 EXPORTS = ("mla_workspace_bytes", "mla_cache_append", "mla_decode", "mla_prefill",
            "mla_get_device_status", "mla_status_string", "mla_workspace_offset", "mla_set_attention_events",
-           "mla_decode_static", "mla_kernel_launches")
+           "mla_decode_static", "mla_kernel_launches", "mla_check_wait_timeout")
 
 
 class MLAError(RuntimeError):
@@ -77,6 +77,8 @@ def _load():
     lib.mla_decode_static.restype = i32
     lib.mla_kernel_launches.argtypes = []
     lib.mla_kernel_launches.restype = ctypes.c_ulonglong
+    lib.mla_check_wait_timeout.argtypes = [vp, vp]
+    lib.mla_check_wait_timeout.restype = i32
     lib.mla_set_attention_events.argtypes = [vp, vp]
     lib.mla_set_attention_events.restype = None
     return lib
@@ -202,6 +204,11 @@ def decode_static(dims, weights, h, cache, seqlen, u, stream=None):
     _check(_lib().mla_decode_static(ctypes.byref(dims), ctypes.byref(weights), _ptr(h), int(h.shape[0]),
                                     ctypes.byref(cache), _ptr(seqlen), _ptr(u), _stream(stream)),
            "mla_decode_static")
+
+
+def check_wait_timeout(workspace, stream=None):
+    """Runs the library's bounded-wait self-check (about 2 s on the GPU)."""
+    _check(_lib().mla_check_wait_timeout(_ptr(workspace), _stream(stream)), "mla_check_wait_timeout")
 
 
 def device_status(workspace, stream=None):

@@ -263,6 +263,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
                         (4 * static_cast<int>(rank) + cj) * 64, y_peer, pol_twice);
         }
       });
+      // every load issued has landed before the CTA may leave (after an abort,
+      // loads can still be in flight into stages nobody consumes)
+      if constexpr (kFp8) drain_ring(raw_full, kRS, it);
+      else drain_ring(full, kStages, it);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer

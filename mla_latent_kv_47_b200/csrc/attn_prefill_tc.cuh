@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(192, 1) attn_prefill_tc_kernel(const __grid_co
       const uint64_t keep = policy_evict_last();
       mbar_arrive_expect_tx(q_full, kQBytes);
       for (int c = 0; c < 3; ++c) tma_load_2d(sq + c * kChunk, &a.map_q, q_full, h * 192 + c * 64, q0, keep);
+      int k_issued = 0, v_issued = 0;
       for (int j = 0; j < nk; ++j) {
         const int s = j & 1;
         const uint32_t ph = ((j >> 1) & 1) ^ 1;
@@ -115,12 +116,18 @@ __global__ void __launch_bounds__(192, 1) attn_prefill_tc_kernel(const __grid_co
         tma_load_2d(kd, &a.map_kc, &k_full[s], h * 128, y, keep);
         tma_load_2d(kd + kChunk, &a.map_kc, &k_full[s], h * 128 + 64, y, keep);
         tma_load_2d(kd + 2 * kChunk, &a.map_kr, &k_full[s], 512, y, keep);
+        ++k_issued;
         if (!mbar_wait(&v_empty[s], ph, wc)) break;
         mbar_arrive_expect_tx(&v_full[s], kVBytes);
         uint8_t* vd = sv + s * kVBytes;
         tma_load_2d(vd, &a.map_v, &v_full[s], h * 128, y, keep);
         tma_load_2d(vd + kChunk, &a.map_v, &v_full[s], h * 128 + 64, y, keep);
+        ++v_issued;
       }
+      // every issued load has landed before the CTA may leave
+      drain_ring(q_full, 1, 1);
+      drain_ring(k_full, 2, k_issued);
+      drain_ring(v_full, 2, v_issued);
     }
   } else if (warp == 1) {
     if (elect_one()) {

@@ -177,7 +177,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       if (!args.x_independent) griddep_wait();
       for (int i = 0; i < pre; ++i)
         for (int j = 0; j < stage_kbs(i); ++j) load_b(i, j);
-      for (int i = pre; i < nk; ++i) {
+      int issued = pre;
+      for (int i = pre; i < nk; ++i, ++issued) {
         const int s = i % STAGES;
         if (!mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, wc)) break;
         mbar_arrive_expect_tx(&full[s], stage_kbs(i) * (bytesA + bytesB));
@@ -186,6 +187,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
           load_b(i, j);
         }
       }
+      drain_ring(full, STAGES, issued);  // every issued load has landed before the CTA may leave
     }
   } else if (warp == 1) {
     if (elect_one()) {

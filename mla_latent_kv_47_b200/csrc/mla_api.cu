@@ -801,10 +801,37 @@ mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const 
   return MLA_OK;
 }
 
+// One CTA whose thread 0 waits on a barrier nothing will complete: the
+// bounded wait gives up after its time limit and records FAULT_WAIT_TIMEOUT.
+// No load, store or MMA is in flight, so nothing lands after the CTA exits.
+__global__ void wait_timeout_kernel(int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const WaitCtx wc{status, &abort_flag};
+    mbar_wait(&bar, 0, wc);
+  }
+  __syncthreads();
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
 extern "C" {
+
+mla_status mla_check_wait_timeout(void* workspace, mla_stream_t stream) {
+  if (!workspace) return MLA_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return MLA_ERR_MISALIGNED;
+  g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
+  wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(static_cast<int*>(workspace));
+  return cudaPeekAtLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
 
 unsigned long long mla_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }
 

@@ -157,6 +157,22 @@ __device__ __forceinline__ bool mbar_wait_inline(uint64_t* bar, uint32_t parity,
   }
 }
 
+// Waits, within the time limit and whatever the abort flag says, until every
+// TMA load issued into a ring has landed: `issued` loads went into the ring's
+// slots in order (load t into slot t % stages, completing on full[t % stages]),
+// and a barrier's phases complete in order, so it suffices to wait for the
+// last armed phase of each slot.  A CTA that gave up on a wait calls this
+// before it exits, so that no load can land in shared memory it no longer owns.
+__device__ __forceinline__ void drain_ring(uint64_t* full, int stages, int issued) {
+  for (int s = 0; s < stages && s < issued; ++s) {
+    const int last = issued - 1 - ((issued - 1 - s) % stages);  // the last load into slot s
+    const uint32_t parity = (last / stages) & 1;
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(smem_u32(&full[s]), parity) && globaltimer() - t0 < kWaitLimitNs) {
+    }
+  }
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;

@@ -208,3 +208,8 @@ def test_e4m3_cache_arguments_are_checked(m):
     bad = m.make_dims(synth.PRESETS["v2"].dims)
     bad.cache_format = 5
     assert _call_decode(m, bad, W, A, 4, C, A, A, A, 1 << 40) == -2
+
+
+def test_wait_timeout_check_needs_a_workspace(m):
+    assert m.lib.mla_check_wait_timeout(None, None) == -4
+    assert m.lib.mla_check_wait_timeout((1 << 20) + 16, None) == -3

@@ -299,3 +299,18 @@ def test_score_jump_past_the_kernel_range_is_reported(m):
     code, detail = m.device_status(ws)
     assert code == -6 and detail & m.FAULT_RANGE, (code, detail)
     assert m.device_status(ws) == (0, 0)
+
+
+def test_bounded_wait_gives_up_and_the_context_stays_usable(m):
+    """A pipeline wait that nothing satisfies gives up after its time limit,
+    reports FAULT_WAIT_TIMEOUT through the status word, and leaves the GPU
+    context usable: a decode right after it passes the gate."""
+    p = synth.preset("tiny")
+    dims = m.make_dims(p.dims)
+    ws = m.alloc_workspace(dims, 1, 1)
+    m.check_wait_timeout(ws)
+    code, detail = m.device_status(ws)
+    assert code == -6 and detail == m.FAULT_WAIT_TIMEOUT, (code, detail)
+    st = run_decode(m, "tiny", checked=[0])
+    for s in st.values():
+        gu.assert_gate(s, 1e-4, 1e-4)
