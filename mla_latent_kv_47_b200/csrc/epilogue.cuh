@@ -275,20 +275,22 @@ __device__ __forceinline__ void epi_rope_run(const Epi& e, const TokenMap& tk, i
 // shared-memory loads and global stores overlap); cache and rotary kinds take
 // the general one.
 __device__ __forceinline__ void epi_flush(const Epi& e, const TokenMap& tk, int m0, int rows_valid, int n_base, int n_cols,
-                                          int n_end, int head, const uint8_t* stage, int tid, int nthr, int* status) {
+                                          int n_end, int head, const uint8_t* stage, int tid, int nthr, int* status,
+                                          int ml_lo = 0, int ml_hi = 128) {
+  // only the tile rows [ml_lo, ml_hi) (multiples of 8) are written
   const int kind = e.kind;
   const bool rot = epi_rotary(kind);
   if (!rot && kind != EPI_CACHE_CKV) {
-    // runs of 16 bytes: 8 bf16 or 4 fp32 rows; log2 of runs per token
-    const int lg = e.out_f32 ? 5 : 4;
+    // runs of 16 bytes: 8 bf16 or 4 fp32 rows
     const int es = e.out_f32 ? 4 : 2;
     uint8_t* const out = static_cast<uint8_t*>(e.out);
     const long long ld = e.ld;
     const long long off0 = kind == EPI_PER_HEAD ? static_cast<long long>(head) * e.hs : e.col0;
-    const int total = n_cols << lg;
+    const int lg_lo = __ffs(((ml_hi - ml_lo) / (16 / es))) - 1;  // log2 of runs per token in the row range
+    const int total = n_cols << lg_lo;
 #pragma unroll 4
     for (int id = tid; id < total; id += nthr) {
-      const int nl = id >> lg, ml = (id & ((1 << lg) - 1)) * (16 / es);
+      const int nl = id >> lg_lo, ml = ml_lo + (id & ((1 << lg_lo) - 1)) * (16 / es);
       const int n = n_base + nl, m = m0 + ml;
       if (n >= n_end || m >= rows_valid) continue;
       long long idx;
@@ -300,9 +302,9 @@ __device__ __forceinline__ void epi_flush(const Epi& e, const TokenMap& tk, int 
   }
   const bool f32 = rot || e.out_f32;  // staging type
   const int vec = (!rot && e.out_f32) ? 4 : 8;  // rows per run
-  const int runs = 128 / vec;
+  const int runs = (ml_hi - ml_lo) / vec;
   for (int id = tid; id < n_cols * runs; id += nthr) {
-    const int nl = id / runs, ml = (id % runs) * vec;
+    const int nl = id / runs, ml = ml_lo + (id % runs) * vec;
     const int n = n_base + nl, m = m0 + ml;
     if (n >= n_end || m >= rows_valid) continue;
     uint8_t* dst = epi_addr(e, tk, m, n, head, status);

@@ -24,6 +24,7 @@ enum GemmMode : int {
 };
 
 constexpr int kMaxSeg = 4;
+constexpr int kMaxClusterK = 8;  // splits of one tile reduced inside a cluster (portable cluster size)
 
 struct GemmArgs {
   CUtensorMap mapA[kMaxSeg];
@@ -41,7 +42,8 @@ struct GemmArgs {
   int kb_total;                // K / 64
   int kb_per_split;
   int splits;
-  float* partials;             // [tiles][splits][BN/4][128][4] fp32 (splits > 1)
+  int cluster_k;               // > 1: the splits of a tile form one cluster and reduce through shared memory
+  float* partials;             // [tiles][splits][BN/4][128][4] fp32 (splits > 1, cluster_k <= 1)
   int* status;
   int x_independent;           // 1: X is a call input no earlier kernel writes; only the epilogue waits
   TokenMap tok;
@@ -58,6 +60,8 @@ struct GemmSmem {
   static constexpr int kB = KBB * kSlabB;
   static constexpr int kStage = kA + kB;
   static constexpr int kBytes = 1024 + STAGES * kStage + 256;
+  // cluster split-K keeps the fp32 partial tile and a staging tile in the A buffers
+  static constexpr bool kClusterK = MT == 1 && STAGES * kA >= 2 * BN * 128 * 4;
 };
 
 // MT > 1 (per-head modes, no split-K): one CTA computes MT consecutive
@@ -229,7 +233,21 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     if (!*abort_flag) {
       const Epi& e = args.epi[seg];
       const int tile_id = mt + gridDim.x * nt;
-      if (args.splits > 1) {
+      if (args.cluster_k > 1) {
+        // split-K inside a cluster: this split's partial tile goes to the idle
+        // pipeline buffers, [BN/4 column groups][128 rows][4]; the reduction
+        // after the cluster barrier below reads it from every CTA
+        float4* my = reinterpret_cast<float4*>(sA);
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          float v[16];
+          tmem_ld16(trow + c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            my[((c >> 2) + q) * 128 + row] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+      } else if (args.splits > 1) {
         // split-K: store this split's partial tile ([BN/4 column groups][128 rows][4],
         // so a warp moves 512 contiguous bytes per float4); gemm_splitk_epilogue_kernel
         // sums the splits in order and applies the epilogue
@@ -269,6 +287,45 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   // warps arrive, and TMEM would be freed under their loads).
   __syncwarp();
   __syncthreads();
+  if (args.cluster_k > 1) {
+    // ---- split-K reduction across the cluster: CTA z of the S splits sums
+    // rows [z 128/S, (z+1) 128/S) of the tile over all S partials, in split
+    // order, and runs the epilogue on them.  Every CTA takes both barriers,
+    // aborted or not, so none waits for a CTA that left.
+    cluster_sync();  // every partial tile is in its CTA's shared memory
+    if (warp >= 2 && !*abort_flag) {
+      const int S = args.cluster_k;
+      const int z = static_cast<int>(cluster_ctarank());
+      const int nr = 128 / S, r0 = z * nr;
+      const int tid = threadIdx.x - 64;
+      const Epi& e = args.epi[seg];
+      uint8_t* stage = sA + BN * 128 * 4;  // after the partial tile
+      const uint32_t part = smem_u32(sA);
+      for (int u = tid; u < (BN / 4) * nr; u += 128) {
+        const int cg = u / nr, row = r0 + u % nr;
+        // all S loads in flight together, then the sum in split order
+        float4 p[kMaxClusterK];
+#pragma unroll
+        for (int q = 0; q < kMaxClusterK; ++q)
+          if (q < S) p[q] = ld_shared_cluster_v4(mapa(part + (cg * 128 + row) * 16, static_cast<uint32_t>(q)));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < kMaxClusterK; ++q)
+          if (q < S) {
+            acc.x += p[q].x;
+            acc.y += p[q].y;
+            acc.z += p[q].z;
+            acc.w += p[q].w;
+          }
+        const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
+        epi_stage<4>(e, nt * BN + 4 * cg, args.N, vals, stage, 4 * cg, row);
+      }
+      named_bar_sync(1, 128);
+      epi_flush(e, args.tok, m0, args.seg_rows[seg], nt * BN, BN, args.N, head, stage, tid, 128, args.status, r0,
+                r0 + nr);
+    }
+    cluster_sync();  // no CTA reads another's shared memory any more
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);

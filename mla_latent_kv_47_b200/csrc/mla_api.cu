@@ -213,12 +213,32 @@ struct GemmConfig {
 
 template <int BN, bool AMN, int STAGES, int KBB, int MT = 1>
 mla_status launch_tc(const GemmArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
-  constexpr int smem = GemmSmem<BN, STAGES, KBB, MT>::kBytes;
+  using L = GemmSmem<BN, STAGES, KBB, MT>;
+  constexpr int smem = L::kBytes;
   auto kern = gemm_tc_kernel<BN, AMN, STAGES, KBB, MT>;
   static std::atomic<unsigned long long> attr_done{0};
   const mla_status s = set_smem_limit(kern, smem, attr_done);
   if (s != MLA_OK) return s;
-  return launch(kern, grid, dim3(192), smem, st, pdl, a);
+  if (a.cluster_k <= 1) return launch(kern, grid, dim3(192), smem, st, pdl, a);
+  // the splits of a tile (grid z) form one cluster
+  if (!L::kClusterK || a.cluster_k > kMaxClusterK || static_cast<int>(grid.z) != a.cluster_k)
+    return MLA_ERR_UNSUPPORTED;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = a.cluster_k;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaLaunchKernelEx(&cfg, kern, a) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 // The instantiated configurations (bn, stages, K blocks per stage).
@@ -303,6 +323,21 @@ mla_status run_gemm_tc(const Ctx& c, const GemmSpec& g, const GemmConfig& cfg) {
   int kbps = (a.kb_total + splits - 1) / splits;
   kbps = (kbps + cfg.kbb - 1) / cfg.kbb * cfg.kbb;  // whole stages per split
   splits = (a.kb_total + kbps - 1) / kbps;
+  // Split-K inside clusters where the tile shape leaves room in shared memory
+  // for the partial and staging tiles: the S splits of a tile (S a power of
+  // two <= 8 that divides the K blocks into whole stages) sum their partials
+  // through distributed shared memory, with no fp32 round trip through HBM and
+  // no second kernel.
+  const bool cluster_fits = mt_per_cta == 1 && cfg.stages * cfg.kbb * 16384 >= 2 * bn * 128 * 4;
+  if (splits > 1 && cluster_fits) {
+    int S = 1;
+    while (2 * S <= kMaxClusterK && tiles * 2 * S <= target && a.kb_total % (2 * S * cfg.kbb) == 0) S *= 2;
+    if (S > 1) {
+      splits = S;
+      kbps = a.kb_total / S;
+      a.cluster_k = S;
+    }
+  }
   a.splits = splits;
   a.kb_per_split = kbps;
   a.partials = reinterpret_cast<float*>(c.ws + c.L.gpart);
@@ -311,7 +346,7 @@ mla_status run_gemm_tc(const Ctx& c, const GemmSpec& g, const GemmConfig& cfg) {
   k.mt = mt_per_cta;
   mla_status s = g.mode == GEMM_HEAD_MNMAJOR ? launch_tc_cfg<true>(k, a, grid, c.st, c.pdl)
                                             : launch_tc_cfg<false>(k, a, grid, c.st, c.pdl);
-  if (s != MLA_OK || splits == 1) return s;
+  if (s != MLA_OK || splits == 1 || a.cluster_k > 1) return s;
   // split-K: a wide second kernel sums the partials in split order and runs the epilogue
   const dim3 rgrid(m_tiles, bn / 4);
   switch (bn) {
