@@ -13,6 +13,7 @@
 #include "attn_prefill_tc.cuh"
 #include "gemm_tc.cuh"
 #include "simt.cuh"
+#include "uv_combine.cuh"
 
 using namespace mla;
 
@@ -245,6 +246,7 @@ mla_status launch_tc(const GemmArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
 template <bool AMN>
 mla_status launch_tc_cfg(const GemmConfig& k, const GemmArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
   if (k.mt == 4 && k.bn == 64 && k.stages == 2 && k.kbb == 1) return launch_tc<64, AMN, 2, 1, 4>(a, grid, st, pdl);
+  if (k.mt == 2 && k.bn == 64 && k.stages == 2 && k.kbb == 1) return launch_tc<64, AMN, 2, 1, 2>(a, grid, st, pdl);
   if (k.mt != 1) return MLA_ERR_UNSUPPORTED;
 #define MLA_GEMM_CFG(BN, S, KB) \
   if (k.bn == BN && k.stages == S && k.kbb == KB) return launch_tc<BN, AMN, S, KB>(a, grid, st, pdl);
@@ -410,7 +412,7 @@ mla_status run_gemm(const Ctx& c, const GemmSpec& g) {
     GemmConfig cfg = choose_gemm_config(g.N, c.num_sms);
     // per-head weight blocks of several 128-row tiles (W_UK^T: d_c rows per head)
     // share one X block: a CTA per head streams them all, one accumulator each
-    if (g.mode != GEMM_DENSE && g.N <= 64 && g.rows[0] % 512 == 0) cfg = {64, 2, 1, c.num_sms, 4};
+    if (g.mode != GEMM_DENSE && g.N <= 64 && g.rows[0] % 512 == 0) cfg = {64, 2, 1, c.num_sms, 2};
     return run_gemm_tc(c, g, cfg);
   }
   // fp32 storage (check_dims admits bf16 only with tensor-core shapes)
@@ -663,6 +665,30 @@ int decode_workers(const mla_dims& d, int num_sms) {
   return W < 1 ? 1 : W;
 }
 
+// a6 + a7 in one kernel (tensor-core path): combine the attention partials
+// into the W_UV product's B operand, o = W_UV_i o_lat_i, and write o_lat.
+mla_status launch_uv_combine(const Ctx& c, const mla_weights* w, const float* opart, const float* ml,
+                             const int* seg_start, int B, void* olat, void* o, const TokenMap& tk) {
+  const mla_dims& d = c.d;
+  const long long HD = static_cast<long long>(d.n_h) * d.d_h;
+  UvCombineArgs a;
+  memset(&a, 0, sizeof(a));
+  if (!make_map_2d(&a.mapA, w->W_UV, d.d_c, HD, d.d_c, 128)) return MLA_ERR_CUDA;
+  a.o_part = opart;
+  a.ml_part = ml;
+  a.seg_start = seg_start;
+  a.n_h = d.n_h;
+  a.N = B;
+  a.olat = static_cast<__nv_bfloat16*>(olat);
+  a.epi = epi_kind(EPI_PER_HEAD, o, HD, d.d_h, 0, 0, 1.f);
+  a.tok = tk;
+  a.status = c.status;
+  static std::atomic<unsigned long long> attr_done{0};
+  const mla_status s = set_smem_limit(uv_combine_kernel, uvc::kSmem, attr_done);
+  if (s != MLA_OK) return s;
+  return launch(uv_combine_kernel, dim3(d.n_h, (B + 63) / 64), dim3(uvc::kThreads), uvc::kSmem, c.st, c.pdl, a);
+}
+
 // The decode launch sequence (a1 .. a8 of the hot path) on an already checked
 // context; shared by mla_decode and the no-allocation variant.
 mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const mla_cache* cache,
@@ -786,7 +812,10 @@ mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const 
     if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
   }
   attn_event(g_attn_end, c.st);
-  {
+  if (tc_attn && tc_gemm_ok(d)) {
+    // ---- a6 + a7 fused: the combine feeds the absorbed W_UV product directly
+    if ((s = launch_uv_combine(c, w, opart, ml, seg_start, B, olat, o, tk)) != MLA_OK) return s;
+  } else {
     dim3 grid(B, (d.n_h + 3) / 4);  // one warp per (sequence, head)
     if (d.dtype == MLA_FP32)
       s = launch(combine_kernel<float>, grid, dim3(128), 0, c.st, c.pdl, opart, ml, seg_start, d.n_h, d.d_c,
@@ -795,9 +824,7 @@ mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const 
       s = launch(combine_kernel<__nv_bfloat16>, grid, dim3(128), 0, c.st, c.pdl, opart, ml, seg_start, d.n_h, d.d_c,
                  static_cast<__nv_bfloat16*>(olat));
     if (s != MLA_OK) return s;
-  }
-  // ---- a7: absorbed W_UV on the latent output: o_i = W_UV_i o_lat_i
-  {
+    // ---- a7: absorbed W_UV on the latent output: o_i = W_UV_i o_lat_i
     GemmSpec g;
     g.mode = GEMM_HEAD_KMAJOR;
     g.A[0] = w->W_UV;

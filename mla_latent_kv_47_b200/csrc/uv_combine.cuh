@@ -1,0 +1,221 @@
+// uv_combine.cuh -- the split-KV combine and the absorbed W_UV product of a
+// decode step in one kernel ("DeepSeek-V2 summary" (7shi.hateblo.jp), App. C:
+// the output o_t,i = W_UV_i sum_j softmax_j c^KV_j, with W_UV absorbed after
+// the attention over the latents):
+//
+//   o_lat[b,i] = sum_s 2^(m_s - M) O_s[i]  /  sum_s 2^(m_s - M) l_s     (M = max_s m_s)
+//   o[b,i]     = W_UV_i o_lat[b,i]
+//
+// over the pieces s of sequence b, from the attention kernel's unnormalised
+// partials O_s (fp32) and (m_s, l_s).  One CTA per (head i, 64 sequences):
+// eight warps combine the partials straight into the MMA's B operand in
+// shared memory (64 tokens x 512 latent columns, bf16, 128B swizzle, one K
+// block of 64 columns at a time so the MMAs start on the first block), while
+// the TMA brings the head's 128 x 512 block of W_UV; one thread issues
+// M = 128 (d_h rows), N = 64 tcgen05 MMAs over the 8 K blocks, and the
+// epilogue writes o through the GEMM's per-head epilogue.  The normalised
+// latents are also written out (bf16), as the separate combine did.
+//
+// The arithmetic is the two-kernel path's: the same weights, the same
+// accumulation order over the pieces, the same rounding to bf16, the same
+// MMA order over K.  Warp roles (320 threads): warp 0 TMA, warp 1 TMEM owner
+// and MMA issuer, warps 2-9 combine, warps 2-5 then the epilogue.
+#pragma once
+#include "epilogue.cuh"
+
+namespace mla {
+
+struct UvCombineArgs {
+  CUtensorMap mapA;      // W_UV [n_h d_h][d_c] bf16, box {64, 128}, 128B swizzle
+  const float* o_part;   // [slots][n_h][512] unnormalised partial latent outputs
+  const float* ml_part;  // [slots][n_h][2] (m, l) of each partial
+  const int* seg_start;  // [N + 1] first slot of each sequence
+  int n_h, N;            // heads, sequences (tokens)
+  __nv_bfloat16* olat;   // [N][n_h][512] the normalised latent outputs
+  Epi epi;               // EPI_PER_HEAD into o [N][n_h d_h]
+  TokenMap tok;
+  int* status;
+};
+
+namespace uvc {
+constexpr int kThreads = 320;
+constexpr int kKb = 8;                  // d_c / 64 K blocks
+constexpr int kSlabA = 128 * 128;       // 128 rows x 64 columns bf16
+constexpr int kSlabB = 64 * 128;        // 64 tokens x 64 columns bf16
+constexpr int kUnroll = 2;              // pieces whose loads are in flight together
+constexpr int kSmem = 1024 + kKb * kSlabA + kKb * kSlabB + 256;
+static_assert(kSmem <= 232448, "shared memory budget");
+}  // namespace uvc
+
+__global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __grid_constant__ UvCombineArgs a) {
+  using namespace uvc;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kKb * kSlabA;
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(sB + kKb * kSlabB);
+  uint64_t* b_full = a_full + kKb;
+  uint64_t* accum = b_full + kKb;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int head = blockIdx.x, nt = blockIdx.y;
+
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < kKb; ++k) {
+      mbar_init(&a_full[k], 1);
+      mbar_init(&b_full[k], 8);  // one arrival per combine warp
+    }
+    mbar_init(accum, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tmap(&a.mapA);
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 64);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  WaitCtx wc{a.status, abort_flag};
+  if (threadIdx.x == 0) griddep_launch_dependents();
+
+  if (warp == 0) {
+    // ---- the head's W_UV block: a weight, independent of earlier kernels,
+    // so it streams while the attention drains
+    if (elect_one()) {
+      const uint64_t pol = policy_evict_first();
+      for (int k = 0; k < kKb; ++k) {
+        mbar_arrive_expect_tx(&a_full[k], kSlabA);
+        tma_load_2d(sA + k * kSlabA, &a.mapA, &a_full[k], k * 64, head * 128, pol);
+      }
+      drain_ring(a_full, kKb, kKb);  // every load has landed before the CTA may leave
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);
+      for (int k = 0; k < kKb; ++k) {
+        if (!mbar_wait(&a_full[k], 0, wc) || !mbar_wait(&b_full[k], 0, wc)) break;
+        tc_fence_after();
+        const uint32_t ab = smem_u32(sA + k * kSlabA), bb = smem_u32(sB + k * kSlabB);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tmem, sdesc_sw128(ab + kk * 32, 16, 1024), sdesc_sw128(bb + kk * 32, 16, 1024), idesc,
+                 (k | kk) ? 1u : 0u);
+      }
+      mma_commit(accum);  // also after an abort: the epilogue then waits only for the MMAs issued
+    }
+  } else {
+    // ---- combine: thread t takes token nl = t / 4 of the tile and the 16
+    // columns [16 q, 16 q + 16) of every 64-column K block (q = t % 4)
+    griddep_wait();  // the partials come from the attention kernel
+    const int t = threadIdx.x - 64;
+    const int nl = t >> 2, q = t & 3;
+    const int n = nt * 64 + nl;
+    int s0 = 0, s1 = 0;
+    float M = -INFINITY, inv = 0.f;
+    if (n < a.N) {
+      s0 = a.seg_start[n];
+      s1 = a.seg_start[n + 1];
+      for (int s = s0; s < s1; ++s) M = fmaxf(M, a.ml_part[(static_cast<long long>(s) * a.n_h + head) * 2]);
+      float Ls = 0.f;
+      for (int s = s0; s < s1; ++s) {
+        const long long i = (static_cast<long long>(s) * a.n_h + head) * 2;
+        Ls += exp2f(a.ml_part[i] - M) * a.ml_part[i + 1];
+      }
+      inv = 1.f / Ls;
+    }
+    __nv_bfloat16* orow = a.olat + (static_cast<long long>(n) * a.n_h + head) * 512;
+    for (int k = 0; k < kKb; k += 2) {  // two K blocks per pass: 8 float4 loads of each piece in flight
+      float4 acc[2][4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[j][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sb = s0; sb < s1; sb += kUnroll) {
+        float wgt[kUnroll];
+        float4 v[kUnroll][2][4];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const bool on = sb + u < s1;
+          wgt[u] = on ? exp2f(a.ml_part[(static_cast<long long>(sb + u) * a.n_h + head) * 2] - M) : 0.f;
+          const float4* src =
+              reinterpret_cast<const float4*>(a.o_part + (static_cast<long long>(sb + u) * a.n_h + head) * 512);
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              v[u][j][i] = on ? __ldcs(src + ((k + j) * 64 + 16 * q) / 4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              acc[j][i].x += wgt[u] * v[u][j][i].x;
+              acc[j][i].y += wgt[u] * v[u][j][i].y;
+              acc[j][i].z += wgt[u] * v[u][j][i].z;
+              acc[j][i].w += wgt[u] * v[u][j][i].w;
+            }
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[j][i].x * inv, acc[j][i].y * inv);
+          const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[j][i].z * inv, acc[j][i].w * inv);
+          pk[2 * i] = *reinterpret_cast<const uint32_t*>(&lo);
+          pk[2 * i + 1] = *reinterpret_cast<const uint32_t*>(&hi);
+        }
+        const uint4 p0 = make_uint4(pk[0], pk[1], pk[2], pk[3]), p1 = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        // row nl of K block k + j: 16-byte pieces 2q and 2q + 1, swizzled by the row
+        uint8_t* row = sB + (k + j) * kSlabB + nl * 128;
+        *reinterpret_cast<uint4*>(row + (((2 * q) ^ (nl & 7)) << 4)) = p0;
+        *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ (nl & 7)) << 4)) = p1;
+        if (n < a.N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + (k + j) * 64 + 16 * q);
+          dst[0] = p0;
+          dst[1] = p1;
+        }
+      }
+      fence_proxy_async_smem();  // the MMAs read the tile through the async proxy
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&b_full[k]);
+        mbar_arrive(&b_full[k + 1]);
+      }
+    }
+    if (warp < 6) {
+      // ---- epilogue: warps 2..5, thread <-> TMEM lane (row m of W_UV_i)
+      const int q4 = warp & 3;
+      const int row = q4 * 32 + lane;
+      const uint32_t trow = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+      mbar_wait(accum, 0, wc);
+      tc_fence_after();
+      named_bar_sync(1, 128);  // every epilogue thread sees the same abort decision
+      if (!*abort_flag) {
+        uint8_t* stage = sA;   // every MMA retired: the A tiles are free
+#pragma unroll 1
+        for (int c = 0; c < 64; c += 16) {
+          float v[16];
+          tmem_ld16(trow + c, v);
+          tmem_wait_ld();
+          epi_stage<16>(a.epi, nt * 64 + c, a.N, v, stage, c, row);
+        }
+        named_bar_sync(1, 128);
+        epi_flush(a.epi, a.tok, 0, 128, nt * 64, 64, a.N, head, stage, threadIdx.x - 64, 128, a.status);
+      }
+    }
+  }
+  __syncwarp();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
+}  // namespace mla
