@@ -405,25 +405,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       ++piece;
       if constexpr (kFp8) {
         // ---- E4M3 rows: decode each raw stage of the piece into its bf16
-        // stage.  A warp takes one (row, 256-code segment) at a time: 32 lanes
-        // read 8 codes each (256 contiguous bytes) and write 16 bytes into one
-        // of the segment's four 128-byte swizzled chunk rows.
+        // stage.  A task is 512 codes: one own row (lanes 0-15 its codes
+        // 0-255, lanes 16-31 its codes 256-511) or two partner rows (one per
+        // half warp); a lane reads 16 codes (16 contiguous bytes) and writes
+        // two 16-byte pieces of one swizzled chunk row.  Warp cw takes tasks
+        // cw + 4 i, six at a time: their code and scale loads are issued
+        // before any conversion.
         const int cw = warp - 2;  // converter warp 0..3
-        const int cc = lane >> 3, u = lane & 7;
+        const int hl = lane >> 4, l16 = lane & 15;
+        constexpr int kTasks = kHalf + kHalf / 2, kBatch = 6;
+        static_assert(kTasks == 4 * 2 * kBatch, "converter tasks");
         for (int t = p.t0; t < p.t1; ++t, ++cv) {
           const int r = cv % kRS, s = cv % kStages;
           if (!mbar_wait(&raw_full[r], (cv / kRS) & 1, wc)) return;
           if (!mbar_wait(&empty[s], ((cv / kStages) & 1) ^ 1, wc)) return;
           const uint8_t* raw = raws + r * C::kRawBytes;
           uint8_t* st = stages + s * kStageBytes;
-          for (int task = cw; task < 3 * kHalf; task += 4) {
-            const int row = task % kHalf, seg = task / kHalf;  // seg 0, 1: own codes; 2: the partner's
-            const uint8_t* src = raw + (seg == 0 ? C::kRawOwn0 : seg == 1 ? C::kRawOwn1 : C::kRawPeer) + row * 256;
-            const int k = static_cast<int8_t>(raw[(seg < 2 ? C::kRawOwnS : C::kRawPeerS) + row * 16]);
-            const uint2 codes = *reinterpret_cast<const uint2*>(src + lane * 8);
-            const uint4 v = e4m3x8_to_bf16(codes, ldexpf(1.f, k));
-            const int chunk = (seg < 2 ? 4 * seg : kOwnChunks) + cc;
-            *reinterpret_cast<uint4*>(st + chunk * kChunkBytes + row * 128 + ((u ^ (row & 7)) << 4)) = v;
+          for (int i0 = 0; i0 < kTasks / 4; i0 += kBatch) {
+            uint4 codes[kBatch];
+            float scl[kBatch];
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+              const int task = cw + 4 * (i0 + i);
+              const bool own = task < kHalf;
+              const int row = own ? task : 2 * (task - kHalf) + hl;
+              const uint8_t* src = raw + (own ? (hl ? C::kRawOwn1 : C::kRawOwn0) : C::kRawPeer) + row * 256 + l16 * 16;
+              codes[i] = *reinterpret_cast<const uint4*>(src);
+              const int k = static_cast<int8_t>(raw[(own ? C::kRawOwnS : C::kRawPeerS) + row * 16]);
+              scl[i] = k >= -126 ? __int_as_float((k + 127) << 23) : ldexpf(1.f, k);  // 2^k
+            }
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+              const int task = cw + 4 * (i0 + i);
+              const bool own = task < kHalf;
+              const int row = own ? task : 2 * (task - kHalf) + hl;
+              const uint4 lo = e4m3x8_to_bf16(make_uint2(codes[i].x, codes[i].y), scl[i]);
+              const uint4 hi = e4m3x8_to_bf16(make_uint2(codes[i].z, codes[i].w), scl[i]);
+              // columns 16 l16 .. +15 of the 256-column segment: chunk l16 / 4,
+              // pieces 2 (l16 % 4) and +1; the half warps store opposite
+              // parities first, so each store spreads over all banks
+              const int chunk = (own ? 4 * hl : kOwnChunks) + (l16 >> 2);
+              uint8_t* dst = st + chunk * kChunkBytes + row * 128;
+              const int pc = 2 * (l16 & 3), sw = row & 7, f = hl ^ (row & 1);
+              *reinterpret_cast<uint4*>(dst + (((pc + f) ^ sw) << 4)) = f ? hi : lo;
+              *reinterpret_cast<uint4*>(dst + (((pc + (f ^ 1)) ^ sw) << 4)) = f ? lo : hi;
+            }
           }
           fence_proxy_async_smem();  // the MMAs read the stage through the async proxy
           __syncwarp();
