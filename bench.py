@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--workload", choices=["v2", "lite", "ragged"], default="v2")
     ap.add_argument("--ctx", type=int, default=0, help="override cached tokens per sequence (profiling cases)")
     ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling cases)")
+    ap.add_argument("--cache", choices=["dtype", "e4m3"], default="dtype",
+                    help="latent cache rows of the --profile run (the headline line is always bf16 rows)")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true", help="skip the V2-Lite and ragged decode objects")
@@ -428,7 +430,7 @@ def run_ours(args):
     g.manual_seed(1000 + rank)
     if args.profile_prefill:
         return profile_prefill(m, dev, g, args.profile_prefill, args.steps, barrier)
-    S = DecodeSetup(m, dev, g, args.workload, args.ctx, args.batch)
+    S = DecodeSetup(m, dev, g, args.workload, args.ctx, args.batch, cache=args.cache if args.profile else "dtype")
     d, L, B = S.p.dims, S.L, S.B
 
     for _ in range(max(args.warmup, 3)):

@@ -16,8 +16,9 @@
 // O[:, 256r, 256r + 256).  The pair splits every 64-token tile by tokens for
 // the scores: CTA r computes S for the tile's rows [32r, 32r + 32) over all
 // 576 columns (tcgen05.mma, M = 128 heads, N = 32, K = 576), the two CTAs
-// swap their per-head tile maxima (512 bytes) so both take the same max, and
-// each sends the bf16 P of its 32 rows (8 KB) into the partner's P buffer.
+// swap their per-head maxima of a piece's first tile (512 bytes) so both take
+// the same reference, and each sends the bf16 P of its 32 rows (8 KB) into
+// the partner's P buffer.
 // Both then run O_r += P C_r over all 64 rows (N = 256): CTA r TMA-loads its
 // own 32 rows whole and the partner's 32 rows in its own 256 columns, so the
 // pair reads the partner-row columns twice, the second time from L2.  A PV
@@ -32,7 +33,8 @@
 // tile whose scores rise past it sets FAULT_RANGE.
 //
 // Warp roles (448 threads per CTA):
-//   warp 0      TMA producer (3-stage ring)
+//   warp 0      TMA producer (bf16 rows: the three rings below; E4M3 rows:
+//               raw stages and bf16 stages)
 //   warp 1      TMEM owner and MMA issuer: S(j) once tile j landed and the S
 //               buffer was read out, PV(j) once both halves of P(j) are in place
 //   warps 2-5   Q_lat of each piece: chunks 0-6 (bf16 pairs) into TMEM, chunks
@@ -61,7 +63,6 @@ constexpr int kQTmemChunks = 7;                        // Q chunks held in TMEM;
 constexpr int kQSmemChunks = 9 - kQTmemChunks;
 constexpr int kQChunkBytes = 128 * 128;                // 128 heads x 64 columns, bf16
 constexpr int kPBytes = 128 * 128;                     // P: 128 heads x 64 rows, bf16 (CTA 0's rows first)
-constexpr int kPBufs = 2;
 constexpr int kMaxSlots = 4;                           // partner tile maxima in flight (tile j in slot j % 4)
 constexpr int kAuxBytes = 3072;                        // partner maxima, CTA 1's l, barriers
 // TMEM columns: O half [0,256), S [256,288), Q chunks 0-6 (bf16 pairs) [288,512)
@@ -70,9 +71,13 @@ constexpr float kRangeLog2 = 96.f;                     // largest exponent of P 
 constexpr int kRow = 576;                              // d_c + d_R
 static_assert(kTmemQ + kQTmemChunks * 32 == kTmemCols, "TMEM budget");
 
-// Stage layouts of the two cache formats.  The MMAs always read bf16 stages:
-// own rows' c^KV chunks 0-7 (and, for bf16 rows, the k^R chunk 8), then the
-// partner rows' chunks in this CTA's c^KV columns.  For E4M3 rows the TMA
+// Stage layouts of the two cache formats.  The MMAs always read bf16 tiles:
+// the own rows' c^KV chunks 0-7 and k^R chunk 8, and the partner rows'
+// chunks in this CTA's c^KV columns.  For bf16 rows the TMA loads them into
+// three rings, each released as soon as its last reader retired (ring A: the
+// own rows' chunks only the scores read; ring B: the own rows in this CTA's
+// columns; ring C: the partner rows), which keeps more tiles in flight than
+// whole 53 KB stages would in the same shared memory.  For E4M3 rows the TMA
 // fills a raw stage (k^R chunk in bf16 with the 128B swizzle, the own rows'
 // 512 code bytes as two boxes of 256, the partner rows' 256 code bytes in
 // this CTA's columns, and the scale bytes of both), and the converter warps
@@ -88,8 +93,28 @@ struct Cfg {
   static constexpr int kRawOwnS = 4096 + 3 * 8192, kRawPeerS = kRawOwnS + 512;
   static constexpr int kRawTx = kRawPeerS + 512;         // bytes the TMA brings per raw stage
   static constexpr int kRawBytes = kFp8 ? 30720 : 0;     // rounded up to 1 KB (the swizzled chunk's alignment)
-  // bf16 stages | raw stages | Q chunks 7-8 | P x 2 | aux
-  static constexpr int kSmem = 1024 + kStages * kStageBytes + kRawStages * kRawBytes + kQSmemChunks * kQChunkBytes +
+  // bf16 rows: three rings instead of whole stages, so that each part of a
+  // tile is held only as long as it is read.  Ring A: the own rows' chunks
+  // that only the scores read (the partner's c^KV columns and k^R), free
+  // once S retires.  Ring B: the own rows in this CTA's columns (S and PV).
+  // Ring C: the partner's rows in this CTA's columns (PV only), loaded when
+  // the PV before frees its slot.
+  static constexpr int kRingA = 2, kRingB = 5, kRingC = 2;
+  static constexpr int kABytes = 5 * kChunkBytes, kBBytes = 4 * kChunkBytes, kCBytes = 4 * kChunkBytes;
+  static constexpr int kStageRegion =
+      kFp8 ? kStages * kStageBytes : kRingA * kABytes + kRingB * kBBytes + kRingC * kCBytes;
+  static constexpr int kBars = kFp8 ? kStages : kRingA + kRingB + kRingC;  // full / empty barriers of the rings
+  static_assert(kFp8 || (kRingB >= kRingC && kRingB - kRingC < 8), "ring C trails ring B by fewer than 8 tiles");
+  // Ring C's load of tile g is issued with ring B's load of tile g + kRingB -
+  // kRingC, after ring A's load of tile g + kRingB - kRingC - 1, which waits
+  // for S(g + kRingB - kRingC - 1 - kRingA).  The last tile g of a piece needs
+  // its ring C load before the next piece's first S can issue, so that S
+  // index must not pass g.
+  static_assert(kFp8 || kRingB <= kRingA + kRingC + 1, "ring C's loads must not wait for a later piece");
+  // P buffers: P(g) is written once PV(g - kPBufs) retired in both CTAs
+  static constexpr int kPBufs = 2;
+  // stages (rings) | raw stages | Q chunks 7-8 | P x 2 | aux
+  static constexpr int kSmem = 1024 + kStageRegion + kRawStages * kRawBytes + kQSmemChunks * kQChunkBytes +
                                kPBufs * kPBytes + kAuxBytes;
   static_assert(kSmem <= 232448, "shared memory budget");
   static_assert(!kFp8 || kRawTx <= kRawBytes, "raw stage");
@@ -142,21 +167,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* stages = smem;
-  uint8_t* raws = stages + kStages * kStageBytes;     // E4M3 rows: raw stages (TMA)
+  uint8_t* raws = stages + C::kStageRegion;          // E4M3 rows: raw stages (TMA)
   uint8_t* qs = raws + C::kRawStages * C::kRawBytes;  // Q chunks 7-8, MMA A operand
-  uint8_t* pbuf = qs + kQSmemChunks * kQChunkBytes;   // [2] P (bf16), MMA A operand
-  uint8_t* aux = pbuf + kPBufs * kPBytes;
+  uint8_t* pbuf = qs + kQSmemChunks * kQChunkBytes;   // [kPBufs] P (bf16), MMA A operand
+  uint8_t* aux = pbuf + C::kPBufs * kPBytes;
   float* mx = reinterpret_cast<float*>(aux);          // [4][128] the partner's tile maxima (st.async)
   float* lsh = mx + kMaxSlots * 128;                  // [128] CTA 1's share of l, in CTA 0 (st.async)
   uint64_t* full = reinterpret_cast<uint64_t*>(aux + 2560);
-  uint64_t* empty = full + kStages;
-  uint64_t* s_full = empty + kStages;  // S(j) in TMEM (MMA -> softmax)
+  uint64_t* empty = full + C::kBars;
+  uint64_t* s_full = empty + C::kBars;  // S(j) in TMEM (MMA -> softmax)
   uint64_t* s_free = s_full + 1;       // S read out (softmax -> MMA)
   uint64_t* mx_full = s_free + 1;      // [4] the partner's maxima of tile j landed (slot j % 4)
-  uint64_t* p_full = mx_full + kMaxSlots;  // [2] this CTA's half of P(j) written
-  uint64_t* px_full = p_full + 2;      // [2] the partner's half of P(j) landed
-  uint64_t* pv_done = px_full + 2;     // [2] PV(j) retired in both CTAs (one commit from each)
-  uint64_t* q_full = pv_done + 2;
+  constexpr int kPB = C::kPBufs;
+  uint64_t* p_full = mx_full + kMaxSlots;  // [kPB] this CTA's half of P(j) written (buffer j % kPB)
+  uint64_t* px_full = p_full + kPB;    // [kPB] the partner's half of P(j) landed
+  uint64_t* pv_done = px_full + kPB;   // [kPB] PV(j) retired in both CTAs (one commit from each)
+  uint64_t* q_full = pv_done + kPB;
   uint64_t* q_free = q_full + 1;       // last S of the piece retired (MMA -> Q warps)
   uint64_t* o_done = q_free + 1;
   uint64_t* l_full = o_done + 1;       // CTA 0: CTA 1's l of the piece landed
@@ -164,6 +190,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   uint64_t* raw_full = drain + 1;      // [2] E4M3 rows: raw stage loaded (TMA)
   uint64_t* raw_empty = raw_full + 2;  // [2] E4M3 rows: raw stage read by the converter and by S's k^R MMAs
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(raw_empty + 2);
+  static_assert(2560 + (2 * C::kBars + 15 + 3 * C::kPBufs) * 8 + 8 <= kAuxBytes, "aux layout: maxima, l, barriers");
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const uint32_t rank = cluster_ctarank();
@@ -172,7 +199,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::kBars; ++s) {
       mbar_init(&full[s], kFp8 ? 4 : 1);  // E4M3 rows: one arrival per converter warp
       mbar_init(&empty[s], 1);
     }
@@ -183,7 +210,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     mbar_init(s_full, 1);
     mbar_init(s_free, 8);        // one arrival per softmax warp
     for (int i = 0; i < kMaxSlots; ++i) mbar_init(&mx_full[i], 1);  // armed per phase with the partner's 512 bytes
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kPB; ++i) {
       mbar_init(&p_full[i], 8);   // one arrival per softmax warp
       mbar_init(&px_full[i], 1);  // armed per phase with the partner's 8 KB
       mbar_init(&pv_done[i], 2);  // this CTA's and the partner's PV commit
@@ -196,7 +223,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
     for (int i = 0; i < kMaxSlots; ++i) mbar_arrive_expect_tx(&mx_full[i], 128 * 4);
-    for (int i = 0; i < 2; ++i) mbar_arrive_expect_tx(&px_full[i], kPBytes / 2);
+    for (int i = 0; i < kPB; ++i) mbar_arrive_expect_tx(&px_full[i], kPBytes / 2);
     if (rank == 0) mbar_arrive_expect_tx(l_full, 128 * 4);
   }
   if (warp == 0 && lane == 0) {
@@ -216,6 +243,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   griddep_wait();  // Q_lat and the new cache rows come from the preceding kernels
   WaitCtx wc{a.status, abort_flag};
+  // bf16 rows: slots of tile g in the three rings, and their barriers
+  constexpr int kRA = C::kRingA, kRB = C::kRingB, kRC = C::kRingC;
+  uint8_t* const ring_a = stages;
+  uint8_t* const ring_b = ring_a + kRA * C::kABytes;
+  uint8_t* const ring_c = ring_b + kRB * C::kBBytes;
+  auto slot_a = [&](int g) { return ring_a + (g % kRA) * C::kABytes; };
+  auto slot_b = [&](int g) { return ring_b + (g % kRB) * C::kBBytes; };
+  auto slot_c = [&](int g) { return ring_c + (g % kRC) * C::kCBytes; };
+  auto bar_a = [&](int g) { return g % kRA; };
+  auto bar_b = [&](int g) { return kRA + g % kRB; };
+  auto bar_c = [&](int g) { return kRA + kRB + g % kRC; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -225,6 +263,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       const uint64_t pol_once = policy_evict_first();
       const uint64_t pol_twice = policy_evict_normal();
       int it = 0;
+      int n_a = 0, n_b = 0, n_c = 0;  // bf16 rows: loads issued into each ring
+      int yp_hist[8];                 // bf16 rows: the partner rows' start of the last 8 tiles
+      // bf16 rows: ring C's chunks of tile gc (the partner's rows in this CTA's columns)
+      auto load_c = [&](int gc) -> bool {
+        if (!mbar_wait(&empty[bar_c(gc)], ((gc / kRC) & 1) ^ 1, wc)) return false;
+        mbar_arrive_expect_tx(&full[bar_c(gc)], C::kCBytes);
+        for (int j = 0; j < 4; ++j)
+          tma_load_2d(slot_c(gc) + j * kChunkBytes, &a.map_cache, &full[bar_c(gc)],
+                      (4 * static_cast<int>(rank) + j) * 64, yp_hist[gc & 7], pol_twice);
+        ++n_c;
+        return true;
+      };
       for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
         if (*abort_flag) return;
         const long long row0 = a.lay.block_table ? 0 : a.lay.seq_start[p.b];  // contiguous layout
@@ -249,24 +299,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
             tma_load_2d(dst + C::kRawPeerS, &a.map_scale, &raw_full[r], a.scale_x, y_peer, pol_twice);
             continue;
           }
-          const int s = it % kStages;
-          if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, wc)) return;
-          mbar_arrive_expect_tx(&full[s], kStageBytes);
-          uint8_t* dst = stages + s * kStageBytes;
+          // tile it: ring C's chunks of tile it - (kRB - kRC) first (its slot
+          // frees with the same PV as ring B's slot of tile it), then ring A
+          // (the own rows' score-only chunks) and ring B (the own rows in this
+          // CTA's columns)
           const int y_own = static_cast<int>(y0 + kHalf * rank), y_peer = static_cast<int>(y0 + kHalf * peer);
-          for (int ci = 0; ci < kOwnChunks; ++ci) {
-            const bool shared = ci >= 4 * static_cast<int>(peer) && ci < 4 * static_cast<int>(peer) + 4;
-            tma_load_2d(dst + ci * kChunkBytes, &a.map_cache, &full[s], ci * 64, y_own, shared ? pol_twice : pol_once);
-          }
-          for (int cj = 0; cj < kPeerChunks; ++cj)
-            tma_load_2d(dst + (kOwnChunks + cj) * kChunkBytes, &a.map_cache, &full[s],
-                        (4 * static_cast<int>(rank) + cj) * 64, y_peer, pol_twice);
+          yp_hist[it & 7] = y_peer;
+          if (it - (kRB - kRC) >= 0 && !load_c(it - (kRB - kRC))) return;
+          if (!mbar_wait(&empty[bar_a(it)], ((it / kRA) & 1) ^ 1, wc)) return;
+          mbar_arrive_expect_tx(&full[bar_a(it)], C::kABytes);
+          for (int j = 0; j < 4; ++j)  // the partner reads these rows in its columns too
+            tma_load_2d(slot_a(it) + j * kChunkBytes, &a.map_cache, &full[bar_a(it)], (4 * static_cast<int>(peer) + j) * 64,
+                        y_own, pol_twice);
+          tma_load_2d(slot_a(it) + 4 * kChunkBytes, &a.map_cache, &full[bar_a(it)], 512, y_own, pol_once);
+          ++n_a;
+          if (!mbar_wait(&empty[bar_b(it)], ((it / kRB) & 1) ^ 1, wc)) return;
+          mbar_arrive_expect_tx(&full[bar_b(it)], C::kBBytes);
+          for (int j = 0; j < 4; ++j)
+            tma_load_2d(slot_b(it) + j * kChunkBytes, &a.map_cache, &full[bar_b(it)], (4 * static_cast<int>(rank) + j) * 64,
+                        y_own, pol_once);
+          ++n_b;
         }
       });
+      if constexpr (!kFp8) {
+        for (int gc = it - (kRB - kRC) > 0 ? it - (kRB - kRC) : 0; gc < it && !*abort_flag; ++gc)
+          if (!load_c(gc)) break;
+      }
       // every load issued has landed before the CTA may leave (after an abort,
       // loads can still be in flight into stages nobody consumes)
-      if constexpr (kFp8) drain_ring(raw_full, kRS, it);
-      else drain_ring(full, kStages, it);
+      if constexpr (kFp8) {
+        drain_ring(raw_full, kRS, it);
+      } else {
+        drain_ring(full + bar_a(0), kRA, n_a);
+        drain_ring(full + bar_b(0), kRB, n_b);
+        drain_ring(full + bar_c(0), kRC, n_c);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -287,17 +354,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           if (npv < ns) {
             const int g = it + npv;
             const int s = g % kStages;
-            const int b = g & 1;
-            const uint32_t ph = (g >> 1) & 1;
-            if (mbar_test_wait(smem_u32(&p_full[b]), ph) && mbar_test_wait_cluster(smem_u32(&px_full[b]), ph)) {
+            const int b = g % kPB;
+            const uint32_t ph = (g / kPB) & 1;
+            // bf16 rows: the partner rows' chunks come with ring C
+            const bool c_ready = kFp8 || mbar_test_wait(smem_u32(&full[bar_c(g)]), (g / kRC) & 1);
+            if (c_ready && mbar_test_wait(smem_u32(&p_full[b]), ph) &&
+                mbar_test_wait_cluster(smem_u32(&px_full[b]), ph)) {
               tc_fence_after();
               fence_proxy_async_smem();  // the partner's half came in through st.async
-              // next phase: the partner's half of P(g + 2), which it sends only
-              // after this PV retired
+              // next phase: the partner's half of P(g + kPB), which it sends
+              // only after this PV retired
               mbar_arrive_expect_tx(&px_full[b], kPBytes / 2);
               const uint32_t st = smem_u32(stages + s * kStageBytes);
-              const uint32_t own_rows = st + 4 * rank * kChunkBytes;      // own rows, this CTA's c^KV columns
-              const uint32_t peer_rows = st + kOwnChunks * kChunkBytes;   // partner rows, the same columns
+              // own rows and partner rows, this CTA's c^KV columns
+              const uint32_t own_rows = kFp8 ? st + 4 * rank * kChunkBytes : smem_u32(slot_b(g));
+              const uint32_t peer_rows = kFp8 ? st + kOwnChunks * kChunkBytes : smem_u32(slot_c(g));
               const uint32_t pb = smem_u32(pbuf + b * kPBytes);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {  // rows [16 kk, 16 kk + 16) of the tile; CTA 0's rows first
@@ -306,7 +377,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
                        sdesc_sw128(rows + (kk & 1) * 2048, kChunkBytes, 1024), idesc_pv, (npv > 0 || kk > 0) ? 1u : 0u);
               }
               mma_commit_multicast(&pv_done[b], 0x3);  // P buffer b is free in both CTAs once both commits land
-              mma_commit(&empty[s]);
+              if constexpr (kFp8) {
+                mma_commit(&empty[s]);
+              } else {
+                mma_commit(&empty[bar_b(g)]);
+                mma_commit(&empty[bar_c(g)]);
+              }
               if (npv == nt - 1) mma_commit(o_done);
               ++npv;
               issued = true;
@@ -315,23 +391,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           if (!issued && ns < nt) {
             const int g = it + ns;
             const int s = g % kStages;
-            if (mbar_test_wait(smem_u32(&full[s]), (g / kStages) & 1) &&
-                mbar_test_wait(smem_u32(s_free), (g & 1) ^ 1)) {
+            const bool data = kFp8 ? mbar_test_wait(smem_u32(&full[s]), (g / kStages) & 1)
+                                   : mbar_test_wait(smem_u32(&full[bar_a(g)]), (g / kRA) & 1) &&
+                                         mbar_test_wait(smem_u32(&full[bar_b(g)]), (g / kRB) & 1);
+            if (data && mbar_test_wait(smem_u32(s_free), (g & 1) ^ 1)) {
               tc_fence_after();
               const uint32_t st = smem_u32(stages + s * kStageBytes);
+              // the own rows' chunk ci (64 columns; 8 = k^R): E4M3 rows keep
+              // c^KV in the bf16 stage and k^R in the raw stage; bf16 rows
+              // keep this CTA's columns in ring B and the rest in ring A
+              auto own_chunk = [&](int ci) -> uint32_t {
+                if constexpr (kFp8) {
+                  return ci == 8 ? smem_u32(raws + (g % kRS) * C::kRawBytes + C::kRawKr) : st + ci * kChunkBytes;
+                } else {
+                  const int r4 = 4 * static_cast<int>(rank);
+                  if (ci >= r4 && ci < r4 + 4) return smem_u32(slot_b(g)) + (ci - r4) * kChunkBytes;
+                  return smem_u32(slot_a(g)) + (ci < 8 ? ci - 4 * static_cast<int>(peer) : 4) * kChunkBytes;
+                }
+              };
               const uint32_t dS = tmem + kTmemS;
               for (int ci = 0; ci < kQTmemChunks; ++ci) {
+                const uint32_t bchunk = own_chunk(ci);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                  mma_ts(dS, tmem + kTmemQ + ci * 32 + kk * 8, sdesc_sw128(st + ci * kChunkBytes + kk * 32, 16, 1024),
+                  mma_ts(dS, tmem + kTmemQ + ci * 32 + kk * 8, sdesc_sw128(bchunk + kk * 32, 16, 1024),
                          idesc_s, (ci | kk) ? 1u : 0u);
                 }
               }
               for (int ci = 0; ci < kQSmemChunks; ++ci) {
-                const int chunk = kQTmemChunks + ci;
-                // E4M3 rows: k^R (chunk 8) stays in the raw stage, already bf16
-                const uint32_t bchunk = (kFp8 && chunk == 8) ? smem_u32(raws + (g % kRS) * C::kRawBytes + C::kRawKr)
-                                                             : st + chunk * kChunkBytes;
+                const uint32_t bchunk = own_chunk(kQTmemChunks + ci);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                   mma_ss(dS, sdesc_sw128(smem_u32(qs) + ci * kQChunkBytes + kk * 32, 16, 1024),
@@ -340,6 +428,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
               }
               mma_commit(s_full);
               if constexpr (kFp8) mma_commit(&raw_empty[g % kRS]);  // the raw stage's k^R was read
+              else mma_commit(&empty[bar_a(g)]);                     // ring A is read by S only
               if (ns == nt - 1) mma_commit(q_free);  // no MMA of this piece reads Q any more
               ++ns;
               issued = true;
@@ -493,8 +582,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       const int nt = p.t1 - p.t0;
       for (int k = 0; k < nt; ++k) {
         const int g = it + k;
-        const int b = g & 1;
-        const uint32_t ph = (g >> 1) & 1;
+        const int b = g % kPB;
+        const uint32_t ph = (g / kPB) & 1;
         if (!mbar_wait(s_full, g & 1, wc)) return;
         tc_fence_after();
         uint32_t sr[16];
@@ -545,7 +634,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
         }
         l_run += lsum;
-        // ---- P buffer b is free in both CTAs once PV(g-2) retired in both
+        // ---- P buffer b is free in both CTAs once PV(g - kPB) retired in both
         if (!mbar_wait_inline(&pv_done[b], ph ^ 1, wc)) return;
         tc_fence_after();
         const int v64 = min(kAttnTileTokens, L1 - tile0);  // valid rows of the tile
@@ -553,12 +642,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
           // rows past the sequence may hold anything (even NaN); 0 * NaN would
           // poison O, so the rows this CTA multiplies into O are zeroed
           uint8_t* st = stages + (g % kStages) * kStageBytes;
+          // bf16 rows: the partner rows' chunks come with ring C, maybe later.
+          // A parity wait only tells apart phases one apart, so the slot's
+          // previous load (tile g - kRC) must have landed first: its PV has
+          // retired (PV(g - kPB) did, above; a later one is waited for here).
+          if constexpr (!kFp8) {
+            if (kRC < kPB && g >= kRC &&
+                !mbar_wait_inline(&pv_done[(g - kRC) % kPB], ((g - kRC) / kPB) & 1, wc))
+              return;
+            if (!mbar_wait(&full[bar_c(g)], (g / kRC) & 1, wc)) return;
+          }
           const int n16 = (kAttnTileTokens - v64) * 32;  // 16-byte pieces: 4 chunks x 8 per row
           for (int idx = (warp - 6) * 32 + lane; idx < n16; idx += 256) {
             const int row = v64 + (idx >> 5), c16 = idx & 31;
             const bool own = (row >> 5) == static_cast<int>(rank);
-            const int chunk = (own ? 4 * static_cast<int>(rank) : kOwnChunks) + (c16 >> 3);
-            *reinterpret_cast<uint4*>(st + chunk * kChunkBytes + (row & 31) * 128 + (c16 & 7) * 16) = make_uint4(0, 0, 0, 0);
+            uint8_t* base = kFp8 ? st + (own ? 4 * static_cast<int>(rank) : kOwnChunks) * kChunkBytes
+                                 : (own ? slot_b(g) : slot_c(g));
+            *reinterpret_cast<uint4*>(base + (c16 >> 3) * kChunkBytes + (row & 31) * 128 + (c16 & 7) * 16) =
+                make_uint4(0, 0, 0, 0);
           }
         }
         // ---- this CTA's half of P(g): rows [32 rank + 16 th, +16) of the tile,
@@ -607,11 +708,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       it += nt;
       ++piece;
     });
-    // The partner's PV commits for the last uses of both P buffers land in
+    // The partner's PV commits for the last uses of the P buffers land in
     // this CTA's shared memory: they must have arrived before the CTA may exit.
     if (lead && !*abort_flag) {
-      for (int b = 0; b < 2; ++b) {
-        const int uses = (it + 1 - b) / 2;  // tiles g < it with g & 1 == b
+      for (int b = 0; b < kPB; ++b) {
+        const int uses = (it + kPB - 1 - b) / kPB;  // tiles g < it with g % kPB == b
         if (uses > 0 && !mbar_wait<true>(&pv_done[b], (uses - 1) & 1, wc)) break;
       }
     }
