@@ -32,18 +32,20 @@
 // rescaled.  The kernel's range is P <= 2^96 (ample for fp32 O and l); a
 // tile whose scores rise past it sets FAULT_RANGE.
 //
-// Warp roles (448 threads per CTA):
+// Warp roles (448 threads per CTA; 576 for E4M3 rows):
 //   warp 0      TMA producer (bf16 rows: the three rings below; E4M3 rows:
 //               raw stages and bf16 stages)
 //   warp 1      TMEM owner and MMA issuer: S(j) once tile j landed and the S
 //               buffer was read out, PV(j) once both halves of P(j) are in place
 //   warps 2-5   Q_lat of each piece: chunks 0-6 (bf16 pairs) into TMEM, chunks
-//               7-8 into shared memory, both MMA A operands
+//               7-8 into shared memory, both MMA A operands; for E4M3 rows
+//               also half of the decode of each raw stage into a bf16 stage
 //   warps 6-13  softmax: warp 6+i and warp 10+i share lane quarter i mod 4,
 //               16 heads each; two threads per head (rows 0-15 and 16-31 of
 //               this CTA's half, via the 16-lane TMEM access shape).  Softmax
 //               against the piece's reference max (above), and the per-piece
 //               epilogue; CTA 1 sends its share of l to CTA 0.
+//   warps 14-17 E4M3 rows only: the other half of the decode
 #pragma once
 #include "mla.h"
 #include "ptx.cuh"
@@ -55,7 +57,6 @@ constexpr int kAttnTileTokens = 64;
 constexpr bool kAttnTcReady = true;
 
 namespace attn {
-constexpr int kThreads = 448;
 constexpr int kHalf = 32;                              // rows of a tile whose scores one CTA computes
 constexpr int kChunkBytes = kHalf * 128;               // 32 token rows x 64 latent columns, bf16, 128B swizzle
 constexpr int kPeerChunks = 4;                         // partner's rows: this CTA's 256 c^KV columns
@@ -113,6 +114,11 @@ struct Cfg {
   static_assert(kFp8 || kRingB <= kRingA + kRingC + 1, "ring C's loads must not wait for a later piece");
   // P buffers: P(g) is written once PV(g - kPBufs) retired in both CTAs
   static constexpr int kPBufs = 2;
+  // E4M3 rows: the decode, bound by its latency rather than its arithmetic,
+  // is split over eight warps, the four Q warps and four more (warps 14-17)
+  // that do nothing else
+  static constexpr int kConvWarps = kFp8 ? 8 : 0;
+  static constexpr int kThreads = kFp8 ? 576 : 448;
   // stages (rings) | raw stages | Q chunks 7-8 | P x 2 | aux
   static constexpr int kSmem = 1024 + kStageRegion + kRawStages * kRawBytes + kQSmemChunks * kQChunkBytes +
                                kPBufs * kPBytes + kAuxBytes;
@@ -156,7 +162,7 @@ __device__ __forceinline__ uint4 e4m3x8_to_bf16(uint2 raw, float scale) {
 }
 
 template <bool kFp8>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::Cfg<kFp8>::kThreads, 1)
     attn_decode_tc_kernel(const __grid_constant__ AttnArgs a) {
   using namespace attn;
   using C = Cfg<kFp8>;
@@ -200,12 +206,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kBars; ++s) {
-      mbar_init(&full[s], kFp8 ? 4 : 1);  // E4M3 rows: one arrival per converter warp
+      mbar_init(&full[s], kFp8 ? C::kConvWarps : 1);  // E4M3 rows: one arrival per converter warp
       mbar_init(&empty[s], 1);
     }
     for (int r = 0; r < C::kRawStages; ++r) {
       mbar_init(&raw_full[r], 1);
-      mbar_init(&raw_empty[r], 5);        // four converter warps and the commit after S
+      mbar_init(&raw_empty[r], C::kConvWarps + 1);  // the converter warps and the commit after S
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 8);        // one arrival per softmax warp
@@ -254,6 +260,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
   auto bar_a = [&](int g) { return g % kRA; };
   auto bar_b = [&](int g) { return kRA + g % kRB; };
   auto bar_c = [&](int g) { return kRA + kRB + g % kRC; };
+
+  // E4M3 rows: decode raw stage cv into its bf16 stage, warp cw's share.  A
+  // task is 512 codes: one own row (lanes 0-15 its codes 0-255, lanes 16-31
+  // its codes 256-511) or two partner rows (one per half warp); a lane reads
+  // 16 codes (16 contiguous bytes) and writes two 16-byte pieces of one
+  // swizzled chunk row.  Warp cw takes tasks cw + kConvWarps i; their code
+  // and scale loads are all issued before any conversion.
+  auto convert_tile = [&](int cw, int cv) -> bool {
+    constexpr int kCW = C::kConvWarps > 0 ? C::kConvWarps : 1;
+    constexpr int kTasks = kHalf + kHalf / 2, kBatch = kTasks / kCW;
+    static_assert(!kFp8 || kTasks == kCW * kBatch, "converter tasks");
+    const int hl = lane >> 4, l16 = lane & 15;
+    const int r = cv % kRS, s = cv % kStages;
+    if (!mbar_wait(&raw_full[r], (cv / kRS) & 1, wc)) return false;
+    if (!mbar_wait(&empty[s], ((cv / kStages) & 1) ^ 1, wc)) return false;
+    const uint8_t* raw = raws + r * C::kRawBytes;
+    uint8_t* st = stages + s * kStageBytes;
+    uint4 codes[kBatch];
+    float scl[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int task = cw + kCW * i;
+      const bool own = task < kHalf;
+      const int row = own ? task : 2 * (task - kHalf) + hl;
+      const uint8_t* src = raw + (own ? (hl ? C::kRawOwn1 : C::kRawOwn0) : C::kRawPeer) + row * 256 + l16 * 16;
+      codes[i] = *reinterpret_cast<const uint4*>(src);
+      const int k = static_cast<int8_t>(raw[(own ? C::kRawOwnS : C::kRawPeerS) + row * 16]);
+      scl[i] = k >= -126 ? __int_as_float((k + 127) << 23) : ldexpf(1.f, k);  // 2^k
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int task = cw + kCW * i;
+      const bool own = task < kHalf;
+      const int row = own ? task : 2 * (task - kHalf) + hl;
+      const uint4 lo = e4m3x8_to_bf16(make_uint2(codes[i].x, codes[i].y), scl[i]);
+      const uint4 hi = e4m3x8_to_bf16(make_uint2(codes[i].z, codes[i].w), scl[i]);
+      // columns 16 l16 .. +15 of the 256-column segment: chunk l16 / 4,
+      // pieces 2 (l16 % 4) and +1; the half warps store opposite parities
+      // first, so each store spreads over all banks
+      const int chunk = (own ? 4 * hl : kOwnChunks) + (l16 >> 2);
+      uint8_t* dst = st + chunk * kChunkBytes + row * 128;
+      const int pc = 2 * (l16 & 3), sw = row & 7, f = hl ^ (row & 1);
+      *reinterpret_cast<uint4*>(dst + (((pc + f) ^ sw) << 4)) = f ? hi : lo;
+      *reinterpret_cast<uint4*>(dst + (((pc + (f ^ 1)) ^ sw) << 4)) = f ? lo : hi;
+    }
+    fence_proxy_async_smem();  // the MMAs read the stage through the async proxy
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&full[s]);
+      mbar_arrive(&raw_empty[r]);
+    }
+    return true;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -493,61 +552,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(attn::kThreads, 1)
       mbar_arrive(q_full);
       ++piece;
       if constexpr (kFp8) {
-        // ---- E4M3 rows: decode each raw stage of the piece into its bf16
-        // stage.  A task is 512 codes: one own row (lanes 0-15 its codes
-        // 0-255, lanes 16-31 its codes 256-511) or two partner rows (one per
-        // half warp); a lane reads 16 codes (16 contiguous bytes) and writes
-        // two 16-byte pieces of one swizzled chunk row.  Warp cw takes tasks
-        // cw + 4 i, six at a time: their code and scale loads are issued
-        // before any conversion.
-        const int cw = warp - 2;  // converter warp 0..3
-        const int hl = lane >> 4, l16 = lane & 15;
-        constexpr int kTasks = kHalf + kHalf / 2, kBatch = 6;
-        static_assert(kTasks == 4 * 2 * kBatch, "converter tasks");
-        for (int t = p.t0; t < p.t1; ++t, ++cv) {
-          const int r = cv % kRS, s = cv % kStages;
-          if (!mbar_wait(&raw_full[r], (cv / kRS) & 1, wc)) return;
-          if (!mbar_wait(&empty[s], ((cv / kStages) & 1) ^ 1, wc)) return;
-          const uint8_t* raw = raws + r * C::kRawBytes;
-          uint8_t* st = stages + s * kStageBytes;
-          for (int i0 = 0; i0 < kTasks / 4; i0 += kBatch) {
-            uint4 codes[kBatch];
-            float scl[kBatch];
-#pragma unroll
-            for (int i = 0; i < kBatch; ++i) {
-              const int task = cw + 4 * (i0 + i);
-              const bool own = task < kHalf;
-              const int row = own ? task : 2 * (task - kHalf) + hl;
-              const uint8_t* src = raw + (own ? (hl ? C::kRawOwn1 : C::kRawOwn0) : C::kRawPeer) + row * 256 + l16 * 16;
-              codes[i] = *reinterpret_cast<const uint4*>(src);
-              const int k = static_cast<int8_t>(raw[(own ? C::kRawOwnS : C::kRawPeerS) + row * 16]);
-              scl[i] = k >= -126 ? __int_as_float((k + 127) << 23) : ldexpf(1.f, k);  // 2^k
-            }
-#pragma unroll
-            for (int i = 0; i < kBatch; ++i) {
-              const int task = cw + 4 * (i0 + i);
-              const bool own = task < kHalf;
-              const int row = own ? task : 2 * (task - kHalf) + hl;
-              const uint4 lo = e4m3x8_to_bf16(make_uint2(codes[i].x, codes[i].y), scl[i]);
-              const uint4 hi = e4m3x8_to_bf16(make_uint2(codes[i].z, codes[i].w), scl[i]);
-              // columns 16 l16 .. +15 of the 256-column segment: chunk l16 / 4,
-              // pieces 2 (l16 % 4) and +1; the half warps store opposite
-              // parities first, so each store spreads over all banks
-              const int chunk = (own ? 4 * hl : kOwnChunks) + (l16 >> 2);
-              uint8_t* dst = st + chunk * kChunkBytes + row * 128;
-              const int pc = 2 * (l16 & 3), sw = row & 7, f = hl ^ (row & 1);
-              *reinterpret_cast<uint4*>(dst + (((pc + f) ^ sw) << 4)) = f ? hi : lo;
-              *reinterpret_cast<uint4*>(dst + (((pc + (f ^ 1)) ^ sw) << 4)) = f ? lo : hi;
-            }
-          }
-          fence_proxy_async_smem();  // the MMAs read the stage through the async proxy
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&full[s]);
-            mbar_arrive(&raw_empty[r]);
-          }
-        }
+        // ---- E4M3 rows: this warp's share of the decode of the piece's tiles
+        for (int t = p.t0; t < p.t1; ++t, ++cv)
+          if (!convert_tile(warp - 2, cv)) return;
       }
+    });
+  } else if (warp >= 14) {
+    // ------------------------------------------------------------ E4M3 rows: the
+    // other converter warps
+    int cv = 0;
+    for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
+      if (*abort_flag) return;
+      for (int t = p.t0; t < p.t1; ++t, ++cv)
+        if (!convert_tile(4 + warp - 14, cv)) return;
     });
   } else {
     // ------------------------------------------------------------ softmax + epilogue

@@ -615,7 +615,8 @@ mla_status launch_attn_kernel(const AttnArgs& a, int W, cudaStream_t st, bool pd
   static std::atomic<unsigned long long> attr_done{0};
   const mla_status s = set_smem_limit(attn_decode_tc_kernel<kFp8>, attn::Cfg<kFp8>::kSmem, attr_done);
   if (s != MLA_OK) return s;
-  return launch(attn_decode_tc_kernel<kFp8>, dim3(2 * W), dim3(attn::kThreads), attn::Cfg<kFp8>::kSmem, st, pdl, a);
+  return launch(attn_decode_tc_kernel<kFp8>, dim3(2 * W), dim3(attn::Cfg<kFp8>::kThreads), attn::Cfg<kFp8>::kSmem, st,
+                pdl, a);
 }
 
 mla_status launch_attn_decode_tc(const mla_dims& d, const __nv_bfloat16* qlat, const mla_cache* cache,
