@@ -62,6 +62,14 @@ struct GemmSmem {
   static constexpr int kBytes = 1024 + STAGES * kStage + 256;
   // cluster split-K keeps the fp32 partial tile and a staging tile in the A buffers
   static constexpr bool kClusterK = MT == 1 && STAGES * kA >= 2 * BN * 128 * 4;
+  // token columns the idle pipeline buffers stage at once (fp32 staging): all
+  // BN, or the largest power of two that fits
+  static constexpr int stage_cols() {
+    int c = BN;
+    while (c > 16 && c * 128 * 4 > STAGES * kStage) c /= 2;
+    return c;
+  }
+  static constexpr int kStageCols = stage_cols();
 };
 
 // MT > 1 (per-head modes, no split-K): one CTA computes MT consecutive
@@ -69,7 +77,8 @@ struct GemmSmem {
 template <int BN, bool A_MN, int STAGES, int KBB, int MT = 1>
 __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ GemmArgs args) {
   using L = GemmSmem<BN, STAGES, KBB, MT>;
-  static_assert(STAGES * L::kStage >= BN * 128 * 4, "the pipeline stages must hold an fp32 staging tile");
+  static_assert(L::kStageCols * 128 * 4 <= STAGES * L::kStage && BN % L::kStageCols == 0,
+                "the pipeline stages hold the fp32 staging tile, whole or in column chunks");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
@@ -262,21 +271,26 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
             my[((c >> 2) + q) * 128 + row] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         }
       } else {
-        // the pipeline stages are idle now (every MMA retired): they hold the staging tile
+        // the pipeline stages are idle now (every MMA retired): they hold the
+        // staging tile, kStageCols token columns at a time
         uint8_t* stage = sA;
+        constexpr int kCh = L::kStageCols;
 #pragma unroll 1
         for (int t = 0; t < MT; ++t) {
 #pragma unroll 1
-          for (int c = 0; c < BN; c += 16) {
-            float v[16];
-            tmem_ld16(trow + t * BN + c, v);
-            tmem_wait_ld();
-            epi_stage<16>(e, nt * BN + c, args.N, v, stage, c, row);
+          for (int c0 = 0; c0 < BN; c0 += kCh) {
+#pragma unroll 1
+            for (int c = c0; c < c0 + kCh; c += 16) {
+              float v[16];
+              tmem_ld16(trow + t * BN + c, v);
+              tmem_wait_ld();
+              epi_stage<16>(e, nt * BN + c, args.N, v, stage, c - c0, row);
+            }
+            named_bar_sync(1, 128);
+            epi_flush(e, args.tok, m0 + t * 128, args.seg_rows[seg], nt * BN + c0, kCh, args.N, head, stage,
+                      threadIdx.x - 64, 128, args.status);
+            if (t + 1 < MT || c0 + kCh < BN) named_bar_sync(1, 128);  // the staging tile is refilled
           }
-          named_bar_sync(1, 128);
-          epi_flush(e, args.tok, m0 + t * 128, args.seg_rows[seg], nt * BN, BN, args.N, head, stage, threadIdx.x - 64, 128,
-                    args.status);
-          if (t + 1 < MT) named_bar_sync(1, 128);  // the staging tile is refilled
         }
       }
     }

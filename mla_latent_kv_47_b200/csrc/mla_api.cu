@@ -252,19 +252,20 @@ mla_status launch_tc_cfg(const GemmConfig& k, const GemmArgs& a, dim3 grid, cuda
   if (k.bn == BN && k.stages == S && k.kbb == KB) return launch_tc<BN, AMN, S, KB>(a, grid, st, pdl);
   MLA_GEMM_CFG(32, 5, 1) MLA_GEMM_CFG(64, 4, 1) MLA_GEMM_CFG(128, 3, 1) MLA_GEMM_CFG(256, 4, 1)
   MLA_GEMM_CFG(32, 4, 2) MLA_GEMM_CFG(64, 4, 2) MLA_GEMM_CFG(32, 2, 4) MLA_GEMM_CFG(64, 2, 4)
-  MLA_GEMM_CFG(64, 2, 2) MLA_GEMM_CFG(32, 2, 2) MLA_GEMM_CFG(128, 2, 2)
+  MLA_GEMM_CFG(64, 2, 2) MLA_GEMM_CFG(32, 2, 2) MLA_GEMM_CFG(128, 2, 2) MLA_GEMM_CFG(256, 2, 1)
 #undef MLA_GEMM_CFG
   return MLA_ERR_UNSUPPORTED;
 }
 
-// Default configuration for N tokens: weight-streaming shapes (N <= 64) take
-// two K blocks per stage and four stages (one CTA per SM), larger N the
-// 128/256-wide tiles.
+// Default configuration for N tokens: weight-streaming shapes (N <= 128)
+// take 3-5 stages of one K block, larger N 256-wide tiles with two stages, so
+// that two CTAs share an SM and one's epilogue (staged in column chunks)
+// overlaps the other's MMAs.
 GemmConfig choose_gemm_config(int N, int num_sms) {
   if (N <= 32) return {32, 5, 1, 2 * num_sms};
   if (N <= 64) return {64, 4, 1, 2 * num_sms};
   if (N <= 128) return {128, 3, 1, 2 * num_sms};
-  return {256, 4, 1, num_sms};
+  return {256, 2, 1, 2 * num_sms};
 }
 
 mla_status run_gemm_tc(const Ctx& c, const GemmSpec& g, const GemmConfig& cfg) {
@@ -1148,7 +1149,7 @@ extern "C" mla_status mla_prefill(const mla_dims* dims, const mla_weights* w, co
     static std::atomic<unsigned long long> attr_done{0};
     if ((s = set_smem_limit(attn_prefill_tc_kernel, pf::kSmem, attr_done)) != MLA_OK) return s;
     g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
-    attn_prefill_tc_kernel<<<dim3(a.n_qt, d.n_h), 192, pf::kSmem, c.st>>>(a);
+    attn_prefill_tc_kernel<<<dim3(a.n_qt, d.n_h), pf::kThreads, pf::kSmem, c.st>>>(a);
     if (cudaPeekAtLastError() != cudaSuccess) return MLA_ERR_CUDA;
   } else {
     if (d.dtype != MLA_FP32) return MLA_ERR_UNSUPPORTED;  // bf16 is on the tensor-core kernel alone

@@ -390,6 +390,16 @@ __device__ __forceinline__ void tmem_st16x2(uint32_t taddr, const uint32_t (&r)[
       : "memory");
 }
 
+// 16 lanes x 32 bit, twice, 8 columns: thread t < 16 writes lane (taddr.lane +
+// t), columns taddr.col .. +7; thread t >= 16 writes lane (taddr.lane + t -
+// 16), columns taddr.col + 8 .. +15.
+__device__ __forceinline__ void tmem_st16x2_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x8.b32 [%0], 8, {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+      "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
 // ------------------------------------------------------------------ programmatic dependent launch
 // Kernels of one call are chained with programmatic stream serialisation: a
 // kernel may start while its predecessor drains, so it must call
