@@ -11,7 +11,9 @@
 // eight warps combine the partials straight into the MMA's B operand in
 // shared memory (64 tokens x 512 latent columns, bf16, 128B swizzle, one K
 // block of 64 columns at a time so the MMAs start on the first block), while
-// the TMA brings the head's 128 x 512 block of W_UV; one thread issues
+// the TMA streams the head's 128 x 512 block of W_UV through a 3-slot ring
+// (small enough that the next GEMM's CTAs fit beside this one's and fetch
+// their weights early); one thread issues
 // M = 128 (d_h rows), N = 64 tcgen05 MMAs over the 8 K blocks, and the
 // epilogue writes o through the GEMM's per-head epilogue.  The normalised
 // latents are also written out (bf16), as the separate combine did.
@@ -43,7 +45,8 @@ constexpr int kKb = 8;                  // d_c / 64 K blocks
 constexpr int kSlabA = 128 * 128;       // 128 rows x 64 columns bf16
 constexpr int kSlabB = 64 * 128;        // 64 tokens x 64 columns bf16
 constexpr int kUnroll = 2;              // pieces whose loads are in flight together
-constexpr int kSmem = 1024 + kKb * kSlabA + kKb * kSlabB + 256;
+constexpr int kRingA = 3;               // W_UV K blocks in flight
+constexpr int kSmem = 1024 + kRingA * kSlabA + kKb * kSlabB + 256;
 static_assert(kSmem <= 232448, "shared memory budget");
 }  // namespace uvc
 
@@ -52,9 +55,10 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
-  uint8_t* sB = smem + kKb * kSlabA;
-  uint64_t* a_full = reinterpret_cast<uint64_t*>(sB + kKb * kSlabB);
-  uint64_t* b_full = a_full + kKb;
+  uint8_t* sB = smem + kRingA * kSlabA;
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(sB + kKb * kSlabB);  // [kRingA]
+  uint64_t* a_empty = a_full + kRingA;                                // [kRingA]
+  uint64_t* b_full = a_empty + kRingA;                                // [kKb]
   uint64_t* accum = b_full + kKb;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -62,10 +66,11 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
   const int head = blockIdx.x, nt = blockIdx.y;
 
   if (threadIdx.x == 0) {
-    for (int k = 0; k < kKb; ++k) {
+    for (int k = 0; k < kRingA; ++k) {
       mbar_init(&a_full[k], 1);
-      mbar_init(&b_full[k], 8);  // one arrival per combine warp
+      mbar_init(&a_empty[k], 1);
     }
+    for (int k = 0; k < kKb; ++k) mbar_init(&b_full[k], 8);  // one arrival per combine warp
     mbar_init(accum, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -86,23 +91,28 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
     // so it streams while the attention drains
     if (elect_one()) {
       const uint64_t pol = policy_evict_first();
-      for (int k = 0; k < kKb; ++k) {
-        mbar_arrive_expect_tx(&a_full[k], kSlabA);
-        tma_load_2d(sA + k * kSlabA, &a.mapA, &a_full[k], k * 64, head * 128, pol);
+      int issued = 0;
+      for (int k = 0; k < kKb; ++k, ++issued) {
+        const int r = k % kRingA;
+        if (!mbar_wait(&a_empty[r], ((k / kRingA) & 1) ^ 1, wc)) break;
+        mbar_arrive_expect_tx(&a_full[r], kSlabA);
+        tma_load_2d(sA + r * kSlabA, &a.mapA, &a_full[r], k * 64, head * 128, pol);
       }
-      drain_ring(a_full, kKb, kKb);  // every load has landed before the CTA may leave
+      drain_ring(a_full, kRingA, issued);  // every load has landed before the CTA may leave
     }
   } else if (warp == 1) {
     if (elect_one()) {
       constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);
       for (int k = 0; k < kKb; ++k) {
-        if (!mbar_wait(&a_full[k], 0, wc) || !mbar_wait(&b_full[k], 0, wc)) break;
+        const int r = k % kRingA;
+        if (!mbar_wait(&a_full[r], (k / kRingA) & 1, wc) || !mbar_wait(&b_full[k], 0, wc)) break;
         tc_fence_after();
-        const uint32_t ab = smem_u32(sA + k * kSlabA), bb = smem_u32(sB + k * kSlabB);
+        const uint32_t ab = smem_u32(sA + r * kSlabA), bb = smem_u32(sB + k * kSlabB);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ss(tmem, sdesc_sw128(ab + kk * 32, 16, 1024), sdesc_sw128(bb + kk * 32, 16, 1024), idesc,
                  (k | kk) ? 1u : 0u);
+        mma_commit(&a_empty[r]);  // the slot takes K block k + kRingA once these MMAs retired
       }
       mma_commit(accum);  // also after an abort: the epilogue then waits only for the MMAs issued
     }
