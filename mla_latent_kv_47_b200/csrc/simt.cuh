@@ -67,13 +67,40 @@ __host__ __device__ __forceinline__ long long worker_begin(int w, long long T, i
   return (static_cast<long long>(w) * T) / W;
 }
 
+// Inclusive scan of v over a 1024-thread block (shuffles within each warp,
+// then the 32 warp totals in warp 0); `total` is the block's sum.  Every
+// thread calls it; it leaves `warp_tot` free for the next call.
+__device__ __forceinline__ long long block_scan_1024(long long v, long long* warp_tot, long long& total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) warp_tot[wid] = v;
+  __syncthreads();
+  if (wid == 0) {
+    long long t = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long n = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += n;
+    }
+    warp_tot[lane] = t;
+  }
+  __syncthreads();
+  if (wid > 0) v += warp_tot[wid - 1];
+  total = warp_tot[31];
+  __syncthreads();
+  return v;
+}
+
 // Also fills the call's RoPE (cos, sin) table for the B new tokens (at
 // positions seqlen[b]) when `rope` is not null, one launch fewer per step.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seqlen, int B, int tile_tokens, int W,
                                                     int* tile_start, int* seg_start, int* status, const TokenMap tk,
                                                     float2* rope) {
-  __shared__ long long s_scan[1024];
-  __shared__ long long s_base;
+  __shared__ long long s_warp[32];
   griddep_wait();
   if (threadIdx.x == 0) griddep_launch_dependents();
   if (rope) {
@@ -85,8 +112,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seqlen, int B
     }
   }
   // pass 1: cumulative tiles
-  if (threadIdx.x == 0) s_base = 0;
-  __syncthreads();
+  long long base = 0;
   for (int b0 = 0; b0 < B; b0 += 1024) {
     const int b = b0 + threadIdx.x;
     long long v = 0;
@@ -95,26 +121,17 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seqlen, int B
       if (L < 0) atomicOr(status, FAULT_PLAN);
       v = (max(L, 0) + 1 + tile_tokens - 1) / tile_tokens;
     }
-    s_scan[threadIdx.x] = v;
-    __syncthreads();
-    for (int off = 1; off < 1024; off <<= 1) {
-      const long long add = threadIdx.x >= off ? s_scan[threadIdx.x - off] : 0;
-      __syncthreads();
-      s_scan[threadIdx.x] += add;
-      __syncthreads();
-    }
-    if (b < B) tile_start[b + 1] = static_cast<int>(s_base + s_scan[threadIdx.x]);
-    __syncthreads();
-    if (threadIdx.x == 1023) s_base += s_scan[1023];
-    __syncthreads();
+    long long total;
+    v = block_scan_1024(v, s_warp, total);
+    if (b < B) tile_start[b + 1] = static_cast<int>(base + v);
+    base += total;
   }
   if (threadIdx.x == 0) tile_start[0] = 0;
-  const long long T = s_base;
+  const long long T = base;
   const int We = static_cast<int>(T < W ? T : W);  // workers that get tiles
-  __syncthreads();
+  __syncthreads();  // tile_start written before pass 2 reads it
   // pass 2: pieces per sequence
-  if (threadIdx.x == 0) s_base = 0;
-  __syncthreads();
+  base = 0;
   for (int b0 = 0; b0 < B; b0 += 1024) {
     const int b = b0 + threadIdx.x;
     long long v = 0;
@@ -123,18 +140,10 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seqlen, int B
       const long long t1 = tile_start[b + 1];
       v = worker_of_tile(t1 - 1, T, We) - worker_of_tile(t0, T, We) + 1;
     }
-    s_scan[threadIdx.x] = v;
-    __syncthreads();
-    for (int off = 1; off < 1024; off <<= 1) {
-      const long long add = threadIdx.x >= off ? s_scan[threadIdx.x - off] : 0;
-      __syncthreads();
-      s_scan[threadIdx.x] += add;
-      __syncthreads();
-    }
-    if (b < B) seg_start[b + 1] = static_cast<int>(s_base + s_scan[threadIdx.x]);
-    __syncthreads();
-    if (threadIdx.x == 1023) s_base += s_scan[1023];
-    __syncthreads();
+    long long total;
+    v = block_scan_1024(v, s_warp, total);
+    if (b < B) seg_start[b + 1] = static_cast<int>(base + v);
+    base += total;
   }
   if (threadIdx.x == 0) seg_start[0] = 0;
 }
