@@ -8,10 +8,14 @@
 // the N operand (N = 32..256), so decode batches of 32-128 tokens still use
 // full-rate M=128 MMAs and the kernel streams the weights at HBM speed.
 // Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
-// issues tcgen05.mma, warps 2-5 run the epilogue (one TMEM lane per thread).
-// Split-K: CTAs of one output tile write fp32 partials; a second, wide kernel
-// (gemm_splitk_epilogue_kernel) sums them in split order and runs the epilogue,
-// so the reduction is spread over the whole GPU instead of one CTA per tile.
+// issues tcgen05.mma, warps 2-5 run the epilogue (one TMEM lane per thread),
+// staged in the idle pipeline buffers (in column chunks when the whole tile
+// does not fit).
+// Split-K: where the tile shape leaves room, the splits of a tile run as one
+// cluster and sum their fp32 partials through distributed shared memory;
+// otherwise they write fp32 partials and a second, wide kernel
+// (gemm_splitk_epilogue_kernel) sums them.  Either way the sum runs in split
+// order, so results do not depend on scheduling.
 #pragma once
 #include "epilogue.cuh"
 

@@ -818,14 +818,12 @@ mla_status decode_run(Ctx& c, const mla_weights* w, const void* h, int B, const 
     // ---- a6 + a7 fused: the combine feeds the absorbed W_UV product directly
     if ((s = launch_uv_combine(c, w, opart, ml, seg_start, B, olat, o, tk)) != MLA_OK) return s;
   } else {
+    // fp32 storage (bf16 is on the tensor-core kernels alone): a separate combine, then W_UV
+    if (d.dtype != MLA_FP32) return MLA_ERR_UNSUPPORTED;
     dim3 grid(B, (d.n_h + 3) / 4);  // one warp per (sequence, head)
-    if (d.dtype == MLA_FP32)
-      s = launch(combine_kernel<float>, grid, dim3(128), 0, c.st, c.pdl, opart, ml, seg_start, d.n_h, d.d_c,
-                 static_cast<float*>(olat));
-    else
-      s = launch(combine_kernel<__nv_bfloat16>, grid, dim3(128), 0, c.st, c.pdl, opart, ml, seg_start, d.n_h, d.d_c,
-                 static_cast<__nv_bfloat16*>(olat));
-    if (s != MLA_OK) return s;
+    if ((s = launch(combine_kernel<float>, grid, dim3(128), 0, c.st, c.pdl, opart, ml, seg_start, d.n_h, d.d_c,
+                    static_cast<float*>(olat))) != MLA_OK)
+      return s;
     // ---- a7: absorbed W_UV on the latent output: o_i = W_UV_i o_lat_i
     GemmSpec g;
     g.mode = GEMM_HEAD_KMAJOR;
