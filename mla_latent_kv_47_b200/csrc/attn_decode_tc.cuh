@@ -32,20 +32,20 @@
 // rescaled.  The kernel's range is P <= 2^96 (ample for fp32 O and l); a
 // tile whose scores rise past it sets FAULT_RANGE.
 //
-// Warp roles (448 threads per CTA; 576 for E4M3 rows):
+// Warp roles (448 threads per CTA; 704 for E4M3 rows):
 //   warp 0      TMA producer (bf16 rows: the three rings below; E4M3 rows:
 //               raw stages and bf16 stages)
 //   warp 1      TMEM owner and MMA issuer: S(j) once tile j landed and the S
 //               buffer was read out, PV(j) once both halves of P(j) are in place
 //   warps 2-5   Q_lat of each piece: chunks 0-6 (bf16 pairs) into TMEM, chunks
 //               7-8 into shared memory, both MMA A operands; for E4M3 rows
-//               also half of the decode of each raw stage into a bf16 stage
+//               also a third of the decode of each raw stage into a bf16 stage
 //   warps 6-13  softmax: warp 6+i and warp 10+i share lane quarter i mod 4,
 //               16 heads each; two threads per head (rows 0-15 and 16-31 of
 //               this CTA's half, via the 16-lane TMEM access shape).  Softmax
 //               against the piece's reference max (above), and the per-piece
 //               epilogue; CTA 1 sends its share of l to CTA 0.
-//   warps 14-17 E4M3 rows only: the other half of the decode
+//   warps 14-21 E4M3 rows only: the other two thirds of the decode
 #pragma once
 #include "mla.h"
 #include "ptx.cuh"
@@ -115,10 +115,10 @@ struct Cfg {
   // P buffers: P(g) is written once PV(g - kPBufs) retired in both CTAs
   static constexpr int kPBufs = 2;
   // E4M3 rows: the decode, bound by its latency rather than its arithmetic,
-  // is split over eight warps, the four Q warps and four more (warps 14-17)
-  // that do nothing else
-  static constexpr int kConvWarps = kFp8 ? 8 : 0;
-  static constexpr int kThreads = kFp8 ? 576 : 448;
+  // is split over twelve warps, the four Q warps and eight more (warps
+  // 14-21) that do nothing else
+  static constexpr int kConvWarps = kFp8 ? 12 : 0;
+  static constexpr int kThreads = kFp8 ? 704 : 448;
   // stages (rings) | raw stages | Q chunks 7-8 | P x 2 | aux
   static constexpr int kSmem = 1024 + kStageRegion + kRawStages * kRawBytes + kQSmemChunks * kQChunkBytes +
                                kPBufs * kPBytes + kAuxBytes;
