@@ -40,7 +40,13 @@ struct UvCombineArgs {
 };
 
 namespace uvc {
-constexpr int kThreads = 320;
+constexpr int kCombWarps = 16;          // warps that combine (warps 2 .. 2 + kCombWarps - 1)
+constexpr int kThreads = 64 + 32 * kCombWarps;
+constexpr int kTPR = kCombWarps * 32 / 64;  // combine threads per token
+constexpr int kCPT = 64 / kTPR;             // columns of a K block per thread
+constexpr int kF4 = kCPT / 4;               // float4 loads of a K block per thread and piece
+constexpr int kKbPass = 4;                  // K blocks per pass: kKbPass * kF4 loads of each piece in flight
+static_assert(kCPT % 8 == 0 && 8 % kKbPass == 0, "combine thread mapping");
 constexpr int kKb = 8;                  // d_c / 64 K blocks
 constexpr int kSlabA = 128 * 128;       // 128 rows x 64 columns bf16
 constexpr int kSlabB = 64 * 128;        // 64 tokens x 64 columns bf16
@@ -70,7 +76,7 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
       mbar_init(&a_full[k], 1);
       mbar_init(&a_empty[k], 1);
     }
-    for (int k = 0; k < kKb; ++k) mbar_init(&b_full[k], 8);  // one arrival per combine warp
+    for (int k = 0; k < kKb; ++k) mbar_init(&b_full[k], kCombWarps);  // one arrival per combine warp
     mbar_init(accum, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -117,11 +123,11 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
       mma_commit(accum);  // also after an abort: the epilogue then waits only for the MMAs issued
     }
   } else {
-    // ---- combine: thread t takes token nl = t / 4 of the tile and the 16
-    // columns [16 q, 16 q + 16) of every 64-column K block (q = t % 4)
+    // ---- combine: thread t takes token nl = t / kTPR of the tile and the
+    // kCPT columns [kCPT q, kCPT q + kCPT) of every 64-column K block (q = t % kTPR)
     griddep_wait();  // the partials come from the attention kernel
     const int t = threadIdx.x - 64;
-    const int nl = t >> 2, q = t & 3;
+    const int nl = t / kTPR, q = t % kTPR;
     const int n = nt * 64 + nl;
     int s0 = 0, s1 = 0;
     float M = -INFINITY, inv = 0.f;
@@ -137,15 +143,15 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
       inv = 1.f / Ls;
     }
     __nv_bfloat16* orow = a.olat + (static_cast<long long>(n) * a.n_h + head) * 512;
-    for (int k = 0; k < kKb; k += 2) {  // two K blocks per pass: 8 float4 loads of each piece in flight
-      float4 acc[2][4];
+    for (int k = 0; k < kKb; k += kKbPass) {
+      float4 acc[kKbPass][kF4];
 #pragma unroll
-      for (int j = 0; j < 2; ++j)
+      for (int j = 0; j < kKbPass; ++j)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[j][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < kF4; ++i) acc[j][i] = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int sb = s0; sb < s1; sb += kUnroll) {
         float wgt[kUnroll];
-        float4 v[kUnroll][2][4];
+        float4 v[kUnroll][kKbPass][kF4];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
           const bool on = sb + u < s1;
@@ -153,17 +159,17 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
           const float4* src =
               reinterpret_cast<const float4*>(a.o_part + (static_cast<long long>(sb + u) * a.n_h + head) * 512);
 #pragma unroll
-          for (int j = 0; j < 2; ++j)
+          for (int j = 0; j < kKbPass; ++j)
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              v[u][j][i] = on ? __ldcs(src + ((k + j) * 64 + 16 * q) / 4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int i = 0; i < kF4; ++i)
+              v[u][j][i] = on ? __ldcs(src + ((k + j) * 64 + kCPT * q) / 4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u)
 #pragma unroll
-          for (int j = 0; j < 2; ++j)
+          for (int j = 0; j < kKbPass; ++j)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < kF4; ++i) {
               acc[j][i].x += wgt[u] * v[u][j][i].x;
               acc[j][i].y += wgt[u] * v[u][j][i].y;
               acc[j][i].z += wgt[u] * v[u][j][i].z;
@@ -171,32 +177,31 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
             }
       }
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        uint32_t pk[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[j][i].x * inv, acc[j][i].y * inv);
-          const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[j][i].z * inv, acc[j][i].w * inv);
-          pk[2 * i] = *reinterpret_cast<const uint32_t*>(&lo);
-          pk[2 * i + 1] = *reinterpret_cast<const uint32_t*>(&hi);
-        }
-        const uint4 p0 = make_uint4(pk[0], pk[1], pk[2], pk[3]), p1 = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        // row nl of K block k + j: 16-byte pieces 2q and 2q + 1, swizzled by the row
+      for (int j = 0; j < kKbPass; ++j) {
+        // row nl of K block k + j: the kCPT / 8 16-byte pieces from kCPT q / 8 on, swizzled by the row
         uint8_t* row = sB + (k + j) * kSlabB + nl * 128;
-        *reinterpret_cast<uint4*>(row + (((2 * q) ^ (nl & 7)) << 4)) = p0;
-        *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ (nl & 7)) << 4)) = p1;
-        if (n < a.N) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + (k + j) * 64 + 16 * q);
-          dst[0] = p0;
-          dst[1] = p1;
+        uint4* dst = reinterpret_cast<uint4*>(orow + (k + j) * 64 + kCPT * q);
+#pragma unroll
+        for (int pc = 0; pc < kCPT / 8; ++pc) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const float4 f = acc[j][2 * pc + i];
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(f.x * inv, f.y * inv);
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(f.z * inv, f.w * inv);
+            pk[2 * i] = *reinterpret_cast<const uint32_t*>(&lo);
+            pk[2 * i + 1] = *reinterpret_cast<const uint32_t*>(&hi);
+          }
+          const uint4 pv = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(row + (((kCPT / 8 * q + pc) ^ (nl & 7)) << 4)) = pv;
+          if (n < a.N) dst[pc] = pv;
         }
       }
       fence_proxy_async_smem();  // the MMAs read the tile through the async proxy
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&b_full[k]);
-        mbar_arrive(&b_full[k + 1]);
-      }
+      if (lane == 0)
+#pragma unroll
+        for (int j = 0; j < kKbPass; ++j) mbar_arrive(&b_full[k + j]);
     }
     if (warp < 6) {
       // ---- epilogue: warps 2..5, thread <-> TMEM lane (row m of W_UV_i)
