@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "attn_decode_sh.cuh"
 #include "attn_decode_tc.cuh"
 #include "attn_prefill_tc.cuh"
 #include "gemm_tc.cuh"
@@ -620,6 +621,12 @@ mla_status launch_attn_kernel(const AttnArgs& a, int W, cudaStream_t st, bool pd
                 pdl, a);
 }
 
+bool attn_tc_ok(const mla_dims& d);
+
+// Few heads (V2-Lite's 16) on bf16 rows take the single-CTA kernel with the
+// tokens as the MMA's M dimension.
+bool attn_sh_ok(const mla_dims& d) { return attn_tc_ok(d) && d.n_h <= attn_sh::kNH && !cache_fp8(d); }
+
 mla_status launch_attn_decode_tc(const mla_dims& d, const __nv_bfloat16* qlat, const mla_cache* cache,
                                  const int32_t* seqlen, const int* tile_start, const int* seg_start, int B, int W,
                                  int n_h, float* o_part, float* ml, int* status, cudaStream_t st, bool pdl) {
@@ -649,7 +656,15 @@ mla_status launch_attn_decode_tc(const mla_dims& d, const __nv_bfloat16* qlat, c
   a.o_part = o_part;
   a.ml_part = ml;
   a.status = status;
-  return fp8 ? launch_attn_kernel<true>(a, W, st, pdl) : launch_attn_kernel<false>(a, W, st, pdl);
+  if (fp8) return launch_attn_kernel<true>(a, W, st, pdl);
+  if (attn_sh_ok(d)) {
+    // few heads: one CTA per worker, tokens as the MMA's M
+    static std::atomic<unsigned long long> attr_done{0};
+    const mla_status s = set_smem_limit(attn_decode_sh_kernel, attn_sh::kSmem, attr_done);
+    if (s != MLA_OK) return s;
+    return launch(attn_decode_sh_kernel, dim3(W), dim3(attn_sh::kThreads), attn_sh::kSmem, st, pdl, a);
+  }
+  return launch_attn_kernel<false>(a, W, st, pdl);
 }
 
 bool prefill_tc_ok(const mla_dims& d) {
@@ -660,10 +675,13 @@ bool attn_tc_ok(const mla_dims& d) {
   return kAttnTcReady && d.dtype == MLA_BF16 && d.n_h <= 128 && d.d_c == 512 && d.d_R == 64;
 }
 
-// Attention workers of a decode call: one 2-CTA cluster per SM pair on the
-// tensor-core path, two CTAs per SM on the CUDA-core path.
+// Attention workers of a decode call: one CTA per SM on the few-head kernel,
+// one 2-CTA cluster per SM pair on the other tensor-core path, two CTAs per SM
+// on the CUDA-core path.
 int decode_workers(const mla_dims& d, int num_sms) {
-  const int W = attn_tc_ok(d) ? std::min(kMaxWorkers, num_sms / 2) : std::min(kMaxWorkers, num_sms * 2);
+  const int W = attn_sh_ok(d)   ? std::min(kMaxWorkers, num_sms)
+                : attn_tc_ok(d) ? std::min(kMaxWorkers, num_sms / 2)
+                                : std::min(kMaxWorkers, num_sms * 2);
   return W < 1 ? 1 : W;
 }
 
