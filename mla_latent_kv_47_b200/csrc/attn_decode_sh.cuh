@@ -21,9 +21,14 @@
 // and l are never rescaled, and P is capped at 2^96 (FAULT_RANGE past it).
 //
 // Warp roles (192 threads): warp 0 TMA producer (2 stages of 64 tokens x 576
-// columns), warp 1 TMEM owner and MMA issuer, warps 2-5 Q of each piece, the
-// softmax (warp q takes tokens 16 q .. 16 q + 15 of a tile, two threads per
-// token, 8 heads each) and the per-piece epilogue.
+// columns), warp 1 TMEM owner and MMA issuer, warps 2-5 Q, the softmax (warp
+// q takes tokens 16 q .. 16 q + 15 of a tile, two threads per token, 8 heads
+// each) and the per-piece epilogue.  Q has two buffers: the next piece's Q is
+// loaded as soon as the current piece's last P is written, so the next
+// piece's score MMAs run during the epilogue, and the epilogue writes (m, l)
+// before it waits for the last PV product.  A tile's 36 score MMAs are issued
+// back to back once its whole stage has landed: issuing them a chunk at a
+// time as the chunks land measured slower.
 #pragma once
 #include "attn_decode_tc.cuh"
 
@@ -43,7 +48,7 @@ constexpr int kAuxBytes = 2048;
 constexpr uint32_t kTmemS = 0, kTmemO = 32, kTmemCols = 128;
 constexpr float kRangeLog2 = 96.f;
 constexpr int kRow = 576;
-constexpr int kSmem = 1024 + kStages * kStageBytes + kQBytes + 2 * kPBytes + kAuxBytes;
+constexpr int kSmem = 1024 + kStages * kStageBytes + 2 * kQBytes + 2 * kPBytes + kAuxBytes;
 static_assert(kSmem <= 232448, "shared memory budget");
 static_assert(kQChunk % 1024 == 0 && kPBytes % 1024 == 0, "1024-byte alignment of the swizzled tiles");
 }  // namespace attn_sh
@@ -62,8 +67,8 @@ __global__ void __launch_bounds__(attn_sh::kThreads, 1) attn_decode_sh_kernel(co
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* stages = smem;
-  uint8_t* qs = stages + kStages * kStageBytes;  // Q: 9 chunks of 16 heads x 64 columns (MMA B operand)
-  uint8_t* pbuf = qs + kQBytes;                  // [2] P^T (MMA B operand)
+  uint8_t* qs = stages + kStages * kStageBytes;  // [2] Q: 9 chunks of 16 heads x 64 columns (MMA B operand)
+  uint8_t* pbuf = qs + 2 * kQBytes;              // [2] P^T (MMA B operand)
   uint8_t* aux = pbuf + 2 * kPBytes;
   float* mxs = reinterpret_cast<float*>(aux);    // [2 pieces][4 warps][16 heads] maxima of the first tile
   float* lxs = mxs + 2 * 4 * kNH;                // [4 warps][16 heads] l of the piece
@@ -73,15 +78,15 @@ __global__ void __launch_bounds__(attn_sh::kThreads, 1) attn_decode_sh_kernel(co
   uint64_t* s_free = s_full + 2;        // [2] S^T(j) read out
   uint64_t* p_full = s_free + 2;        // [2] P^T(j) written (buffer j % 2)
   uint64_t* p_free = p_full + 2;        // [2] PV(j) retired
-  uint64_t* q_full = p_free + 2;
-  uint64_t* q_free = q_full + 1;        // last S of the piece retired
-  uint64_t* o_done = q_free + 1;
+  uint64_t* q_full = p_free + 2;        // [2] Q of piece j in buffer j % 2
+  uint64_t* q_free = q_full + 2;        // [2] last S of piece j retired
+  uint64_t* o_done = q_free + 2;
   uint64_t* drain = o_done + 1;
   uint64_t* mx_bar = drain + 1;         // [2] the four warps' maxima of piece j in mxs (buffer j % 2)
   uint64_t* l_bar = mx_bar + 2;         // the four warps' l of the piece in lxs
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(l_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  static_assert(1024 + (2 * kStages + 15) * 8 + 8 <= kAuxBytes, "aux layout");
+  static_assert(1024 + (2 * kStages + 17) * 8 + 8 <= kAuxBytes, "aux layout");
   static_assert((2 * 4 * kNH + 4 * kNH) * 4 <= 1024, "aux layout: maxima and l");
 
   const int w = blockIdx.x;
@@ -98,9 +103,9 @@ __global__ void __launch_bounds__(attn_sh::kThreads, 1) attn_decode_sh_kernel(co
       mbar_init(&p_full[i], 4);
       mbar_init(&p_free[i], 1);
       mbar_init(&mx_bar[i], 4);
+      mbar_init(&q_full[i], 4);
+      mbar_init(&q_free[i], 1);
     }
-    mbar_init(q_full, 4);
-    mbar_init(q_free, 1);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
     mbar_init(l_bar, 4);
@@ -153,13 +158,13 @@ __global__ void __launch_bounds__(attn_sh::kThreads, 1) attn_decode_sh_kernel(co
       int it = 0, piece = 0;
       for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
         if (*abort_flag) return;
-        if (!mbar_wait(q_full, piece & 1, wc)) return;
+        if (!mbar_wait(&q_full[piece & 1], (piece >> 1) & 1, wc)) return;
         tc_fence_after();
         const int nt = p.t1 - p.t0;
         int ns = 0, npv = 0;
         uint32_t spins = 0;
         uint64_t t_idle = 0;
-        const uint32_t qb = smem_u32(qs);
+        const uint32_t qb = smem_u32(qs + (piece & 1) * kQBytes);
         while (npv < nt) {
           bool issued = false;
           if (npv < ns) {  // O^T += C^T P^T(g)
@@ -196,7 +201,7 @@ __global__ void __launch_bounds__(attn_sh::kThreads, 1) attn_decode_sh_kernel(co
                          sdesc_sw128(qb + c * kQChunk + kk * 32, 16, 1024), idesc_s, (c | kk) ? 1u : 0u);
               }
               mma_commit(&s_full[b]);
-              if (ns == nt - 1) mma_commit(q_free);  // no MMA of this piece reads Q any more
+              if (ns == nt - 1) mma_commit(&q_free[piece & 1]);  // no MMA of this piece reads its Q any more
               ++ns;
               issued = true;
             }
@@ -227,23 +232,38 @@ __global__ void __launch_bounds__(attn_sh::kThreads, 1) attn_decode_sh_kernel(co
     const int tl16 = lane & 15, hg = lane >> 4;  // token within the quarter, head group (heads 8 hg .. +7)
     const uint32_t tq = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int tid = threadIdx.x - 64;         // 0 .. 127
+    // Q of sequence b into buffer j: the B-operand chunks (16 heads x 576
+    // columns, 128B swizzle), heads past n_h zero
+    auto load_q = [&](int b, int j) {
+      const __nv_bfloat16* qb = a.qlat + static_cast<long long>(b) * a.n_h * kRow;
+      uint4 v[kNH * 72 / 128];
+#pragma unroll
+      for (int r = 0; r < kNH * 72 / 128; ++r) {  // 72 pieces of 16 bytes per head row
+        const int i = tid + 128 * r, h = i / 72, pc = i % 72;
+        v[r] = h < a.n_h ? *reinterpret_cast<const uint4*>(qb + h * kRow + pc * 8) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int r = 0; r < kNH * 72 / 128; ++r) {
+        const int i = tid + 128 * r, h = i / 72, pc = i % 72, c = pc >> 3, u = pc & 7;
+        st_shared_v4(smem_u32(qs + j * kQBytes) + c * kQChunk + h * 128 + ((u ^ (h & 7)) << 4), v[r]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&q_full[j]);
+    };
+    static_assert(kNH * 72 % 128 == 0, "Q pieces per thread");
+    // the worker's last tile: pieces after the current one are the next
+    // sequences while their tiles start before it
+    long long r1 = 0;
+    {
+      const long long T = a.tile_start[a.B];
+      const int We = static_cast<int>(T < a.W ? T : a.W);
+      if (T > 0 && w < We) r1 = worker_begin(w + 1, T, We);
+    }
     int it = 0, piece = 0;
     for_each_piece(w, a.W, a.B, a.tile_start, a.seg_start, [&](const Piece& p) {
       if (*abort_flag) return;
-      // ---- Q of the piece's sequence into the B-operand chunks (16 heads x
-      // 576 columns, 128B swizzle); the previous piece's S products retired
-      if (piece > 0 && !mbar_wait(q_free, (piece - 1) & 1, wc)) return;
-      {
-        const __nv_bfloat16* qb = a.qlat + static_cast<long long>(p.b) * a.n_h * kRow;
-        for (int i = tid; i < kNH * 72; i += 128) {  // 72 pieces of 16 bytes per head row
-          const int h = i / 72, pc = i % 72, c = pc >> 3, u = pc & 7;
-          const uint4 v = h < a.n_h ? *reinterpret_cast<const uint4*>(qb + h * kRow + pc * 8) : make_uint4(0, 0, 0, 0);
-          st_shared_v4(smem_u32(qs) + c * kQChunk + h * 128 + ((u ^ (h & 7)) << 4), v);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(q_full);
-      }
+      if (piece == 0) load_q(p.b, 0);  // later pieces' Q is loaded ahead, below
       const int L1 = a.seqlen[p.b] + 1;
       float m[8], l[8];
 #pragma unroll
@@ -335,20 +355,14 @@ __global__ void __launch_bounds__(attn_sh::kThreads, 1) attn_decode_sh_kernel(co
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[b]);
       }
-      // ---- epilogue of the piece: O^T (latent rows in TMEM lanes) to o_part,
-      // and (m, l) per head to ml_part
-      if (!mbar_wait(o_done, piece & 1, wc)) return;
-      tc_fence_after();
-#pragma unroll 1
-      for (int mt = 0; mt < 4; ++mt) {
-        float o[16];
-        tmem_ld16(tq + kTmemO + mt * kNH, o);  // latent 128 mt + 32 q4 + lane, heads 0..15
-        tmem_wait_ld();
-        const int lat = 128 * mt + 32 * q4 + lane;
-#pragma unroll
-        for (int h = 0; h < kNH; ++h)
-          if (h < a.n_h) a.o_part[(static_cast<long long>(p.slot) * a.n_h + h) * 512 + lat] = o[h];
+      // ---- the next piece's Q into the other buffer, so that its S products
+      // run during this piece's epilogue (the buffer's piece - 1 S retired)
+      if (p.b + 1 < a.B && a.tile_start[p.b + 1] < r1) {
+        if (piece > 0 && !mbar_wait(&q_free[(piece + 1) & 1], ((piece - 1) >> 1) & 1, wc)) return;
+        load_q(p.b + 1, (piece + 1) & 1);
       }
+      // ---- epilogue of the piece: (m, l) per head to ml_part while the last
+      // PV product runs, then O^T (latent rows in TMEM lanes) to o_part.
       // l per head: over the 16 tokens of each half warp, then the four warps
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -369,6 +383,20 @@ __global__ void __launch_bounds__(attn_sh::kThreads, 1) attn_decode_sh_kernel(co
         const float lh = ((lxs[lane] + lxs[kNH + lane]) + lxs[2 * kNH + lane]) + lxs[3 * kNH + lane];
         a.ml_part[(static_cast<long long>(p.slot) * a.n_h + lane) * 2] = mh;
         a.ml_part[(static_cast<long long>(p.slot) * a.n_h + lane) * 2 + 1] = lh;
+      }
+      if (!mbar_wait(o_done, piece & 1, wc)) return;
+      tc_fence_after();
+      {
+        float o[4][16];
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) tmem_ld16(tq + kTmemO + mt * kNH, o[mt]);  // latent 128 mt + 32 q4 + lane
+        tmem_wait_ld();
+        float* op = a.o_part + static_cast<long long>(p.slot) * a.n_h * 512 + 32 * q4 + lane;
+#pragma unroll
+        for (int h = 0; h < kNH; ++h)
+          if (h < a.n_h)
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt) op[h * 512 + 128 * mt] = o[mt][h];
       }
       tc_fence_before();
       it += nt;
