@@ -190,6 +190,29 @@ mla_status launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// launch() with clusters of cz CTAs along grid z (gridDim.z == cz).
+template <typename... KArgs, typename... Args>
+mla_status launch_cluster_z(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                            int cz, Args... args) {
+  if (cz <= 1) return launch(kern, grid, block, smem, st, pdl, args...);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = cz;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 constexpr int kMaxDevices = 64;
 
 // Raises a kernel's dynamic shared-memory limit on the current device.  The
@@ -413,8 +436,11 @@ mla_status run_gemm(const Ctx& c, const GemmSpec& g) {
   if (tc_gemm_ok(c.d)) {
     GemmConfig cfg = choose_gemm_config(g.N, c.num_sms);
     // per-head weight blocks of several 128-row tiles (W_UK^T: d_c rows per head)
-    // share one X block: a CTA per head streams them all, one accumulator each
-    if (g.mode != GEMM_DENSE && g.N <= 64 && g.rows[0] % 512 == 0) cfg = {64, 2, 1, c.num_sms, 2};
+    // share one X block: where the tiles fill the SMs twice over (V2's 128
+    // heads), a CTA takes two of them, one accumulator each; fewer tiles
+    // (V2-Lite's 16 heads) keep one per CTA, which measured 2 us faster there
+    if (g.mode != GEMM_DENSE && g.N <= 64 && g.rows[0] % 512 == 0 && g.heads * (g.rows[0] / 128) >= 2 * c.num_sms)
+      cfg = {64, 2, 1, c.num_sms, 2};
     return run_gemm_tc(c, g, cfg);
   }
   // fp32 storage (check_dims admits bf16 only with tensor-core shapes)
@@ -699,6 +725,11 @@ mla_status launch_uv_combine(const Ctx& c, const mla_weights* w, const float* op
   a.seg_start = seg_start;
   a.n_h = d.n_h;
   a.N = B;
+  // K splits: while the (head, 64-sequence) tiles would fill under half the
+  // SMs, split each tile's 8 K blocks over a cluster of up to 4 (V2-Lite: 16 heads)
+  const int tiles = d.n_h * ((B + 63) / 64);
+  a.ks = 1;
+  while (a.ks < uvc::kMaxKs && 2 * tiles * a.ks <= c.num_sms) a.ks *= 2;
   a.olat = static_cast<__nv_bfloat16*>(olat);
   a.epi = epi_kind(EPI_PER_HEAD, o, HD, d.d_h, 0, 0, 1.f);
   a.tok = tk;
@@ -706,7 +737,8 @@ mla_status launch_uv_combine(const Ctx& c, const mla_weights* w, const float* op
   static std::atomic<unsigned long long> attr_done{0};
   const mla_status s = set_smem_limit(uv_combine_kernel, uvc::kSmem, attr_done);
   if (s != MLA_OK) return s;
-  return launch(uv_combine_kernel, dim3(d.n_h, (B + 63) / 64), dim3(uvc::kThreads), uvc::kSmem, c.st, c.pdl, a);
+  return launch_cluster_z(uv_combine_kernel, dim3(d.n_h, (B + 63) / 64, a.ks), dim3(uvc::kThreads), uvc::kSmem, c.st,
+                          c.pdl, a.ks, a);
 }
 
 // The decode launch sequence (a1 .. a8 of the hot path) on an already checked

@@ -8,7 +8,7 @@
 //
 // over the pieces s of sequence b, from the attention kernel's unnormalised
 // partials O_s (fp32) and (m_s, l_s).  One CTA per (head i, 64 sequences):
-// eight warps combine the partials straight into the MMA's B operand in
+// sixteen warps combine the partials straight into the MMA's B operand in
 // shared memory (64 tokens x 512 latent columns, bf16, 128B swizzle, one K
 // block of 64 columns at a time so the MMAs start on the first block), while
 // the TMA streams the head's 128 x 512 block of W_UV through a 3-slot ring
@@ -18,11 +18,23 @@
 // epilogue writes o through the GEMM's per-head epilogue.  The normalised
 // latents are also written out (bf16), as the separate combine did.
 //
-// The arithmetic is the two-kernel path's: the same weights, the same
-// accumulation order over the pieces, the same rounding to bf16, the same
-// MMA order over K.  Warp roles (320 threads): warp 0 TMA, warp 1 TMEM owner
-// and MMA issuer, warps 2-9 combine, warps 2-5 then the epilogue.
+// The combine's arithmetic is the two-kernel path's: the same weights, the
+// same accumulation order over the pieces, the same rounding to bf16.  Warp
+// roles: warp 0 TMA, warp 1 TMEM owner and MMA issuer, warps 2 .. 17 combine,
+// warps 2-5 then the epilogue.
+//
+// Few (head, 64-sequence) tiles (V2-Lite's 16 heads at B <= 64 make 16 CTAs
+// on 148 SMs) split the 8 K blocks over a cluster of ks <= 4 CTAs along grid z:
+// CTA z combines and multiplies K blocks [8 z / ks, 8 (z + 1) / ks) only,
+// stages its fp32 partial tile in the idle W_UV ring, and after a cluster
+// barrier sums rows [128 z / ks, 128 (z + 1) / ks) of the tile over the ks
+// partials, in split order, through distributed shared memory before its
+// epilogue on those rows.  At V2-Lite B = 32, four splits took a decode step
+// from 84.0 to 79.5 us; eight (one K block per CTA) took it to 86.3 us, the
+// cluster barriers and the reduction then costing more than the combine saves.
 #pragma once
+#include <type_traits>
+
 #include "epilogue.cuh"
 
 namespace mla {
@@ -33,6 +45,7 @@ struct UvCombineArgs {
   const float* ml_part;  // [slots][n_h][2] (m, l) of each partial
   const int* seg_start;  // [N + 1] first slot of each sequence
   int n_h, N;            // heads, sequences (tokens)
+  int ks;                // K splits per tile: the cluster size along grid z (1, 2 or 4)
   __nv_bfloat16* olat;   // [N][n_h][512] the normalised latent outputs
   Epi epi;               // EPI_PER_HEAD into o [N][n_h d_h]
   TokenMap tok;
@@ -52,8 +65,10 @@ constexpr int kSlabA = 128 * 128;       // 128 rows x 64 columns bf16
 constexpr int kSlabB = 64 * 128;        // 64 tokens x 64 columns bf16
 constexpr int kUnroll = 2;              // pieces whose loads are in flight together
 constexpr int kRingA = 3;               // W_UV K blocks in flight
+constexpr int kMaxKs = 4;               // K splits of a tile: two K blocks per CTA at most
 constexpr int kSmem = 1024 + kRingA * kSlabA + kKb * kSlabB + 256;
 static_assert(kSmem <= 232448, "shared memory budget");
+static_assert(kRingA * kSlabA >= 128 * 64 * 4, "the W_UV ring holds a partial tile");
 }  // namespace uvc
 
 __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __grid_constant__ UvCombineArgs a) {
@@ -70,13 +85,14 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int head = blockIdx.x, nt = blockIdx.y;
+  const int ks = a.ks, nkb = kKb / ks, kb0 = static_cast<int>(blockIdx.z) * nkb, kb1 = kb0 + nkb;  // this CTA's K blocks
 
   if (threadIdx.x == 0) {
     for (int k = 0; k < kRingA; ++k) {
       mbar_init(&a_full[k], 1);
       mbar_init(&a_empty[k], 1);
     }
-    for (int k = 0; k < kKb; ++k) mbar_init(&b_full[k], kCombWarps);  // one arrival per combine warp
+    for (int k = 0; k < kKb; ++k) mbar_init(&b_full[k], kCombWarps);  // one arrival per combine warp (own blocks)
     mbar_init(accum, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -98,22 +114,22 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
     if (elect_one()) {
       const uint64_t pol = policy_evict_first();
       int issued = 0;
-      for (int k = 0; k < kKb; ++k, ++issued) {
+      for (int k = 0; k < nkb; ++k, ++issued) {
         const int r = k % kRingA;
         if (!mbar_wait(&a_empty[r], ((k / kRingA) & 1) ^ 1, wc)) break;
         mbar_arrive_expect_tx(&a_full[r], kSlabA);
-        tma_load_2d(sA + r * kSlabA, &a.mapA, &a_full[r], k * 64, head * 128, pol);
+        tma_load_2d(sA + r * kSlabA, &a.mapA, &a_full[r], (kb0 + k) * 64, head * 128, pol);
       }
       drain_ring(a_full, kRingA, issued);  // every load has landed before the CTA may leave
     }
   } else if (warp == 1) {
     if (elect_one()) {
       constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);
-      for (int k = 0; k < kKb; ++k) {
+      for (int k = 0; k < nkb; ++k) {
         const int r = k % kRingA;
-        if (!mbar_wait(&a_full[r], (k / kRingA) & 1, wc) || !mbar_wait(&b_full[k], 0, wc)) break;
+        if (!mbar_wait(&a_full[r], (k / kRingA) & 1, wc) || !mbar_wait(&b_full[kb0 + k], 0, wc)) break;
         tc_fence_after();
-        const uint32_t ab = smem_u32(sA + r * kSlabA), bb = smem_u32(sB + k * kSlabB);
+        const uint32_t ab = smem_u32(sA + r * kSlabA), bb = smem_u32(sB + (kb0 + k) * kSlabB);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ss(tmem, sdesc_sw128(ab + kk * 32, 16, 1024), sdesc_sw128(bb + kk * 32, 16, 1024), idesc,
@@ -143,15 +159,16 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
       inv = 1.f / Ls;
     }
     __nv_bfloat16* orow = a.olat + (static_cast<long long>(n) * a.n_h + head) * 512;
-    for (int k = 0; k < kKb; k += kKbPass) {
-      float4 acc[kKbPass][kF4];
+    auto pass = [&](auto nj, int k) {
+      constexpr int NJ = decltype(nj)::value;
+      float4 acc[NJ][kF4];
 #pragma unroll
-      for (int j = 0; j < kKbPass; ++j)
+      for (int j = 0; j < NJ; ++j)
 #pragma unroll
         for (int i = 0; i < kF4; ++i) acc[j][i] = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int sb = s0; sb < s1; sb += kUnroll) {
         float wgt[kUnroll];
-        float4 v[kUnroll][kKbPass][kF4];
+        float4 v[kUnroll][NJ][kF4];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
           const bool on = sb + u < s1;
@@ -159,7 +176,7 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
           const float4* src =
               reinterpret_cast<const float4*>(a.o_part + (static_cast<long long>(sb + u) * a.n_h + head) * 512);
 #pragma unroll
-          for (int j = 0; j < kKbPass; ++j)
+          for (int j = 0; j < NJ; ++j)
 #pragma unroll
             for (int i = 0; i < kF4; ++i)
               v[u][j][i] = on ? __ldcs(src + ((k + j) * 64 + kCPT * q) / 4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -167,7 +184,7 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u)
 #pragma unroll
-          for (int j = 0; j < kKbPass; ++j)
+          for (int j = 0; j < NJ; ++j)
 #pragma unroll
             for (int i = 0; i < kF4; ++i) {
               acc[j][i].x += wgt[u] * v[u][j][i].x;
@@ -177,7 +194,7 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
             }
       }
 #pragma unroll
-      for (int j = 0; j < kKbPass; ++j) {
+      for (int j = 0; j < NJ; ++j) {
         // row nl of K block k + j: the kCPT / 8 16-byte pieces from kCPT q / 8 on, swizzled by the row
         uint8_t* row = sB + (k + j) * kSlabB + nl * 128;
         uint4* dst = reinterpret_cast<uint4*>(orow + (k + j) * 64 + kCPT * q);
@@ -201,7 +218,14 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
       __syncwarp();
       if (lane == 0)
 #pragma unroll
-        for (int j = 0; j < kKbPass; ++j) mbar_arrive(&b_full[k + j]);
+        for (int j = 0; j < NJ; ++j) mbar_arrive(&b_full[k + j]);
+    };
+    // K blocks [kb0, kb1) in passes of kKbPass blocks, or one pass of two
+    static_assert(kKbPass == 4 && kKb / kMaxKs == 2, "passes of the K splits");
+    if (nkb >= kKbPass) {
+      for (int k = kb0; k < kb1; k += kKbPass) pass(std::integral_constant<int, kKbPass>{}, k);
+    } else {
+      pass(std::integral_constant<int, 2>{}, kb0);
     }
     if (warp < 6) {
       // ---- epilogue: warps 2..5, thread <-> TMEM lane (row m of W_UV_i)
@@ -211,7 +235,20 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
       mbar_wait(accum, 0, wc);
       tc_fence_after();
       named_bar_sync(1, 128);  // every epilogue thread sees the same abort decision
-      if (!*abort_flag) {
+      if (!*abort_flag && ks > 1) {
+        // this split's partial tile into the idle W_UV ring, [16 column
+        // groups][128 rows][4] fp32; the cluster reduction below reads it
+        float4* my = reinterpret_cast<float4*>(sA);
+#pragma unroll 1
+        for (int c = 0; c < 64; c += 16) {
+          float v[16];
+          tmem_ld16(trow + c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            my[((c >> 2) + g) * 128 + row] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+        }
+      } else if (!*abort_flag) {
         uint8_t* stage = sA;   // every MMA retired: the A tiles are free
 #pragma unroll 1
         for (int c = 0; c < 64; c += 16) {
@@ -227,6 +264,39 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
   }
   __syncwarp();
   __syncthreads();
+  if (ks > 1) {
+    // ---- split-K reduction across the cluster (every CTA takes both
+    // barriers, aborted or not, so none waits for a CTA that left)
+    cluster_sync();  // every partial tile is in its CTA's shared memory
+    if (warp >= 2 && warp < 6 && !*abort_flag) {
+      const int z = static_cast<int>(cluster_ctarank());
+      const int nr = 128 / ks, r0 = z * nr;
+      const int tid = threadIdx.x - 64;
+      uint8_t* stage = sB;  // every MMA retired: the B tiles are free
+      const uint32_t part = smem_u32(sA);
+      for (int u = tid; u < 16 * nr; u += 128) {
+        const int cg = u / nr, row = r0 + u % nr;
+        float4 p[kMaxKs];
+#pragma unroll
+        for (int q = 0; q < kMaxKs; ++q)
+          if (q < ks) p[q] = ld_shared_cluster_v4(mapa(part + (cg * 128 + row) * 16, static_cast<uint32_t>(q)));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < kMaxKs; ++q)
+          if (q < ks) {
+            acc.x += p[q].x;
+            acc.y += p[q].y;
+            acc.z += p[q].z;
+            acc.w += p[q].w;
+          }
+        const float vals[4] = {acc.x, acc.y, acc.z, acc.w};
+        epi_stage<4>(a.epi, nt * 64 + 4 * cg, a.N, vals, stage, 4 * cg, row);
+      }
+      named_bar_sync(1, 128);
+      epi_flush(a.epi, a.tok, 0, 128, nt * 64, 64, a.N, head, stage, tid, 128, a.status, r0, r0 + nr);
+    }
+    cluster_sync();  // no CTA reads another's shared memory any more
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 64);
