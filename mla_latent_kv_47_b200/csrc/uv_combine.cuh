@@ -150,9 +150,23 @@ __global__ void __launch_bounds__(uvc::kThreads, 1) uv_combine_kernel(const __gr
     if (n < a.N) {
       s0 = a.seg_start[n];
       s1 = a.seg_start[n + 1];
-      for (int s = s0; s < s1; ++s) M = fmaxf(M, a.ml_part[(static_cast<long long>(s) * a.n_h + head) * 2]);
+      // (m, l) of the first kMl pieces in registers, their loads in flight
+      // together; the rest (long sequences) from memory.  Same max, and the
+      // same sum in piece order, as one loop over the pieces.
+      constexpr int kMl = 8;
+      float2 ml[kMl];
+#pragma unroll
+      for (int j = 0; j < kMl; ++j)
+        ml[j] = s0 + j < s1 ? *reinterpret_cast<const float2*>(a.ml_part + (static_cast<long long>(s0 + j) * a.n_h + head) * 2)
+                            : make_float2(-INFINITY, 0.f);
+#pragma unroll
+      for (int j = 0; j < kMl; ++j) M = fmaxf(M, ml[j].x);
+      for (int s = s0 + kMl; s < s1; ++s) M = fmaxf(M, a.ml_part[(static_cast<long long>(s) * a.n_h + head) * 2]);
       float Ls = 0.f;
-      for (int s = s0; s < s1; ++s) {
+#pragma unroll
+      for (int j = 0; j < kMl; ++j)
+        if (s0 + j < s1) Ls += exp2f(ml[j].x - M) * ml[j].y;
+      for (int s = s0 + kMl; s < s1; ++s) {
         const long long i = (static_cast<long long>(s) * a.n_h + head) * 2;
         Ls += exp2f(a.ml_part[i] - M) * a.ml_part[i + 1];
       }
