@@ -36,7 +36,7 @@ def run_decode(m, preset, checked, lengths=None, pad=2, oracle="unabsorbed", dir
     callable of the sequence's length.  `chunk`: tokens per mla_cache_append
     call, with a workspace sized for them (the latent RMSNorm needs it)."""
     from mla_latent_kv_47_b200.cache import LatentCache
-    p = synth.preset(preset)
+    p = synth.preset(preset) if isinstance(preset, str) else preset
     d = p.dims if dims is None else dims
     dims = m.make_dims(d)
     L = list(lengths if lengths is not None else p.seqlen)
@@ -119,6 +119,21 @@ def test_lite_decode_all_sequences(m):
         gu.assert_gate(s)
     print("lite gate", max(s["max_rel"] for s in st.values()), max(s["mean_rel"] for s in st.values()),
           max(s["sum_rel"] for s in st.values()))
+
+
+@pytest.mark.parametrize("n_h", [8, 32])
+def test_other_head_counts(m, n_h):
+    """V2-Lite dims with 8 heads (the few-head attention kernel, its Q rows
+    past n_h zero; the combine split over 4 CTAs) and 32 heads (the 2-CTA
+    kernel with 96 empty head rows; the combine split over 2), on ragged
+    short lengths, every sequence checked."""
+    import dataclasses
+    d = dataclasses.replace(synth.V2_LITE, n_h=n_h)
+    L = (0, 1, 63, 65, 300, 1000)
+    p = synth.Preset(f"lite_h{n_h}", 2, d, len(L), L)
+    st = run_decode(m, p, checked=list(range(len(L))))
+    for s in st.values():
+        gu.assert_gate(s)
 
 
 def test_v2_decode_sampled(m):
