@@ -130,8 +130,11 @@ def _ptr(t):
 
 
 def make_weights(W: dict) -> Weights:
-    """Device weight tensors by name (the RMSNorm gains g_kv / g_q are optional)."""
-    return Weights(*[_ptr(W.get(n)) for n in WEIGHT_FIELDS])
+    """Device weight tensors by name (the RMSNorm gains g_kv / g_q are optional).
+    The returned struct holds the tensors, so their memory lives as long as it does."""
+    w = Weights(*[_ptr(W.get(n)) for n in WEIGHT_FIELDS])
+    w._tensors = [W.get(n) for n in WEIGHT_FIELDS]
+    return w
 
 
 def make_cache(base, seq_start=None, capacity=None, block_table=None, block_size=0) -> Cache:
@@ -142,9 +145,12 @@ def make_cache(base, seq_start=None, capacity=None, block_table=None, block_size
     assert capacity is None or capacity.dtype == torch.int32
     if block_table is not None:
         assert block_table.dtype == torch.int32 and block_table.dim() == 2
-        return Cache(_ptr(base), _ptr(seq_start), _ptr(capacity), int(base.shape[0]), _ptr(block_table),
-                     int(block_size), int(block_table.shape[1]))
-    return Cache(_ptr(base), _ptr(seq_start), _ptr(capacity), int(base.shape[0]), None, 0, 0)
+        c = Cache(_ptr(base), _ptr(seq_start), _ptr(capacity), int(base.shape[0]), _ptr(block_table),
+                  int(block_size), int(block_table.shape[1]))
+    else:
+        c = Cache(_ptr(base), _ptr(seq_start), _ptr(capacity), int(base.shape[0]), None, 0, 0)
+    c._tensors = (base, seq_start, capacity, block_table)  # the struct keeps the memory it points to alive
+    return c
 
 
 def _stream(stream):

@@ -213,3 +213,28 @@ def test_e4m3_cache_arguments_are_checked(m):
 def test_wait_timeout_check_needs_a_workspace(m):
     assert m.lib.mla_check_wait_timeout(None, None) == -4
     assert m.lib.mla_check_wait_timeout((1 << 20) + 16, None) == -3
+
+
+def test_structs_keep_their_tensors_alive(m, monkeypatch):
+    """make_weights / make_cache hand the library raw device pointers; the
+    structs they return hold the tensors, so a caller who drops its own
+    references (e.g. builds the weight dict inline) leaves no dangling pointer."""
+    import gc
+    import weakref
+
+    import torch
+
+    monkeypatch.setattr(m, "_ptr", lambda t: None if t is None else 4096)  # no device here
+    w_t = torch.zeros(4)
+    ref_w = weakref.ref(w_t)
+    w = m.make_weights({"W_O": w_t})
+    base = torch.zeros(2, 3)
+    ss = torch.zeros(1, dtype=torch.int64)
+    ref_b, ref_s = weakref.ref(base), weakref.ref(ss)
+    c = m.make_cache(base, seq_start=ss)
+    del w_t, base, ss
+    gc.collect()
+    assert ref_w() is not None and ref_b() is not None and ref_s() is not None
+    del w, c
+    gc.collect()
+    assert ref_w() is None and ref_b() is None and ref_s() is None
