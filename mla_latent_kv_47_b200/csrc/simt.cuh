@@ -154,9 +154,11 @@ struct Piece {
   int b, t0, t1, slot;
 };
 
-// Pieces of worker w, in order.  Calls f(piece) for each.
+// Pieces of worker w, in order.  Calls f(piece) for each.  Host-callable too
+// (the kernels pass device lambdas; a host check passes host ones).
+#pragma nv_exec_check_disable
 template <typename F>
-__device__ __forceinline__ void for_each_piece(int w, int W, int B, const int* tile_start, const int* seg_start, F&& f) {
+__host__ __device__ __forceinline__ void for_each_piece(int w, int W, int B, const int* tile_start, const int* seg_start, F&& f) {
   const long long T = tile_start[B];
   if (T <= 0) return;
   const int We = static_cast<int>(T < W ? T : W);
